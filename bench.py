@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse linear layer on B200.
+
+Default workload: the large LLM-MLP forward (X[8192,4096] bf16, W[14336,4096]
+in 64x64 blocks at density 0.1 with Zipf(1.1)-skewed block rows).  One step
+is one forward pass Y = X W^T of one batch through the C ABI (bsl_forward);
+the weight is packed once before timing, as the pages' layer fixes its
+sparsity pattern at initialisation (pytorch_block_sparse release note,
+"Future Development Roadmap": patterns are fixed at initialisation), and the
+pack is timed separately (``config.pack_ms``).
+
+Prints ONE JSON line (rank 0).  Multi-GPU (torchrun): every rank runs an
+independent replica of the workload (the layer is not sharded: replicas
+only), ``value`` is the sum over ranks of the work divided by the slowest
+rank's time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # fp64 CPU oracle on a bounded sample
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "block-sparse GEMM effective TFLOP/s, % roofline, speedup vs dense at 75/90% sparse"
+UNIT = "TFLOP/s"
+L2_BYTES_DEFAULT = 126 * 2 ** 20
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload.  The
+# entry is only used while the kernel source still hashes to `src_sha`.
+TRAFFIC = {}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def src_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "sparse_gemm_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def algorithmic(w: synth.Workload, nnz: int):
+    """Flops and HBM bytes per launch of each contraction (minimum traffic:
+    every operand read once, every output written once)."""
+    b, M, N, K = w.b, w.M, w.N, w.K
+    R, C = N // b, K // b
+    flops = 2 * M * b * b * nnz
+    wbytes = nnz * b * b * 2 + (R + 1 + nnz) * 4           # values + BSR index
+    wbytes_t = nnz * b * b * 2 + (C + 1 + 2 * nnz) * 4     # values + CSC index + map
+    return {
+        "fwd": {"flops": flops, "bytes": M * K * 2 + wbytes + M * N * 2},
+        "dx": {"flops": flops, "bytes": M * N * 2 + wbytes_t + M * K * 2},
+        "dw": {"flops": flops, "bytes": M * N * 2 + M * K * 2 + nnz * b * b * 2 + (C + 1 + 2 * nnz) * 4},
+    }
+
+
+def roofline_entry(kind: str, alg: dict, dur_ms: float, pk: dict, burst: bool = True):
+    tc_peak = pk["bf16_tflops"] if burst else pk["bf16_tflops_sustained"]
+    t_tc = alg["flops"] / (tc_peak * 1e12)
+    t_hbm = alg["bytes"] / (pk["hbm_gbs"] * 1e9)
+    s = dur_ms * 1e-3
+    if t_tc >= t_hbm:
+        achieved = alg["flops"] / s / 1e12
+        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4)}
+    achieved = alg["bytes"] / s / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4)}
+
+
+def cpu_sample(w: synth.Workload, inp: dict, budget_s: float, kinds: list[str]):
+    """Time the fp64 oracle, as it is, on a bounded sample of the workload.
+
+    Forward / dX: a sample of token rows (all N or K outputs of each);
+    dW: a sample of stored blocks (each reduced over all M rows).  The
+    operands are widened and the dense-with-zeros weight is built once,
+    outside the timed calls.  Returns (flops_done, seconds, description).
+    """
+    import oracle
+    oracle.build()
+    b = w.b
+    Xd = oracle.widen(inp["X"])
+    Wt = oracle.dense_weight(inp["W"], inp["mask"], b)
+    dYd = oracle.widen(inp["dY"]) if "dY" in inp else None
+    nthreads = oracle.num_threads()
+    per_row = 2 * w.N * w.K                       # dense-with-zeros flops per token row
+    eff_ratio = w.nnz / (w.R * w.C)
+    done_eff, secs, desc = 0.0, 0.0, []
+    share = budget_s / len(kinds)
+    for kind in kinds:
+        if kind in ("fwd", "dx"):
+            def call(rows):
+                if kind == "fwd":
+                    oracle.forward(None, None, None, b, rows=rows, Xd=Xd, Wt=Wt)
+                else:
+                    oracle.backward_input(None, None, None, b, rows=rows, dYd=dYd, Wt=Wt)
+            t0 = time.perf_counter()
+            call(np.arange(min(nthreads, w.M)))
+            t1 = time.perf_counter() - t0
+            n = int(min(w.M, max(1, share / max(t1, 1e-6)) * min(nthreads, w.M)))
+            n = max(1, min(n, w.M))
+            rows = np.random.default_rng(0).choice(w.M, size=n, replace=False)
+            t0 = time.perf_counter()
+            call(rows)
+            dt = time.perf_counter() - t0
+            done_eff += 2 * n * w.N * w.K * eff_ratio
+            secs += dt
+            desc.append(f"{kind}: {n} of {w.M} token rows")
+        else:
+            rr, cc = np.nonzero(inp["mask"])
+            t0 = time.perf_counter()
+            oracle.backward_weight(None, None, inp["mask"], b, blocks=[(int(rr[0]), int(cc[0]))],
+                                   dYd=dYd, Xd=Xd)
+            t1 = time.perf_counter() - t0
+            n = int(max(1, min(len(rr), share / max(t1, 1e-6))))
+            pick = np.random.default_rng(0).choice(len(rr), size=n, replace=False)
+            t0 = time.perf_counter()
+            oracle.backward_weight(None, None, inp["mask"], b,
+                                   blocks=[(int(rr[i]), int(cc[i])) for i in pick], dYd=dYd, Xd=Xd)
+            dt = time.perf_counter() - t0
+            done_eff += 2 * n * b * b * w.M
+            secs += dt
+            desc.append(f"dw: {n} of {len(rr)} blocks")
+    del per_row
+    return done_eff, secs, "; ".join(desc), nthreads
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_gemm_b200 as sg
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    from sparse_gemm_b200 import build as _b
+    _b.build()
+
+    w = synth.WORKLOADS[args.workload]
+    train = w.with_dy
+    inp = synth.make_inputs(w)
+    pk = peaks()
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", L2_BYTES_DEFAULT) or L2_BYTES_DEFAULT
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    Wd = dev_bf16(inp["W"])
+    mask = torch.from_numpy(inp["mask"]).to(dev)
+    X0 = dev_bf16(inp["X"])
+    dY0 = dev_bf16(inp["dY"]) if train else None
+
+    # pack (timed separately: once per weight)
+    stream = torch.cuda.current_stream(dev)
+    Wp = sg.pack(Wd, mask, w.b, nnz=w.nnz)
+    torch.cuda.synchronize()
+    pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pack_ms = []
+    for _ in range(5):
+        pe0.record(stream)
+        sg.pack(Wd, mask, w.b, nnz=w.nnz)
+        pe1.record(stream)
+        torch.cuda.synchronize()
+        pack_ms.append(pe0.elapsed_time(pe1))
+    if sg.device_status(Wp) != 0:
+        raise RuntimeError("pack reported a device error")
+
+    # L2-cold protocol: rotate through copies of every input so that one
+    # rotation touches more than 2x L2 before an input is reused
+    in_bytes = X0.numel() * 2 + (dY0.numel() * 2 if train else 0) + w.nnz * w.b * w.b * 2
+    ncopy = int(min(16, max(2, math.ceil(2 * l2 / in_bytes) + 1)))
+    Xs = [X0] + [X0.clone() for _ in range(ncopy - 1)]
+    dYs = ([dY0] + [dY0.clone() for _ in range(ncopy - 1)]) if train else None
+    Wps = [Wp] + [sg.pack(Wd, mask, w.b, nnz=w.nnz) for _ in range(ncopy - 1)]
+    Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((w.M, w.K), dtype=torch.bfloat16, device=dev) if train else None
+    dWv = torch.empty((w.nnz, w.b, w.b), dtype=torch.bfloat16, device=dev) if train else None
+    ws = torch.empty(max(16, sg.forward_workspace_bytes(w.M, Wp)), dtype=torch.uint8, device=dev)
+    small = w.M <= sg.small_m_max()
+
+    kinds = ["fwd", "dx", "dw"] if train else ["fwd"]
+    launches_per_step = (2 if small else 1) + (2 if train else 0)
+
+    def step(i, evs=None):
+        j = i % ncopy
+        if evs is not None:
+            evs[0].record(stream)
+        sg.forward(Xs[j], Wps[j], out=Y, workspace=ws)
+        if train:
+            if evs is not None:
+                evs[1].record(stream)
+            sg.backward_input(dYs[j], Wps[j], out=dX)
+            if evs is not None:
+                evs[2].record(stream)
+            sg.backward_weight(dYs[j], Xs[j], Wps[j], out=dWv)
+        if evs is not None:
+            evs[-1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if sg.device_status(Wp) != 0:
+        raise RuntimeError("kernels reported a device error")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(kinds) + 1)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    per_kernel = {k: statistics.mean(e[n].elapsed_time(e[n + 1]) for e in evs) for n, k in enumerate(kinds)}
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    alg = algorithmic(w, w.nnz)
+    flops_step = sum(alg[k]["flops"] for k in kinds)
+    value = world * flops_step * K / (total_ms * 1e-3) / 1e12
+    ms_per_step = total_ms / K
+
+    # dominant kernel + its roofline
+    dom = max(per_kernel, key=per_kernel.get)
+    roof = roofline_entry(dom, alg[dom], per_kernel[dom], pk)
+    roof["kernel"] = {"fwd": "k_stream_fwd+k_stream_fixup" if small else "k_spmm_tc (forward)",
+                      "dx": "k_spmm_tc (input gradient)", "dw": "k_sddmm_tc"}[dom]
+    roof["peak_source"] = pk["source"] + (" burst bf16" if roof["unit"] == "TFLOP/s" else " HBM copy")
+    tr = TRAFFIC.get((w.name, dom))
+    roof["traffic"] = tr["bytes"] if tr and tr.get("src_sha") == src_sha(*tr["files"]) else None
+    roof["algorithmic_bytes"] = alg[dom]["bytes"]
+    roof["algorithmic_flops"] = alg[dom]["flops"]
+    roof["tensor_frac_of_sustained"] = round(alg[dom]["flops"] / (per_kernel[dom] * 1e-3) / 1e12
+                                             / pk["bf16_tflops_sustained"], 4)
+
+    # cuBLAS dense of the same shapes (zeros in place), same rotation
+    Wdz = Wd * torch.repeat_interleave(torch.repeat_interleave(mask.to(torch.bfloat16), w.b, 0), w.b, 1)
+    Wdzs = [Wdz] + [Wdz.clone() for _ in range(min(ncopy, 4) - 1)]
+
+    def dense_step(i):
+        j = i % len(Wdzs)
+        x = Xs[i % ncopy]
+        torch.matmul(x, Wdzs[j].t(), out=Y)
+        if train:
+            torch.matmul(dYs[i % ncopy], Wdzs[j], out=dX)
+            torch.matmul(dYs[i % ncopy].t(), x)
+
+    for i in range(max(3, args.warmup)):
+        dense_step(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(K):
+        dense_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = e0.elapsed_time(e1) / K
+
+    # end to end through the public API: pinned host X (+dY) in, Y (+dX, dW) out
+    hX = torch.empty(X0.shape, dtype=torch.bfloat16, pin_memory=True).copy_(X0.cpu())
+    hdY = torch.empty(dY0.shape, dtype=torch.bfloat16, pin_memory=True).copy_(dY0.cpu()) if train else None
+    hY = torch.empty(Y.shape, dtype=torch.bfloat16, pin_memory=True)
+    hdX = torch.empty(dX.shape, dtype=torch.bfloat16, pin_memory=True) if train else None
+    hdW = torch.empty(dWv.shape, dtype=torch.bfloat16, pin_memory=True) if train else None
+    dXin = torch.empty_like(X0)
+    dYin = torch.empty_like(dY0) if train else None
+
+    def e2e_step():
+        dXin.copy_(hX, non_blocking=True)
+        if train:
+            dYin.copy_(hdY, non_blocking=True)
+        sg.forward(dXin, Wp, out=Y, workspace=ws)
+        hY.copy_(Y, non_blocking=True)
+        if train:
+            sg.backward_input(dYin, Wp, out=dX)
+            sg.backward_weight(dYin, dXin, Wp, out=dWv)
+            hdX.copy_(dX, non_blocking=True)
+            hdW.copy_(dWv, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ke = max(3, min(K, 50))
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / ke
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = X0.numel() * 2 + (dY0.numel() * 2 if train else 0)
+    d2h = Y.numel() * 2 + ((dX.numel() + dWv.numel()) * 2 if train else 0)
+
+    if sg.device_status(Wp) != 0:
+        raise RuntimeError("kernels reported a device error")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        done, secs, desc, nthr = cpu_sample(w, inp, args.cpu_budget, kinds)
+        cpu = {"value": round(done / secs / 1e12, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
+               "sample": desc + f" ({secs:.1f} s, fp64 dense-with-zeros loops)"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": w.name, "M": w.M, "N": w.N, "K": w.K, "b": w.b, "nnz": w.nnz,
+            "density": round(w.nnz / (w.R * w.C), 5), "mask": w.mask_kind, "seed": w.seed,
+            "contractions_per_step": kinds, "global_batch": w.M * world,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"rotating {ncopy} copies of every input ({ncopy * in_bytes / 2**20:.0f} MiB > 2x L2)",
+            "pack_ms": round(statistics.median(pack_ms), 4),
+        },
+        "kernels_ms": {k: round(v, 5) for k, v in per_kernel.items()},
+        "roofline": roof,
+        "dense_cublas_ms_per_step": round(dense_ms, 5),
+        "speedup_vs_dense": round(dense_ms / ms_per_step, 3),
+        "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    return out
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: each step is a bounded
+    sample of the workload; value is effective TFLOP/s over the sample."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    w = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(w)
+    kinds = ["fwd", "dx", "dw"] if w.with_dy else ["fwd"]
+    per_step = max(0.5, min(20.0, args.reference_budget / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_sample(w, inp, per_step, kinds)
+    done, secs, descs = 0.0, 0.0, []
+    nthr = 1
+    for _ in range(args.steps):
+        d, s, desc, nthr = cpu_sample(w, inp, per_step, kinds)
+        done += d
+        secs += s
+        descs.append(desc)
+    value = done / secs / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 8), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "b": w.b, "nnz": w.nnz,
+                   "density": round(w.nnz / (w.R * w.C), 5), "mask": w.mask_kind, "seed": w.seed},
+        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
+                         "sample": descs[0] + " per step"},
+        "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="large_fwd", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
+    ap.add_argument("--reference-budget", type=float, default=120.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    out = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * bsl.h -- C ABI of libbsl, the B200 (sm_100a) block-sparse linear layer.
+ *
+ * The layer is Hugging Face pytorch_block_sparse's BlockSparseLinear
+ * (release note, "Block-Sparse Implementation and Usage"): a weight W[N,K]
+ * that keeps only its nonzero b x b blocks, multiplied with dense
+ * activations.  The library computes, in bf16 with fp32 accumulation:
+ *
+ *   forward          Y  = X  . W~^T      X [M,K] -> Y [M,N]
+ *   input gradient   dX = dY . W~        dY[M,N] -> dX[M,K]
+ *   weight gradient  dW = dY^T . X, only at the stored blocks
+ *
+ * where W~ is W with zeros outside the block mask.  The pruned weight is
+ * handed over as a dense tensor with zeros in place plus a block mask, and
+ * the sparse product equals the dense product with that tensor (torchao
+ * sparsity README, introduction).  The stored form is BSR: data blocks plus
+ * the block row pointer / column index arrays (torchao README, Table 4.1,
+ * BSR and CSR rows), with a transposed (CSC) index over the same blocks
+ * (Table 4.1, CSC row).  The masked weight gradient is dW (.) Mask
+ * (torchao README, "Pruning Criteria", out-of-place mask updates).
+ *
+ * Conventions for every entry point:
+ *  - All pointers are DEVICE pointers owned by the caller, unless a
+ *    parameter says "host".  The library never frees caller memory and
+ *    allocates nothing.
+ *  - Matrices are row-major and contiguous (row stride = number of
+ *    columns); bf16 is IEEE bfloat16 (2 bytes), passed as void *.
+ *  - Every pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    asynchronous on it unless stated otherwise.
+ *  - Arguments are checked on the host before any launch; a failed check
+ *    returns a status and launches nothing.  Launch failures return
+ *    BSL_ERR_CUDA.  Problems found on the device (a wait that ran out, a
+ *    packed size that does not match the mask) are written to the device
+ *    status word of the bsl_bsr (first error wins); read it with
+ *    bsl_get_device_status.
+ *  - Outputs are overwritten, never accumulated into.
+ *  - Block size b must be 32 or 64; N and K must be multiples of b.
+ */
+#ifndef BSL_H_
+#define BSL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSL_API __attribute__((visibility("default")))
+#else
+#define BSL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BSL_OK = 0,
+    BSL_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misalignment */
+    BSL_ERR_UNSUPPORTED = 2,   /* block size or size outside what is built */
+    BSL_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed */
+    BSL_ERR_TIMEOUT = 4,       /* a device-side wait ran out of time (device status) */
+    BSL_ERR_NNZ_MISMATCH = 5,  /* mask block count != bsl_bsr.nnz (device status) */
+    BSL_ERR_NO_DEVICE = 6      /* no sm_100 device current */
+} bsl_status;
+
+/* Packed block-sparse weight.  The caller allocates every array (device
+ * memory) with the sizes below, R = N/b, C = K/b; bsl_pack fills them. */
+typedef struct {
+    int32_t N, K, b, nnz;
+    int32_t *row_ptr;     /* [R+1] BSR row pointer: blocks of block row r are row_ptr[r]..row_ptr[r+1]-1 */
+    int32_t *col_idx;     /* [nnz] block column of each block, ascending inside a row */
+    void *values;         /* bf16 [nnz][b][b]; block p row-major, in BSR order */
+    int32_t *col_ptr;     /* [C+1] CSC column pointer over the same blocks */
+    int32_t *row_idx;     /* [nnz] block row of each CSC entry, ascending inside a column */
+    int32_t *csc_to_bsr;  /* [nnz] BSR position of each CSC entry (values are not duplicated) */
+    int32_t *row_order;   /* [R] block rows by block count, largest first, ties lower id first */
+    int32_t *col_order;   /* [C] block columns, same order rule */
+    int32_t *dw_gptr;     /* [C+1] prefix over columns of ceil(col_count / (128/b)) (weight-gradient groups) */
+    int32_t *status;      /* [1] device status word; must be zeroed once at allocation */
+} bsl_bsr;
+
+/* Human-readable name of a status code (static string). */
+BSL_API const char *bsl_status_string(bsl_status s);
+
+/* Description of the last CUDA error this host thread saw inside the
+ * library (the cause behind a BSL_ERR_CUDA), or "none".  The string lives in
+ * thread-local storage until the next call from the same thread. */
+BSL_API const char *bsl_last_cuda_error(void);
+
+/* Count the mask's blocks.  mask: uint8 [R][C], nonzero = block kept.
+ * row_ptr: int32 [R+1] device scratch that receives the BSR row pointer.
+ * nnz_host: HOST int32 that receives the count.  SYNCHRONOUS: waits for the
+ * stream, so the caller can size the packed arrays before bsl_pack. */
+BSL_API bsl_status bsl_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *row_ptr,
+                          int32_t *nnz_host, void *stream);
+
+/* Build the packed weight from a dense bf16 W [N][K] (zeros in place or
+ * not: entries outside the mask are dropped) and a uint8 mask [N/b][K/b].
+ * Fills every array of *out (N, K, b, nnz and the pointers set by the
+ * caller).  If the mask holds a different number of blocks than out->nnz,
+ * the device status becomes BSL_ERR_NNZ_MISMATCH and no array is written
+ * past its size.  A masked-in block is stored even if all its values are 0. */
+BSL_API bsl_status bsl_pack(const void *W, const uint8_t *mask, const bsl_bsr *out, void *stream);
+
+/* Y [M][N] = X [M][K] . W~^T.  Picks the weight-streaming kernel for
+ * M <= bsl_small_m_max() and the tensor-core kernel otherwise.  workspace:
+ * device scratch of bsl_forward_workspace_bytes(M, W) bytes (may be NULL
+ * when that size is 0). */
+BSL_API bsl_status bsl_forward(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/* Largest M routed to the weight-streaming kernel by bsl_forward. */
+BSL_API int32_t bsl_small_m_max(void);
+
+/* Scratch bytes bsl_forward needs for this M (0 for the tensor-core path). */
+BSL_API size_t bsl_forward_workspace_bytes(int32_t M, const bsl_bsr *W);
+
+/* Tensor-core forward for any M >= 1 (persistent tcgen05 kernel; TMA
+ * loads of X tiles and weight blocks, fp32 accumulators in TMEM). */
+BSL_API bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *stream);
+
+/* Weight-streaming forward ("load and sparse expand", lecture summary at
+ * 48:12) for 1 <= M <= bsl_small_m_max(): each warp streams a contiguous,
+ * equal share of the packed blocks once; block rows split between warps
+ * are summed in a fixed order.  workspace: bsl_forward_workspace_bytes(M, W)
+ * bytes; contents on entry do not matter. */
+BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, void *Y,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* dX [M][K] = dY [M][N] . W~ (tensor-core kernel over the CSC index). */
+BSL_API bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *W, void *dX, void *stream);
+
+/* dW_values [nnz][b][b] = blocks of dY^T . X at the stored blocks, in BSR
+ * order (sampled dense-dense product over M; tensor-core kernel). */
+BSL_API bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const bsl_bsr *W,
+                               void *dW_values, void *stream);
+
+/* SYNCHRONOUS: waits for the stream, copies the device status word of W to
+ * *status_host (a bsl_status value) and resets it to BSL_OK. */
+BSL_API bsl_status bsl_get_device_status(const bsl_bsr *W, int32_t *status_host, void *stream);
+
+/* Upper bound, in microseconds, on any device-side wait of the kernels
+ * launched after this call (default 2,000,000, or BSL_WAIT_TIMEOUT_US from
+ * the environment at first use).  A wait that runs out sets
+ * BSL_ERR_TIMEOUT in the device status and the kernel returns. */
+BSL_API void bsl_set_wait_timeout_us(uint64_t timeout_us);
+
+/* Test hook for the bounded waits: launches one block that waits on a
+ * barrier nothing arrives at, for at most timeout_us, then writes
+ * BSL_ERR_TIMEOUT to *status (device int32, zeroed by the caller). */
+BSL_API bsl_status bsl_debug_wait_timeout(int32_t *status, uint64_t timeout_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSL_H_ */

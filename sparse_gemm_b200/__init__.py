@@ -1,0 +1,297 @@
+"""sparse_gemm_b200 -- block-sparse linear layer on B200 (sm_100a).
+
+Thin ctypes binding over ``libbsl.so`` (C ABI in ``include/bsl.h``).  The
+binding only marshals arguments: it checks dtypes and shapes, allocates
+outputs with torch on the tensors' device and passes raw pointers plus the
+current CUDA stream.  Every step of the computation runs in the library's
+CUDA kernels; there is no fallback.  If the library is missing or the
+device is not an sm_100 GPU the calls raise.
+
+Layer (Hugging Face pytorch_block_sparse release note, "Block-Sparse
+Implementation and Usage"): a linear layer whose weight W[N, K] keeps only
+its nonzero b x b blocks.  Forward Y = X W^T, input gradient dX = dY W,
+weight gradient dW = dY^T X at the kept blocks only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "BslError", "BsrWeight", "library", "count_blocks", "pack", "forward", "forward_tc",
+    "forward_stream", "forward_workspace_bytes", "backward_input", "backward_weight",
+    "device_status", "set_wait_timeout_us", "debug_wait_timeout", "small_m_max",
+    "BlockSparseLinearFunction",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsl.so")
+
+STATUS_NAMES = {
+    0: "BSL_OK", 1: "BSL_ERR_INVALID_ARG", 2: "BSL_ERR_UNSUPPORTED", 3: "BSL_ERR_CUDA",
+    4: "BSL_ERR_TIMEOUT", 5: "BSL_ERR_NNZ_MISMATCH", 6: "BSL_ERR_NO_DEVICE",
+}
+
+
+class BslError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)}")
+
+
+class _BSR(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("b", ctypes.c_int32),
+                ("nnz", ctypes.c_int32)] + [
+        (name, ctypes.c_void_p) for name in
+        ("row_ptr", "col_idx", "values", "col_ptr", "row_idx", "csc_to_bsr", "row_order",
+         "col_order", "dw_gptr", "status")]
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libbsl.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m sparse_gemm_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I32, SZ, U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64
+        BP = ctypes.POINTER(_BSR)
+        sig = {
+            "bsl_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "bsl_last_cuda_error": (ctypes.c_char_p, []),
+            "bsl_pack_count": (ctypes.c_int, [P, I32, I32, P, ctypes.POINTER(I32), P]),
+            "bsl_pack": (ctypes.c_int, [P, P, BP, P]),
+            "bsl_forward": (ctypes.c_int, [P, I32, BP, P, P, SZ, P]),
+            "bsl_small_m_max": (I32, []),
+            "bsl_forward_workspace_bytes": (SZ, [I32, BP]),
+            "bsl_forward_tc": (ctypes.c_int, [P, I32, BP, P, P]),
+            "bsl_forward_stream": (ctypes.c_int, [P, I32, BP, P, P, SZ, P]),
+            "bsl_backward_input": (ctypes.c_int, [P, I32, BP, P, P]),
+            "bsl_backward_weight": (ctypes.c_int, [P, P, I32, BP, P, P]),
+            "bsl_get_device_status": (ctypes.c_int, [BP, ctypes.POINTER(I32), P]),
+            "bsl_set_wait_timeout_us": (None, [U64]),
+            "bsl_debug_wait_timeout": (ctypes.c_int, [P, U64, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        detail = library().bsl_last_cuda_error().decode() if st == 3 else ""
+        raise BslError(st, f"{where} [{detail}]" if detail else where)
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _cuda_bf16_2d(t: torch.Tensor, name: str, cols: int | None = None):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 2):
+        raise TypeError(f"{name} must be a 2-D bfloat16 CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+    if cols is not None and t.shape[1] != cols:
+        raise ValueError(f"{name} has {t.shape[1]} columns, expected {cols}")
+
+
+class BsrWeight:
+    """Packed block-sparse weight: device tensors of the bsl_bsr struct."""
+
+    def __init__(self, N: int, K: int, b: int, nnz: int, device):
+        if b not in (32, 64) or N % b or K % b:
+            raise ValueError("b must be 32 or 64 and divide N and K")
+        self.N, self.K, self.b, self.nnz = int(N), int(K), int(b), int(nnz)
+        R, C = N // b, K // b
+        i32 = dict(dtype=torch.int32, device=device)
+        self.row_ptr = torch.empty(R + 1, **i32)
+        self.col_idx = torch.empty(max(nnz, 1), **i32)
+        self.values = torch.empty((max(nnz, 1), b, b), dtype=torch.bfloat16, device=device)
+        self.col_ptr = torch.empty(C + 1, **i32)
+        self.row_idx = torch.empty(max(nnz, 1), **i32)
+        self.csc_to_bsr = torch.empty(max(nnz, 1), **i32)
+        self.row_order = torch.empty(R, **i32)
+        self.col_order = torch.empty(C, **i32)
+        self.dw_gptr = torch.empty(C + 1, **i32)
+        self.status = torch.zeros(1, **i32)
+        self._c = _BSR(self.N, self.K, self.b, self.nnz,
+                       *[t.data_ptr() for t in (self.row_ptr, self.col_idx, self.values, self.col_ptr,
+                                                self.row_idx, self.csc_to_bsr, self.row_order,
+                                                self.col_order, self.dw_gptr, self.status)])
+
+    @property
+    def R(self):
+        return self.N // self.b
+
+    @property
+    def C(self):
+        return self.K // self.b
+
+    @property
+    def device(self):
+        return self.values.device
+
+    def block_values(self) -> torch.Tensor:
+        """Packed values [nnz, b, b] (empty view when nnz == 0)."""
+        return self.values[: self.nnz]
+
+    def cref(self):
+        return ctypes.byref(self._c)
+
+
+def _mask_u8(mask: torch.Tensor, R: int, C: int) -> torch.Tensor:
+    if not (mask.is_cuda and mask.dim() == 2 and tuple(mask.shape) == (R, C)):
+        raise ValueError(f"mask must be a CUDA tensor of shape ({R}, {C})")
+    return mask.to(torch.uint8).contiguous()
+
+
+def count_blocks(mask: torch.Tensor) -> int:
+    """Number of kept blocks in a [R, C] block mask (synchronises the stream)."""
+    R, C = mask.shape
+    m = _mask_u8(mask, R, C)
+    tmp = torch.empty(R + 1, dtype=torch.int32, device=m.device)
+    out = ctypes.c_int32(0)
+    _check(library().bsl_pack_count(m.data_ptr(), R, C, tmp.data_ptr(), ctypes.byref(out), _stream(m)),
+           "bsl_pack_count")
+    return int(out.value)
+
+
+def pack(W: torch.Tensor, mask: torch.Tensor, b: int, nnz: int | None = None) -> BsrWeight:
+    """Pack a dense bf16 weight [N, K] with a block mask [N/b, K/b] (kept = nonzero)."""
+    _cuda_bf16_2d(W, "W")
+    N, K = W.shape
+    m = _mask_u8(mask, N // b, K // b)
+    if nnz is None:
+        nnz = count_blocks(m)
+    Wp = BsrWeight(N, K, b, nnz, W.device)
+    _check(library().bsl_pack(W.data_ptr(), m.data_ptr(), Wp.cref(), _stream(W)), "bsl_pack")
+    Wp._mask = m  # keep the mask alive until the stream has consumed it
+    return Wp
+
+
+def small_m_max() -> int:
+    return int(library().bsl_small_m_max())
+
+
+def forward_workspace_bytes(M: int, Wp: BsrWeight) -> int:
+    return int(library().bsl_forward_workspace_bytes(M, Wp.cref()))
+
+
+def _out(M, cols, like):
+    return torch.empty((M, cols), dtype=torch.bfloat16, device=like.device)
+
+
+def forward(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None,
+            workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T, kernel chosen by M (weight streaming for M <= small_m_max())."""
+    _cuda_bf16_2d(X, "X", Wp.K)
+    M = X.shape[0]
+    Y = _out(M, Wp.N, X) if out is None else out
+    nbytes = forward_workspace_bytes(M, Wp)
+    if nbytes and workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
+    wptr = workspace.data_ptr() if workspace is not None else None
+    wlen = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(library().bsl_forward(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), wptr, wlen, _stream(X)),
+           "bsl_forward")
+    return Y
+
+
+def forward_tc(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T on the tensor-core kernel (any M)."""
+    _cuda_bf16_2d(X, "X", Wp.K)
+    M = X.shape[0]
+    Y = _out(M, Wp.N, X) if out is None else out
+    _check(library().bsl_forward_tc(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), _stream(X)), "bsl_forward_tc")
+    return Y
+
+
+def forward_stream(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T on the weight-streaming kernel (M <= small_m_max())."""
+    _cuda_bf16_2d(X, "X", Wp.K)
+    M = X.shape[0]
+    Y = _out(M, Wp.N, X) if out is None else out
+    nbytes = forward_workspace_bytes(M, Wp)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=X.device)
+    _check(library().bsl_forward_stream(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(), _stream(X)),
+           "bsl_forward_stream")
+    return Y
+
+
+def backward_input(dY: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """dX = dY W (tensor-core kernel over the CSC index)."""
+    _cuda_bf16_2d(dY, "dY", Wp.N)
+    M = dY.shape[0]
+    dX = _out(M, Wp.K, dY) if out is None else out
+    _check(library().bsl_backward_input(dY.data_ptr(), M, Wp.cref(), dX.data_ptr(), _stream(dY)),
+           "bsl_backward_input")
+    return dX
+
+
+def backward_weight(dY: torch.Tensor, X: torch.Tensor, Wp: BsrWeight,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """dW at the kept blocks, [nnz, b, b] in BSR order."""
+    _cuda_bf16_2d(dY, "dY", Wp.N)
+    _cuda_bf16_2d(X, "X", Wp.K)
+    if dY.shape[0] != X.shape[0]:
+        raise ValueError("dY and X must have the same number of rows")
+    dW = torch.empty((max(Wp.nnz, 1), Wp.b, Wp.b), dtype=torch.bfloat16, device=X.device) \
+        if out is None else out
+    _check(library().bsl_backward_weight(dY.data_ptr(), X.data_ptr(), X.shape[0], Wp.cref(),
+                                         dW.data_ptr(), _stream(X)), "bsl_backward_weight")
+    return dW[: Wp.nnz]
+
+
+def device_status(Wp: BsrWeight) -> int:
+    """Read and clear the device status word (synchronises the stream)."""
+    out = ctypes.c_int32(0)
+    _check(library().bsl_get_device_status(Wp.cref(), ctypes.byref(out), _stream(Wp.values)),
+           "bsl_get_device_status")
+    return int(out.value)
+
+
+def set_wait_timeout_us(us: int) -> None:
+    library().bsl_set_wait_timeout_us(int(us))
+
+
+def debug_wait_timeout(status: torch.Tensor, us: int) -> None:
+    """Run the bounded-wait test kernel; it writes BSL_ERR_TIMEOUT (4) to status[0]."""
+    if not (status.is_cuda and status.dtype == torch.int32):
+        raise TypeError("status must be an int32 CUDA tensor")
+    _check(library().bsl_debug_wait_timeout(status.data_ptr(), int(us), _stream(status)),
+           "bsl_debug_wait_timeout")
+
+
+class BlockSparseLinearFunction(torch.autograd.Function):
+    """Autograd wrapper: forward Y = X W^T; backward dX and dW at kept blocks.
+
+    ``values`` is the packed weight's value tensor (the parameter being
+    trained); its gradient is returned in the same [nnz, b, b] layout.
+    """
+
+    @staticmethod
+    def forward(ctx, X, values, Wp):
+        ctx.save_for_backward(X)
+        ctx.Wp = Wp
+        return forward(X.contiguous(), Wp)
+
+    @staticmethod
+    def backward(ctx, dY):
+        (X,) = ctx.saved_tensors
+        Wp = ctx.Wp
+        dY = dY.contiguous()
+        dX = backward_input(dY, Wp) if ctx.needs_input_grad[0] else None
+        dW = backward_weight(dY, X.contiguous(), Wp) if ctx.needs_input_grad[1] else None
+        return dX, dW, None

@@ -1,0 +1,251 @@
+// pack.cu -- dense weight + block mask -> packed block-sparse weight.
+//
+// Stored form (torchao sparsity README, Table 4.1, BSR and CSR/CSC rows):
+// the kept b x b blocks as data, a block-row pointer and block-column index
+// (BSR), and the transposed index over the same blocks (CSC) with a map from
+// each CSC entry to its BSR block, so the values exist once.  The input is
+// the hand-off form of the torchao README introduction: a dense weight with
+// zeros in place, here with an explicit block mask.  Everything is integer
+// or bit-copy work and deterministic: no atomics decide any output order.
+//
+// Kernels, in launch order:
+//   k_counts     one warp per block row / block column: popcount of the mask
+//   k_scan       one CTA: exclusive scans -> row_ptr, col_ptr, dw_gptr; nnz check
+//   k_fill_rows  one warp per block row: col_idx (ascending) by ballot prefix
+//   k_fill_cols  one warp per block column: row_idx, csc_to_bsr
+//   k_gather     16-byte vector copy of every kept block into `values`
+//   k_order      rank of each row / column in the longest-first order
+#include "common.cuh"
+#include "internal.h"
+
+namespace bsl {
+namespace {
+
+constexpr int kWarps = 8;  // warps per CTA in the per-row / per-column kernels
+
+// counts[0..R) -> row_ptr[1..R], counts of columns -> col_ptr[1..C]
+__global__ void k_counts(const uint8_t *__restrict__ mask, int32_t R, int32_t C, int32_t *__restrict__ row_ptr,
+                         int32_t *__restrict__ col_ptr)
+{
+    const int lane = threadIdx.x & 31;
+    const int w = blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (w < R) {
+        const uint8_t *row = mask + static_cast<int64_t>(w) * C;
+        int cnt = 0;
+        for (int c = lane; c < C; c += 32) cnt += row[c] != 0;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0) row_ptr[w + 1] = cnt;
+    } else if (col_ptr && w < R + C) {
+        const int c = w - R;
+        int cnt = 0;
+        for (int r = lane; r < R; r += 32) cnt += mask[static_cast<int64_t>(r) * C + c] != 0;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0) col_ptr[c + 1] = cnt;
+    }
+}
+
+// Block-wide inclusive scan helper over 1024 threads.
+__device__ int block_scan_incl(int v, int *sm)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    if (lane == 31) sm[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        int s = (lane < (int)(blockDim.x >> 5)) ? sm[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int t = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += t;
+        }
+        sm[lane] = s;
+    }
+    __syncthreads();
+    if (wid > 0) v += sm[wid - 1];
+    __syncthreads();
+    return v;
+}
+
+// In-place: ptr[1..n] holds counts; turns ptr[0..n] into the exclusive prefix.
+// If `groups` is set, also writes groups[0..n] = prefix of ceil(count/G).
+__device__ void scan_counts(int32_t *ptr, int32_t n, int32_t *groups, int G, int *sm)
+{
+    int carry = 0, gcarry = 0;
+    if (threadIdx.x == 0) {
+        ptr[0] = 0;
+        if (groups) groups[0] = 0;
+    }
+    for (int base = 0; base < n; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int cnt = i < n ? ptr[i + 1] : 0;
+        const int incl = block_scan_incl(cnt, sm) + carry;
+        int gincl = 0;
+        if (groups) gincl = block_scan_incl((cnt + G - 1) / G, sm) + gcarry;
+        if (i < n) {
+            ptr[i + 1] = incl;
+            if (groups) groups[i + 1] = gincl;
+        }
+        // the last thread of the chunk holds the running totals
+        __shared__ int tot[2];
+        if (threadIdx.x == blockDim.x - 1) {
+            tot[0] = incl;
+            tot[1] = gincl;
+        }
+        __syncthreads();
+        carry = tot[0];
+        gcarry = tot[1];
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(1024) k_scan(int32_t *row_ptr, int32_t R, int32_t *col_ptr, int32_t C,
+                                               int32_t *dw_gptr, int G, int32_t nnz, int32_t *status)
+{
+    __shared__ int sm[32];
+    scan_counts(row_ptr, R, nullptr, 1, sm);
+    if (col_ptr) scan_counts(col_ptr, C, dw_gptr, G, sm);
+    if (threadIdx.x == 0 && status && nnz >= 0 && row_ptr[R] != nnz) set_status(status, BSL_ERR_NNZ_MISMATCH);
+}
+
+__global__ void k_fill_rows(const uint8_t *__restrict__ mask, int32_t R, int32_t C,
+                            const int32_t *__restrict__ row_ptr, int32_t *__restrict__ col_idx, int32_t nnz)
+{
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (r >= R) return;
+    const uint8_t *row = mask + static_cast<int64_t>(r) * C;
+    int pos = row_ptr[r];
+    for (int c0 = 0; c0 < C; c0 += 32) {
+        const int c = c0 + lane;
+        const bool set = c < C && row[c] != 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, set);
+        const int p = pos + __popc(bal & ((1u << lane) - 1u));
+        if (set && p < nnz) col_idx[p] = c;
+        pos += __popc(bal);
+    }
+}
+
+__global__ void k_fill_cols(const uint8_t *__restrict__ mask, int32_t R, int32_t C,
+                            const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
+                            const int32_t *__restrict__ col_ptr, int32_t *__restrict__ row_idx,
+                            int32_t *__restrict__ csc_to_bsr, int32_t nnz)
+{
+    const int lane = threadIdx.x & 31;
+    const int c = blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (c >= C) return;
+    int pos = col_ptr[c];
+    for (int r0 = 0; r0 < R; r0 += 32) {
+        const int r = r0 + lane;
+        const bool set = r < R && mask[static_cast<int64_t>(r) * C + c] != 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, set);
+        const int j = pos + __popc(bal & ((1u << lane) - 1u));
+        if (set && j < nnz) {
+            // BSR position of (r, c): binary search of c in row r's sorted columns
+            int lo = row_ptr[r], hi = row_ptr[r + 1];
+            lo = lo < 0 ? 0 : lo;
+            hi = hi > nnz ? nnz : hi;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (col_idx[mid] < c) lo = mid + 1;
+                else hi = mid;
+            }
+            row_idx[j] = r;
+            csc_to_bsr[j] = lo < nnz ? lo : nnz - 1;
+        }
+        pos += __popc(bal);
+    }
+}
+
+// values[p][i][:] = W[r*b + i][c*b : c*b + b], 16 bytes per thread per step.
+__global__ void k_gather(const uint4 *__restrict__ W, int32_t K, int32_t b, int32_t R,
+                         const int32_t *__restrict__ row_ptr, const int32_t *__restrict__ col_idx,
+                         uint4 *__restrict__ values, int32_t nnz)
+{
+    const int vpr = b / 8;                  // 16-byte vectors per block row
+    const int64_t per_block = static_cast<int64_t>(b) * vpr;
+    // never read past the blocks the mask really has (nnz may disagree with it)
+    const int64_t kept = row_ptr[R] < nnz ? row_ptr[R] : nnz;
+    const int64_t total = per_block * kept;
+    const int64_t wvpr = K / 8;             // 16-byte vectors per W row
+    for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int p = static_cast<int>(t / per_block);
+        const int rem = static_cast<int>(t - static_cast<int64_t>(p) * per_block);
+        const int i = rem / vpr, v = rem - i * vpr;
+        // block row of p: last r with row_ptr[r] <= p
+        int lo = 0, hi = R;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (row_ptr[mid] <= p) lo = mid;
+            else hi = mid;
+        }
+        const int c = col_idx[p];
+        const int64_t src = (static_cast<int64_t>(lo) * b + i) * wvpr + static_cast<int64_t>(c) * vpr + v;
+        values[t] = __ldg(W + src);
+    }
+}
+
+// order[rank] = id, ranking by count (descending) then id (ascending).
+__global__ void k_order(const int32_t *__restrict__ ptr, int32_t n, int32_t *__restrict__ order)
+{
+    extern __shared__ int32_t cnt_sm[];
+    const int id = blockIdx.x * blockDim.x + threadIdx.x;
+    const int my = id < n ? ptr[id + 1] - ptr[id] : 0;
+    int rank = 0;
+    for (int base = 0; base < n; base += blockDim.x) {
+        const int j = base + threadIdx.x;
+        cnt_sm[threadIdx.x] = j < n ? ptr[j + 1] - ptr[j] : -1;
+        __syncthreads();
+        const int lim = min(static_cast<int>(blockDim.x), n - base);
+        for (int q = 0; q < lim; ++q) {
+            const int o = cnt_sm[q];
+            rank += (o > my) || (o == my && base + q < id);
+        }
+        __syncthreads();
+    }
+    if (id < n) order[rank] = id;
+}
+
+}  // namespace
+
+bsl_status launch_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *row_ptr, cudaStream_t s)
+{
+    k_counts<<<(R + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, row_ptr, nullptr);
+    k_scan<<<1, 1024, 0, s>>>(row_ptr, R, nullptr, 0, nullptr, 1, -1, nullptr);
+    return cuda_status(cudaGetLastError());
+}
+
+bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cudaStream_t s)
+{
+    const int32_t R = o->N / o->b, C = o->K / o->b, nnz = o->nnz;
+    const int G = 128 / o->b;
+    // index arrays start as valid indices (0) even if the mask disagrees with nnz
+    if (nnz > 0) {
+        cudaMemsetAsync(o->col_idx, 0, sizeof(int32_t) * nnz, s);
+        cudaMemsetAsync(o->row_idx, 0, sizeof(int32_t) * nnz, s);
+        cudaMemsetAsync(o->csc_to_bsr, 0, sizeof(int32_t) * nnz, s);
+    }
+    k_counts<<<(R + C + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, o->row_ptr, o->col_ptr);
+    k_scan<<<1, 1024, 0, s>>>(o->row_ptr, R, o->col_ptr, C, o->dw_gptr, G, nnz, o->status);
+    k_fill_rows<<<(R + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, o->row_ptr, o->col_idx, nnz);
+    k_fill_cols<<<(C + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, o->row_ptr, o->col_idx,
+                                                                  o->col_ptr, o->row_idx, o->csc_to_bsr, nnz);
+    if (nnz > 0) {
+        const int64_t total = static_cast<int64_t>(nnz) * o->b * (o->b / 8);
+        const int64_t want = (total + 255) / 256;
+        const int grid = static_cast<int>(want < 8L * num_sms() ? want : 8L * num_sms());
+        k_gather<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(W), o->K, o->b, R, o->row_ptr, o->col_idx,
+                                      static_cast<uint4 *>(o->values), nnz);
+    }
+    k_order<<<(R + 255) / 256, 256, 256 * sizeof(int32_t), s>>>(o->row_ptr, R, o->row_order);
+    k_order<<<(C + 255) / 256, 256, 256 * sizeof(int32_t), s>>>(o->col_ptr, C, o->col_order);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace bsl

@@ -1,0 +1,20 @@
+"""Helpers for the GPU tests: numpy bf16 bits <-> torch CUDA tensors."""
+import numpy as np
+import torch
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    """uint16 bf16 bit array -> bf16 CUDA tensor with the same bits."""
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def mask_dev(mask: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(mask, dtype=np.uint8)).cuda()
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
