@@ -26,6 +26,11 @@
  *  - Matrices are row-major and contiguous (row stride = number of
  *    columns); bf16 is IEEE bfloat16 (2 bytes), passed as void *.
  *  - Every pointer must be 16-byte aligned.
+ *  - Kernels run on the device that owns the first data pointer of the
+ *    call (X, dY, W or the status word); the library makes that device
+ *    current for the calling host thread (binding its primary context, so
+ *    calls from fresh threads work) and returns BSL_ERR_INVALID_ARG for a
+ *    pointer that is not device or managed memory.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *    asynchronous on it unless stated otherwise.
  *  - Arguments are checked on the host before any launch; a failed check

@@ -53,6 +53,21 @@ bsl_status check_device()
     return ok ? BSL_OK : BSL_ERR_NO_DEVICE;
 }
 
+// Make the device that owns `p` current for this host thread (this also
+// binds its primary context, which a fresh thread may not have yet), and
+// reject pointers that are not device memory.
+bsl_status bind_device(const void *p)
+{
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the non-sticky error
+        return BSL_ERR_INVALID_ARG;
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return BSL_ERR_INVALID_ARG;
+    if (cudaSetDevice(a.device) != cudaSuccess) return BSL_ERR_NO_DEVICE;
+    return BSL_OK;
+}
+
 bsl_status check_bsr(const bsl_bsr *W)
 {
     if (!W) return BSL_ERR_INVALID_ARG;
@@ -203,6 +218,7 @@ bsl_status bsl_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *ro
                           void *stream)
 {
     if (!mask || !row_ptr || !nnz_host || R <= 0 || C <= 0) return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(row_ptr));
     BSL_TRY(check_device());
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     BSL_TRY(launch_pack_count(mask, R, C, row_ptr, s));
@@ -214,6 +230,7 @@ bsl_status bsl_pack(const void *W, const uint8_t *mask, const bsl_bsr *out, void
 {
     BSL_TRY(check_bsr(out));
     if (!mask || check_matrix(W, out->N) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(W));
     BSL_TRY(check_device());
     return launch_pack(W, mask, out, static_cast<cudaStream_t>(stream));
 }
@@ -230,6 +247,7 @@ bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, void *Y, v
 {
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(X));
     BSL_TRY(check_device());
     return launch_spmm_tc(X, M, W->K, W, false, Y, W->N, static_cast<cudaStream_t>(stream));
 }
@@ -240,6 +258,7 @@ bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, void *
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
     if (M > kSmallMMax) return BSL_ERR_UNSUPPORTED;
+    BSL_TRY(bind_device(X));
     BSL_TRY(check_device());
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < stream_workspace_bytes(M, W))
         return BSL_ERR_INVALID_ARG;
@@ -257,6 +276,7 @@ bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *W, void 
 {
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(dY, M) != BSL_OK || check_matrix(dX, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(dY));
     BSL_TRY(check_device());
     return launch_spmm_tc(dY, M, W->N, W, true, dX, W->K, static_cast<cudaStream_t>(stream));
 }
@@ -267,6 +287,7 @@ bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const b
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(dY, M) != BSL_OK || check_matrix(X, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
     if (W->nnz > 0 && (!dW_values || !aligned(dW_values, 16))) return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(dY));
     BSL_TRY(check_device());
     return launch_sddmm_tc(dY, X, M, W, dW_values, static_cast<cudaStream_t>(stream));
 }
@@ -274,6 +295,7 @@ bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const b
 bsl_status bsl_get_device_status(const bsl_bsr *W, int32_t *status_host, void *stream)
 {
     if (!W || !W->status || !status_host) return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(W->status));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     BSL_TRY(cuda_status(cudaMemcpyAsync(status_host, W->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s)));
     BSL_TRY(cuda_status(cudaMemsetAsync(W->status, 0, sizeof(int32_t), s)));
@@ -289,6 +311,7 @@ void bsl_set_wait_timeout_us(uint64_t timeout_us)
 bsl_status bsl_debug_wait_timeout(int32_t *status, uint64_t timeout_us, void *stream)
 {
     if (!status || !aligned(status, 4)) return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(status));
     BSL_TRY(check_device());
     return launch_debug_wait(status, timeout_us * 1000ull, static_cast<cudaStream_t>(stream));
 }

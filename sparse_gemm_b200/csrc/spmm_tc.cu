@@ -16,8 +16,10 @@
 // is written as zeros.
 //
 // Work unit = (segment, 128-row tile of M).  The grid is persistent (one CTA
-// per SM); units are dealt round-robin in longest-segment-first order so
-// heavy block rows (Zipf-skewed masks) start first.  Per CTA:
+// per SM); units are dealt round-robin, m-tile-major (CTAs busy at the same
+// time share one tile of activation rows in L2) and longest segment first
+// inside a tile (heavy block rows of Zipf-skewed masks start early).  Each
+// CTA caches its unit descriptors in shared memory at start.  Per CTA:
 //   warp 0      TMA producer: X/dY tile (128 x b) + weight block (b x b) per
 //               stored block into an smem ring (swizzled, 64 B or 128 B rows)
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=b,
@@ -48,7 +50,9 @@ struct SpmmCfg {
     static constexpr uint32_t LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t SBO = 8 * ROW_BYTES;      // stride of 8-row core-matrix groups
     static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BUFS * OUT_BYTES + NUM_BARS * 8 + 16 + 1024;
+    static constexpr int TABLE = 1024;                  // unit descriptors cached in smem per CTA
+    static constexpr int SMEM_BYTES =
+        STAGES * STAGE_BYTES + OUT_BUFS * OUT_BYTES + TABLE * 16 + NUM_BARS * 8 + 16 + 1024;
     static_assert(TMEM_COLS == 128 || TMEM_COLS == 256, "TMEM allocation must be a power of two");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -62,6 +66,18 @@ struct SpmmArgs {
     int32_t *status;
     uint64_t timeout_ns;
 };
+
+// Unit i of this CTA (global unit u = blockIdx.x + i * gridDim.x).  Units
+// run m-tile-major: all segments of one 128-row tile of M before the next
+// tile, so the CTAs working at the same time share the tile's rows of the
+// activation in L2; inside a tile, segments go longest first.
+__device__ __forceinline__ int4 unit_info(const SpmmArgs &a, int i)
+{
+    const int u = blockIdx.x + i * gridDim.x;
+    const int mt = u / a.nseg;
+    const int seg = a.seg_order[u - mt * a.nseg];
+    return make_int4(seg, mt * 128, a.seg_ptr[seg], a.seg_ptr[seg + 1]);
+}
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
 {
@@ -87,7 +103,8 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t *smem = align1024(smem_raw);
     uint8_t *stages = smem;
     uint8_t *outbuf = smem + Cfg::STAGES * Cfg::STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BUFS * Cfg::OUT_BYTES);
+    int4 *table = reinterpret_cast<int4 *>(outbuf + Cfg::OUT_BUFS * Cfg::OUT_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(table + Cfg::TABLE);
     uint64_t *full = bars;
     uint64_t *empty = full + Cfg::STAGES;
     uint64_t *tfull = empty + Cfg::STAGES;
@@ -121,41 +138,59 @@ __global__ void __launch_bounds__(192, 1)
         tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
+    const int units = args.nseg * args.mtiles;
+    const int nlocal = blockIdx.x < units ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int ncached = nlocal < Cfg::TABLE ? nlocal : Cfg::TABLE;
+    for (int i = threadIdx.x; i < ncached; i += blockDim.x) table[i] = unit_info(args, i);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-
-    const int units = args.nseg * args.mtiles;
+    auto unit = [&](int i) { return i < Cfg::TABLE ? table[i] : unit_info(args, i); };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            uint32_t stage = 0, phase = 0, issued = 0, issued_par = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                const int seg = args.seg_order[u / args.mtiles];
-                const int m0 = (u % args.mtiles) * Cfg::BM;
-                const int beg = args.seg_ptr[seg], end = args.seg_ptr[seg + 1];
-                for (int j = beg; j < end; ++j) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, tmo, abort_flag)) {
+        // The warp loads up to 32 entries' indices at once (coalesced); lane 0
+        // waits for free stages and issues the copies.
+        uint32_t stage = 0, phase = 0, issued = 0, issued_par = 0;
+        bool ok = true;
+        for (int i = 0; i < nlocal && ok; ++i) {
+            const int4 ui = unit(i);
+            for (int jb = ui.z; jb < ui.w && ok; jb += 32) {
+                const int j = jb + lane;
+                int acol = 0, blk = 0;
+                if (j < ui.w) {
+                    acol = args.seg_idx[j];
+                    blk = args.blk_map ? args.blk_map[j] : j;
+                }
+                const int cnt = min(32, ui.w - jb);
+                for (int t = 0; t < cnt; ++t) {
+                    const int a_t = __shfl_sync(0xffffffffu, acol, t);
+                    const int b_t = __shfl_sync(0xffffffffu, blk, t);
+                    int good = 1;
+                    if (lane == 0) {
+                        good = mbar_wait(&empty[stage], phase ^ 1, tmo, abort_flag);
+                        if (good) {
+                            uint8_t *sa = stages + stage * Cfg::STAGE_BYTES;
+                            mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+                            tma_load_2d(sa, &tmA, &full[stage], a_t * B, ui.y);
+                            tma_load_2d(sa + Cfg::A_BYTES, &tmW, &full[stage], 0, b_t * B);
+                            issued |= 1u << stage;
+                            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                        }
+                    }
+                    if (!__shfl_sync(0xffffffffu, good, 0)) {
                         ok = false;
                         break;
                     }
-                    const int blk = args.blk_map ? args.blk_map[j] : j;
-                    const int acol = args.seg_idx[j];
-                    uint8_t *sa = stages + stage * Cfg::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, &full[stage], acol * B, m0);
-                    tma_load_2d(sa + Cfg::A_BYTES, &tmW, &full[stage], 0, blk * B);
-                    issued |= 1u << stage;
-                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == Cfg::STAGES) {
                         stage = 0;
                         phase ^= 1;
                     }
                 }
             }
+        }
+        if (lane == 0) {
             if (!ok) {
                 *abort_flag = 1;
                 set_status(args.status, BSL_ERR_TIMEOUT);
@@ -171,9 +206,9 @@ __global__ void __launch_bounds__(192, 1)
             constexpr uint32_t idesc = make_idesc_bf16(128, B, false, TRANS);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             bool ok = true, any = false;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                const int seg = args.seg_order[u / args.mtiles];
-                const int beg = args.seg_ptr[seg], end = args.seg_ptr[seg + 1];
+            for (int i = 0; i < nlocal && ok; ++i) {
+                const int4 ui = unit(i);
+                const int beg = ui.z, end = ui.w;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, tmo, abort_flag)) {
                     ok = false;
                     break;
@@ -227,10 +262,10 @@ __global__ void __launch_bounds__(192, 1)
         const int q = warp & 3;           // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;    // tile row = TMEM lane
         uint32_t acc = 0, acc_phase = 0, ob = 0;
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const int seg = args.seg_order[u / args.mtiles];
-            const int m0 = (u % args.mtiles) * Cfg::BM;
-            const bool nonempty = args.seg_ptr[seg + 1] > args.seg_ptr[seg];
+        for (int i = 0; i < nlocal; ++i) {
+            const int4 ui = unit(i);
+            const int seg = ui.x, m0 = ui.y;
+            const bool nonempty = ui.w > ui.z;
             if (et == 0) {
                 bool go = mbar_wait(&tfull[acc], acc_phase, tmo, abort_flag);
                 if (go) bulk_wait_group_read<Cfg::OUT_BUFS - 1>();  // staging buffer `ob` is free

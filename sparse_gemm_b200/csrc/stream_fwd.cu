@@ -9,19 +9,22 @@
 //
 // Decomposition: the BSR block list [0, nnz) is cut into equal contiguous
 // shares, one per warp of a one-CTA-per-SM grid (block counts, not block
-// rows, are balanced).  Each warp streams its share with 2-D TMA loads of
-// consecutive blocks (16 KB in flight per warp, swizzled rows), multiplies
-// each block with the matching X slice using mma.sync m16n8k16 (bf16 in,
-// fp32 accumulate; the product is Y^T[n][m] = W_blk[n][:] . X[m][:]) and keeps
-// one block row's partial sum in registers:
+// rows, are balanced).  Each warp streams its share through its own ring of
+// stages; a stage holds CH consecutive weight blocks (one 2-D TMA copy, rows
+// swizzled) and, for each of them, the matching slice X[0:MP, c*b:(c+1)*b]
+// (one 2-D TMA copy each, rows >= M zero-filled).  Both operands go to
+// registers with ldmatrix and are multiplied with mma.sync m16n8k16 (bf16
+// in, fp32 accumulate) as Y^T[n][m] = W_blk[n][:] . X[m][:]; the partial sum
+// of the current block row stays in registers:
 //   - a block row entirely inside the warp's share is rounded to bf16 and
 //     written to Y directly;
 //   - a block row cut by a share boundary leaves an fp32 partial in the
 //     workspace, slot 0 if it is the share's first row, else slot 1;
-// k_stream_fixup then sums, for every cut row, the partials of the warps
-// covering it in warp order (deterministic), and writes zeros for block rows
-// without blocks.  The sums are over fp32 partials, each computed in a fixed
-// order, so results are identical run to run.
+// k_stream_fixup (launched as a programmatic dependent of the main kernel,
+// so its launch overlaps the main kernel) then sums, for every cut row, the
+// partials of the warps covering it in warp order, and writes zeros for
+// block rows without blocks.  Every sum has a fixed order, so results are
+// identical run to run.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,23 +32,27 @@ namespace bsl {
 namespace {
 
 constexpr int kStreamWarps = 8;
+constexpr int kWarpSmem = 24 * 1024;  // ring bytes per warp
 
-template <int B>
+template <int B, int MP>
 struct StreamCfg {
     static constexpr int ROW_BYTES = B * 2;
-    static constexpr int CH = B == 32 ? 2 : 1;            // blocks per stage
-    static constexpr int STAGE_BYTES = CH * B * ROW_BYTES;
-    static constexpr int STAGES = B == 32 ? 4 : 2;        // per warp
+    static constexpr int CH = B == 32 ? 2 : 1;          // weight blocks per stage
+    static constexpr int W_BLK = B * ROW_BYTES;         // one weight block
+    static constexpr int X_TILE = MP * ROW_BYTES;       // one X slice (MP tokens x b)
+    static constexpr int STAGE_BYTES = CH * (W_BLK + X_TILE);
+    static constexpr int STAGES = kWarpSmem / STAGE_BYTES;
     static constexpr int WARP_BYTES = STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = kStreamWarps * WARP_BYTES + kStreamWarps * STAGES * 8 + 1024;
+    static_assert(STAGES >= 2, "ring too small");
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the swizzled copies");
 };
 
 struct StreamArgs {
-    const __nv_bfloat16 *X;
     __nv_bfloat16 *Y;
     float *ws;
     const int32_t *row_ptr, *col_idx;
-    int32_t M, N, K, R, C, nnz;
+    int32_t M, N, R, C, nnz;
     int32_t *status;
     uint64_t timeout_ns;
 };
@@ -140,43 +147,73 @@ __device__ __forceinline__ void flush_row(const RowAcc<B, MP> &acc, const Stream
 
 template <int B, int MP>
 __global__ void __launch_bounds__(kStreamWarps * 32, 1)
-    k_stream_fwd(const __grid_constant__ CUtensorMap tmW, const StreamArgs a)
+    k_stream_fwd(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                 const StreamArgs a)
 {
-    using Cfg = StreamCfg<B>;
+    using Cfg = StreamCfg<B, MP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint8_t *ring = smem + warp * Cfg::WARP_BYTES;
-    uint64_t *bars =
-        reinterpret_cast<uint64_t *>(smem + kStreamWarps * Cfg::WARP_BYTES) + warp * Cfg::STAGES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStreamWarps * Cfg::WARP_BYTES) + warp * Cfg::STAGES;
+
+    // let the fix-up grid launch now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int GW = gridDim.x * kStreamWarps;
     const int gw = blockIdx.x * kStreamWarps + warp;
     const int q0 = share_begin(gw, GW, a.nnz), q1 = share_begin(gw + 1, GW, a.nnz);
     if (q0 >= q1) return;  // no block for this warp (no block-wide sync follows)
     const int nchunks = (q1 - q0 + Cfg::CH - 1) / Cfg::CH;
+    const int nfirst = nchunks < Cfg::STAGES ? nchunks : Cfg::STAGES;
 
+    // weight copies first: they depend on nothing
     if (lane == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) mbar_init(&bars[s], 1);
         fence_barrier_init();
-        for (int t = 0; t < Cfg::STAGES && t < nchunks; ++t) {
-            mbar_arrive_expect_tx(&bars[t], Cfg::STAGE_BYTES);
+        for (int t = 0; t < nfirst; ++t) {
+            const int nv = min(Cfg::CH, q1 - (q0 + t * Cfg::CH));
+            mbar_arrive_expect_tx(&bars[t], Cfg::CH * Cfg::W_BLK + nv * Cfg::X_TILE);
             tma_load_2d(ring + t * Cfg::STAGE_BYTES, &tmW, &bars[t], 0, (q0 + t * Cfg::CH) * B);
         }
     }
-    __syncwarp();
+    __syncwarp();  // barrier initialisation visible to the whole warp
+    // block columns of 32 consecutive blocks of the share, one per lane
+    int cbase = q0;
+    int cidx = q0 + lane < q1 ? a.col_idx[q0 + lane] : 0;
+    auto col_of = [&](int p) {  // warp-uniform p; refreshes the lane cache when p leaves it
+        if (p >= cbase + 32) {
+            cbase = p;
+            cidx = p + lane < q1 ? a.col_idx[p + lane] : 0;
+        }
+        const int c = __shfl_sync(0xffffffffu, cidx, p - cbase);
+        return c >= 0 && c < a.C ? c : 0;
+    };
+    auto issue_x = [&](int t) {  // X slices of chunk t (lane 0 issues)
+#pragma unroll
+        for (int cb = 0; cb < Cfg::CH; ++cb) {
+            const int p = q0 + t * Cfg::CH + cb;
+            const int c = col_of(p < q1 ? p : q1 - 1);
+            if (lane == 0 && p < q1)
+                tma_load_2d(ring + (t % Cfg::STAGES) * Cfg::STAGE_BYTES + Cfg::CH * Cfg::W_BLK + cb * Cfg::X_TILE,
+                            &tmX, &bars[t % Cfg::STAGES], c * B, 0);
+        }
+    };
+    for (int t = 0; t < nfirst; ++t) issue_x(t);
 
+    // block-row ends of the share, one per lane: rp = row_ptr[rbase + 1 + lane]
     const int first_row = row_of(a.row_ptr, a.R, q0);
+    int rbase = first_row;
+    int rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
     int r = first_row;
-    int row_end = a.row_ptr[r + 1];
+    int row_end = __shfl_sync(0xffffffffu, rp, 0);
+
     RowAcc<B, MP> acc;
     acc.zero();
-    bool have = false;
-    bool ok = true;
-    const int g = lane >> 2, c2 = (lane & 3) * 2;
+    bool have = false, ok = true;
     float *ws_warp = a.ws + static_cast<int64_t>(gw) * 2 * B * MP;
+    int issued = nfirst;
 
-    int issued = nchunks < Cfg::STAGES ? nchunks : Cfg::STAGES;  // chunks whose load was issued
     for (int t = 0; t < nchunks; ++t) {
         const int s = t % Cfg::STAGES;
         const bool landed = mbar_wait(&bars[s], (t / Cfg::STAGES) & 1, a.timeout_ns, nullptr);
@@ -191,41 +228,39 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
             if (p >= q1) break;
             while (p >= row_end) {  // leaving block row r
                 if (have) {
-                    const bool direct = a.row_ptr[r] >= q0;  // row ends inside the share here
+                    const bool direct = a.row_ptr[r] >= q0;  // row began inside the share too
                     flush_row<B, MP>(acc, a, r, direct, ws_warp + (r == first_row ? 0 : B * MP), lane);
                     acc.zero();
                     have = false;
                 }
                 ++r;
-                row_end = a.row_ptr[r + 1];
+                if (r - rbase >= 32) {  // refresh the lane cache of row ends
+                    rbase = r;
+                    rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
+                }
+                row_end = __shfl_sync(0xffffffffu, rp, r - rbase);
             }
             have = true;
-            const int c = a.col_idx[p];
-            const bool col_ok = c >= 0 && c < a.C;
+            const uint32_t xaddr = stage_addr + Cfg::CH * Cfg::W_BLK + cb * Cfg::X_TILE;
 #pragma unroll
             for (int kk = 0; kk < B / 16; ++kk) {
-                // B fragments: X[token][c*B + kk*16 + (2*(lane%4) | +8)], tokens j*8 + lane/4
+                // B operand from the X slice (rows = tokens); one x4 covers
+                // (tile j, k lo), (j, k hi), (j+1, k lo), (j+1, k hi)
                 uint32_t bf[RowAcc<B, MP>::NT][2];
 #pragma unroll
-                for (int j = 0; j < RowAcc<B, MP>::NT; ++j) {
-                    const int m = j * 8 + g;
-                    if (col_ok && m < a.M) {
-                        const __nv_bfloat16 *xp =
-                            a.X + static_cast<int64_t>(m) * a.K + static_cast<int64_t>(c) * B + kk * 16 + c2;
-                        bf[j][0] = __ldg(reinterpret_cast<const uint32_t *>(xp));
-                        bf[j][1] = __ldg(reinterpret_cast<const uint32_t *>(xp + 8));
-                    } else {
-                        bf[j][0] = 0u;
-                        bf[j][1] = 0u;
-                    }
+                for (int j = 0; j < RowAcc<B, MP>::NT; j += 2) {
+                    const int mi = lane >> 3;
+                    const int tok = (j + (mi >> 1)) * 8 + (lane & 7);
+                    const int chunk = kk * 2 + (mi & 1);
+                    ldmatrix_x4(xaddr + tok * Cfg::ROW_BYTES + swz_chunk<B>(chunk, tok) * 16, bf[j][0], bf[j][1],
+                                bf[j + 1][0], bf[j + 1][1]);
                 }
 #pragma unroll
                 for (int i = 0; i < RowAcc<B, MP>::MT; ++i) {
-                    const int row = cb * B + i * 16 + (lane & 15);     // row inside the stage
+                    const int row = cb * B + i * 16 + (lane & 15);  // weight row inside the stage
                     const int chunk = kk * 2 + (lane >> 4);
-                    const uint32_t addr = stage_addr + row * Cfg::ROW_BYTES + swz_chunk<B>(chunk, row) * 16;
                     uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4(addr, a0, a1, a2, a3);
+                    ldmatrix_x4(stage_addr + row * Cfg::ROW_BYTES + swz_chunk<B>(chunk, row) * 16, a0, a1, a2, a3);
 #pragma unroll
                     for (int j = 0; j < RowAcc<B, MP>::NT; ++j)
                         mma_bf16_16816(acc.d[i][j], a0, a1, a2, a3, bf[j][0], bf[j][1]);
@@ -234,21 +269,26 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
         }
         __syncwarp();
         const int tn = t + Cfg::STAGES;
-        if (tn < nchunks) issued = tn + 1;
-        if (lane == 0 && tn < nchunks) {
-            fence_async_smem();  // ldmatrix reads of this stage precede the next TMA write
-            mbar_arrive_expect_tx(&bars[s], Cfg::STAGE_BYTES);
-            tma_load_2d(ring + s * Cfg::STAGE_BYTES, &tmW, &bars[s], 0, (q0 + tn * Cfg::CH) * B);
+        if (tn < nchunks) {
+            if (lane == 0) {
+                fence_async_smem();  // ldmatrix reads of this stage precede the next TMA write
+                const int nv = min(Cfg::CH, q1 - (q0 + tn * Cfg::CH));
+                mbar_arrive_expect_tx(&bars[s], Cfg::CH * Cfg::W_BLK + nv * Cfg::X_TILE);
+                tma_load_2d(ring + s * Cfg::STAGE_BYTES, &tmW, &bars[s], 0, (q0 + tn * Cfg::CH) * B);
+            }
+            issue_x(tn);
+            issued = tn + 1;
         }
     }
     if (!ok) {
-        if (lane == 0) set_status(a.status, BSL_ERR_TIMEOUT);
-        // let this warp's loads land before its shared memory goes away
-        if (lane == 0)
+        if (lane == 0) {
+            set_status(a.status, BSL_ERR_TIMEOUT);
+            // let this warp's copies land before its shared memory goes away
             for (int t = 0; t < Cfg::STAGES && t < issued; ++t) {
                 const int last = t + ((issued - 1 - t) / Cfg::STAGES) * Cfg::STAGES;  // last chunk on stage t
                 mbar_wait(&bars[t], (last / Cfg::STAGES) & 1, a.timeout_ns, nullptr);
             }
+        }
         __syncwarp();
         return;
     }
@@ -263,6 +303,8 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
 template <int B, int MP>
 __global__ void k_stream_fixup(const StreamArgs a, int GW)
 {
+    // wait until the main grid has finished and its writes are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= a.R) return;
@@ -303,18 +345,33 @@ __global__ void k_stream_fixup(const StreamArgs a, int GW)
 }
 
 template <int B, int MP>
-bsl_status run(const CUtensorMap &mw, const StreamArgs &a, cudaStream_t s)
+bsl_status run(const void *X, const void *values, int32_t K, const StreamArgs &a, cudaStream_t s)
 {
-    using Cfg = StreamCfg<B>;
-    auto kern = k_stream_fwd<B, MP>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_status(e);
+    using Cfg = StreamCfg<B, MP>;
     const int grid = num_sms();
-    if (a.nnz > 0) kern<<<grid, kStreamWarps * 32, Cfg::SMEM_BYTES, s>>>(mw, a);
+    if (a.nnz > 0) {
+        CUtensorMap mw, mx;
+        if (!make_map_2d(&mw, values, B, static_cast<uint64_t>(a.nnz) * B, 2 * B, B, Cfg::CH * B, 2 * B) ||
+            !make_map_2d(&mx, X, K, a.M, static_cast<uint64_t>(K) * 2, B, MP, 2 * B))
+            return BSL_ERR_CUDA;
+        auto kern = k_stream_fwd<B, MP>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_status(e);
+        kern<<<grid, kStreamWarps * 32, Cfg::SMEM_BYTES, s>>>(mw, mx, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+    }
     const int rows_per_cta = 8;
-    k_stream_fixup<B, MP><<<(a.R + rows_per_cta - 1) / rows_per_cta, rows_per_cta * 32, 0, s>>>(
-        a, grid * kStreamWarps);
-    return cuda_status(cudaGetLastError());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((a.R + rows_per_cta - 1) / rows_per_cta);
+    cfg.blockDim = dim3(rows_per_cta * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, k_stream_fixup<B, MP>, a, grid * kStreamWarps));
 }
 
 }  // namespace
@@ -328,27 +385,21 @@ size_t stream_workspace_bytes(int32_t M, const bsl_bsr *W)
 bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *ws, cudaStream_t s)
 {
     const int B = W->b;
-    CUtensorMap mw;
-    const int CH = B == 32 ? 2 : 1;
-    if (W->nnz > 0 &&
-        !make_map_2d(&mw, W->values, B, static_cast<uint64_t>(W->nnz) * B, 2 * B, B, CH * B, 2 * B))
-        return BSL_ERR_CUDA;
     StreamArgs a;
-    a.X = static_cast<const __nv_bfloat16 *>(X);
     a.Y = static_cast<__nv_bfloat16 *>(Y);
     a.ws = static_cast<float *>(ws);
     a.row_ptr = W->row_ptr;
     a.col_idx = W->col_idx;
     a.M = M;
     a.N = W->N;
-    a.K = W->K;
     a.R = W->N / B;
     a.C = W->K / B;
     a.nnz = W->nnz;
     a.status = W->status;
     a.timeout_ns = wait_timeout_ns();
-    if (B == 64) return M <= 16 ? run<64, 16>(mw, a, s) : run<64, 32>(mw, a, s);
-    return M <= 16 ? run<32, 16>(mw, a, s) : run<32, 32>(mw, a, s);
+    if (B == 64)
+        return M <= 16 ? run<64, 16>(X, W->values, W->K, a, s) : run<64, 32>(X, W->values, W->K, a, s);
+    return M <= 16 ? run<32, 16>(X, W->values, W->K, a, s) : run<32, 32>(X, W->values, W->K, a, s);
 }
 
 }  // namespace bsl
