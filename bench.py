@@ -277,20 +277,12 @@ def run_gpu(args):
     kinds = ["fwd", "dx", "dw"] if train else ["fwd"]
     launches_per_step = (2 if small else 1) + (2 if train else 0)
 
-    def step(i, evs=None):
+    def step(i):
         j = i % ncopy
-        if evs is not None:
-            evs[0].record(stream)
         sg.forward(Xs[j], Wps[j], out=Y, workspace=ws)
         if train:
-            if evs is not None:
-                evs[1].record(stream)
             sg.backward_input(dYs[j], Wps[j], out=dX)
-            if evs is not None:
-                evs[2].record(stream)
             sg.backward_weight(dYs[j], Xs[j], Wps[j], out=dWv)
-        if evs is not None:
-            evs[-1].record(stream)
 
     for i in range(args.warmup):
         step(i)
@@ -299,20 +291,71 @@ def run_gpu(args):
         raise RuntimeError("kernels reported a device error")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(kinds) + 1)] for _ in range(K)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def capture(fn):
+        """CUDA graph of K consecutive steps (rotating input copies)."""
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(device=dev)
+        cs.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cs):
+            for i in range(K):
+                fn(i)
+        stream.wait_stream(cs)
+        torch.cuda.synchronize()
+        return g
+
+    def replay_ms(g):
+        g.replay()                      # untimed: first replay uploads the graph
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        g.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        return ev0.elapsed_time(ev1)
+
+    timing = "cuda-graph"
+    try:
+        g_step = capture(step)
+        kernel_graphs = {}
+        if train:
+            kernel_graphs["fwd"] = capture(lambda i: sg.forward(Xs[i % ncopy], Wps[i % ncopy], out=Y, workspace=ws))
+            kernel_graphs["dx"] = capture(lambda i: sg.backward_input(dYs[i % ncopy], Wps[i % ncopy], out=dX))
+            kernel_graphs["dw"] = capture(lambda i: sg.backward_weight(dYs[i % ncopy], Xs[i % ncopy],
+                                                                       Wps[i % ncopy], out=dWv))
+    except Exception as e:  # noqa: BLE001 - fall back to eager launches, said so in the output
+        log("graph capture failed, timing eager launches:", repr(e))
+        timing = "eager"
+
     clocks = ClockSampler(local)
     clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    for i in range(K):
-        step(i, evs[i])
-    torch.cuda.synchronize()
+    if timing == "cuda-graph":
+        total_ms = replay_ms(g_step)
+    else:
+        ev0.record(stream)
+        for i in range(K):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        total_ms = ev0.elapsed_time(ev1)
     if world > 1:
         dist.barrier()
+    # keep the GPU busy inside the clock window for at least ~0.5 s
+    t_end = time.time() + 0.5
+    while timing == "cuda-graph" and time.time() < t_end:
+        g_step.replay()
+        torch.cuda.synchronize()
     clk = clocks.stop()
-    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
-    per_kernel = {k: statistics.mean(e[n].elapsed_time(e[n + 1]) for e in evs) for n, k in enumerate(kinds)}
+    if timing == "cuda-graph":
+        if train:
+            per_kernel = {k: replay_ms(g) / K for k, g in kernel_graphs.items()}
+        else:
+            per_kernel = {"fwd": total_ms / K}
+    else:
+        per_kernel = {k: total_ms / K / len(kinds) for k in kinds}
     if world > 1:
         t = torch.tensor([total_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -350,14 +393,17 @@ def run_gpu(args):
 
     for i in range(max(3, args.warmup)):
         dense_step(i)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    e0.record(stream)
-    for i in range(K):
-        dense_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    dense_ms = e0.elapsed_time(e1) / K
+    if timing == "cuda-graph":
+        dense_ms = replay_ms(capture(dense_step)) / K
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            dense_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / K
 
     # end to end through the public API: pinned host X (+dY) in, Y (+dX, dW) out
     hX = torch.empty(X0.shape, dtype=torch.bfloat16, pin_memory=True).copy_(X0.cpu())
@@ -386,12 +432,12 @@ def run_gpu(args):
     ke = max(3, min(K, 50))
     if world > 1:
         dist.barrier()
-    e0.record(stream)
+    ev0.record(stream)
     for _ in range(ke):
         e2e_step()
-    e1.record(stream)
+    ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / ke
+    e2e_ms = ev0.elapsed_time(ev1) / ke
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -423,6 +469,7 @@ def run_gpu(args):
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": f"rotating {ncopy} copies of every input ({ncopy * in_bytes / 2**20:.0f} MiB > 2x L2)",
             "pack_ms": round(statistics.median(pack_ms), 4),
+            "timing": timing,
         },
         "kernels_ms": {k: round(v, 5) for k, v in per_kernel.items()},
         "roofline": roof,
@@ -430,7 +477,7 @@ def run_gpu(args):
         "speedup_vs_dense": round(dense_ms / ms_per_step, 3),
         "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms, 4)},
+                "ms_per_step": round(e2e_ms, 4), "timing": "eager public API calls"},
         "gpu_launches": K * launches_per_step,
         "clocks": clk,
         "cpu_baseline": cpu,

@@ -65,8 +65,14 @@ typedef enum {
     BSL_ERR_CUDA = 3,          /* a CUDA runtime / driver call failed */
     BSL_ERR_TIMEOUT = 4,       /* a device-side wait ran out of time (device status) */
     BSL_ERR_NNZ_MISMATCH = 5,  /* mask block count != bsl_bsr.nnz (device status) */
-    BSL_ERR_NO_DEVICE = 6      /* no sm_100 device current */
+    BSL_ERR_NO_DEVICE = 6,     /* no sm_100 device current */
+    BSL_ERR_SCRATCH_TOO_SMALL = 7  /* bsl_forward_stream_noalloc: the call needs more
+                                      scratch than BSL_NOALLOC_SCRATCH_BYTES */
 } bsl_status;
+
+/* Bytes of device memory that libbsl keeps, on every GPU that loads it, as
+ * the scratch of bsl_forward_stream_noalloc. */
+#define BSL_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
 /* Packed block-sparse weight.  The caller allocates every array (device
  * memory) with the sizes below, R = N/b, C = K/b; bsl_pack fills them. */
@@ -131,6 +137,33 @@ BSL_API bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, vo
  * bytes; contents on entry do not matter. */
 BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, void *Y,
                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same computation and kernels as bsl_forward_stream, for callers that cannot
+ * allocate device memory: code that must not call cudaMalloc once running
+ * (a serving loop with a fixed memory budget, where an allocation can block
+ * or fail), or a plug-in inside another framework that owns all device
+ * memory and gives the library no allocator.  The pages have no counterpart
+ * of this entry point; it exists only for such callers.
+ *
+ * The scratch is a fixed array of BSL_NOALLOC_SCRATCH_BYTES in libbsl's own
+ * device memory, reserved on every GPU that loads the library until the
+ * process exits.  The entry point allocates nothing and calls no
+ * cudaMalloc / cudaFree.  It returns BSL_ERR_SCRATCH_TOO_SMALL, launching
+ * nothing, when the call would need more scratch than that (the need is
+ * bsl_forward_workspace_bytes(M, W) = SMs x 8 warps x 2 x b x M' x 4 bytes,
+ * M' = 16 for M <= 16, else 32; on a 148-SM B200 that is 4.8 MB for b = 32,
+ * M <= 16, and 9.7 MB for b = 32, M <= 32 or b = 64, M <= 16, which fit;
+ * b = 64 with M > 16 needs 19.4 MB and is rejected).
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress), so make that first call outside any stream
+ * capture.  Every call on a device shares the one array, which keeps the
+ * previous call's contents; nothing in it has to start at zero (each call
+ * writes every partial sum before reading it).  Calls whose kernels overlap
+ * on the GPU (different streams without ordering between them) race on the
+ * array: serialise them.  X, Y, W: as for bsl_forward_stream; the kernels
+ * run on the device that owns X. */
+BSL_API bsl_status bsl_forward_stream_noalloc(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *stream);
 
 /* dX [M][K] = dY [M][N] . W~ (tensor-core kernel over the CSC index). */
 BSL_API bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *W, void *dX, void *stream);

@@ -23,6 +23,7 @@ __all__ = [
     "BslError", "BsrWeight", "library", "count_blocks", "pack", "forward", "forward_tc",
     "forward_stream", "forward_workspace_bytes", "backward_input", "backward_weight",
     "device_status", "set_wait_timeout_us", "debug_wait_timeout", "small_m_max",
+    "forward_stream_noalloc",
     "BlockSparseLinearFunction",
 ]
 
@@ -32,6 +33,7 @@ LIB_PATH = os.path.join(_HERE, "libbsl.so")
 STATUS_NAMES = {
     0: "BSL_OK", 1: "BSL_ERR_INVALID_ARG", 2: "BSL_ERR_UNSUPPORTED", 3: "BSL_ERR_CUDA",
     4: "BSL_ERR_TIMEOUT", 5: "BSL_ERR_NNZ_MISMATCH", 6: "BSL_ERR_NO_DEVICE",
+    7: "BSL_ERR_SCRATCH_TOO_SMALL",
 }
 
 
@@ -76,6 +78,7 @@ def library() -> ctypes.CDLL:
             "bsl_get_device_status": (ctypes.c_int, [BP, ctypes.POINTER(I32), P]),
             "bsl_set_wait_timeout_us": (None, [U64]),
             "bsl_debug_wait_timeout": (ctypes.c_int, [P, U64, P]),
+            "bsl_forward_stream_noalloc": (ctypes.c_int, [P, I32, BP, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -227,6 +230,18 @@ def forward_stream(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = No
     _check(library().bsl_forward_stream(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), workspace.data_ptr(),
                                         workspace.numel() * workspace.element_size(), _stream(X)),
            "bsl_forward_stream")
+    return Y
+
+
+def forward_stream_noalloc(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T on the weight-streaming kernel without a caller-provided
+    workspace (for callers that cannot allocate device memory): the scratch
+    is the library's fixed per-GPU array; overlapping calls race on it."""
+    _cuda_bf16_2d(X, "X", Wp.K)
+    M = X.shape[0]
+    Y = _out(M, Wp.N, X) if out is None else out
+    _check(library().bsl_forward_stream_noalloc(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), _stream(X)),
+           "bsl_forward_stream_noalloc")
     return Y
 
 

@@ -38,6 +38,20 @@ std::once_flag g_timeout_once;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+bsl_status check_matrix(const void *p, int64_t rows)
+{
+    if (rows > 0 && (!p || !aligned(p, 16))) return BSL_ERR_INVALID_ARG;
+    return BSL_OK;
+}
+
+#define BSL_TRY(expr)                          \
+    do {                                       \
+        const bsl_status st_ = (expr);         \
+        if (st_ != BSL_OK) return st_;         \
+    } while (0)
+
+}  // namespace
+
 // device must be sm_100 (B200 family); result cached per device
 bsl_status check_device()
 {
@@ -86,20 +100,6 @@ bsl_status check_bsr(const bsl_bsr *W)
     }
     return BSL_OK;
 }
-
-bsl_status check_matrix(const void *p, int64_t rows)
-{
-    if (rows > 0 && (!p || !aligned(p, 16))) return BSL_ERR_INVALID_ARG;
-    return BSL_OK;
-}
-
-#define BSL_TRY(expr)                          \
-    do {                                       \
-        const bsl_status st_ = (expr);         \
-        if (st_ != BSL_OK) return st_;         \
-    } while (0)
-
-}  // namespace
 
 namespace {
 thread_local int g_last_cuda_error = 0;  // last CUDA error seen by this host thread
@@ -198,6 +198,7 @@ const char *bsl_status_string(bsl_status s)
     case BSL_ERR_TIMEOUT: return "BSL_ERR_TIMEOUT";
     case BSL_ERR_NNZ_MISMATCH: return "BSL_ERR_NNZ_MISMATCH";
     case BSL_ERR_NO_DEVICE: return "BSL_ERR_NO_DEVICE";
+    case BSL_ERR_SCRATCH_TOO_SMALL: return "BSL_ERR_SCRATCH_TOO_SMALL";
     }
     return "BSL_ERR_UNKNOWN";
 }

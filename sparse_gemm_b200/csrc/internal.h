@@ -17,6 +17,10 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
                  uint32_t box_inner, uint32_t box_outer, int swizzle_bytes);
 
 int num_sms();
+// Argument and device checks shared by the entry points (api.cu).
+bsl_status bind_device(const void *p);  // make the device owning p current
+bsl_status check_device();              // current device is sm_100
+bsl_status check_bsr(const bsl_bsr *W);
 uint64_t wait_timeout_ns();
 bsl_status cuda_status(cudaError_t e);
 void note_driver_error(int code);
