@@ -16,6 +16,8 @@ rank's time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # fp64 CPU oracle on a bounded sample
+  python bench.py --kernel-only fwd|dx|dw --workload NAME --reps R
+      # runs one contraction R times on one input copy (for ncu captures)
 """
 from __future__ import annotations
 
@@ -521,6 +523,39 @@ def run_reference(args):
     }
 
 
+def run_kernel_only(args):
+    """One contraction of a workload, `--reps` times, on a single input copy
+    (no rotation, no comparison runs): the command the ncu captures use."""
+    import torch
+
+    import sparse_gemm_b200 as sg
+    from sparse_gemm_b200 import build as _b
+    _b.build()
+    w = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(w, with_dy=args.kernel_only != "fwd")
+    dev = torch.device("cuda", 0)
+
+    def to_dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    Wp = sg.pack(to_dev(inp["W"]), torch.from_numpy(inp["mask"]).to(dev), w.b, nnz=w.nnz)
+    X = to_dev(inp["X"])
+    dY = to_dev(inp["dY"]) if args.kernel_only != "fwd" else None
+    torch.cuda.synchronize()
+    for _ in range(args.reps):
+        if args.kernel_only == "fwd":
+            sg.forward(X, Wp)
+        elif args.kernel_only == "dx":
+            sg.backward_input(dY, Wp)
+        else:
+            sg.backward_weight(dY, X, Wp)
+    torch.cuda.synchronize()
+    st = sg.device_status(Wp)
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+    print(json.dumps({"kernel_only": args.kernel_only, "workload": w.name, "reps": args.reps}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -531,9 +566,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
     ap.add_argument("--reference-budget", type=float, default=120.0)
+    ap.add_argument("--kernel-only", choices=["fwd", "dx", "dw"], default=None)
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.kernel_only:
+        run_kernel_only(args)
+        return
     out = run_reference(args) if args.impl == "reference" else run_gpu(args)
     if out is not None:
         print(json.dumps(out), flush=True)

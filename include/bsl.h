@@ -87,6 +87,30 @@ typedef struct {
     int32_t *row_order;   /* [R] block rows by block count, largest first, ties lower id first */
     int32_t *col_order;   /* [C] block columns, same order rule */
     int32_t *dw_gptr;     /* [C+1] prefix over columns of ceil(col_count / (128/b)) (weight-gradient groups) */
+    /* Work plan of the tensor-core forward: block rows taken G = 256/b at a
+     * time in row_order ("row groups", ceil(R/G) of them).  For each group
+     * the members' block columns are merged into one ascending list of
+     * entries; entry = block column | (member mask << 24), bit i set when the
+     * i-th member of the group holds a block in that column.  The blocks of
+     * the present members are listed entry by entry, members in order. */
+    int32_t *rgrp_ptr;    /* [ceil(R/G)+1] entry range of each row group in rgrp_ent */
+    int32_t *rgrp_bptr;   /* [ceil(R/G)+1] block range of each row group in rgrp_blk */
+    int32_t *rgrp_ent;    /* [nnz] entries (at most nnz) */
+    int32_t *rgrp_blk;    /* [nnz] BSR block of each present member */
+    /* The same plan for the input gradient over block columns (col_order, CSC
+     * index); entry = block row | (member mask << 24). */
+    int32_t *cgrp_ptr;    /* [ceil(C/G)+1] */
+    int32_t *cgrp_bptr;   /* [ceil(C/G)+1] */
+    int32_t *cgrp_ent;    /* [nnz] */
+    int32_t *cgrp_blk;    /* [nnz] */
+    /* Copies of the block values in the order the tensor-core kernels read
+     * them (rgrp_blk / cgrp_blk order), each block stored as the image the
+     * tensor core expects in shared memory: row-major b x b bf16 with the
+     * 16-byte chunks of row i permuted to chunk j ^ (i % 8) for b = 64 or
+     * j ^ ((i / 2) % 4) for b = 32.  One entry's blocks are then a single
+     * contiguous copy.  Written by bsl_pack. */
+    void *values_rg;      /* bf16 [nnz][b][b] */
+    void *values_cg;      /* bf16 [nnz][b][b] */
     int32_t *status;      /* [1] device status word; must be zeroed once at allocation */
 } bsl_bsr;
 

@@ -210,6 +210,48 @@ def schedule_order(ptr) -> np.ndarray:
     return np.asarray(sorted(range(len(counts)), key=lambda i: (-counts[i], i)), dtype=np.int32)
 
 
+def group_plan(ptr, idx, order, G: int, blk=None):
+    """Work plan of the tensor-core forward (segments = block rows) or input
+    gradient (segments = block columns).
+
+    Segments are taken G at a time in ``order`` (longest first).  For each
+    group, the block coordinates of its members are merged into one
+    ascending list of distinct values ("entries"); each entry records which
+    members hold a block there (bit i = i-th member of the group).  The
+    blocks of the present members are listed entry by entry, members in
+    group order.  ``ptr``/``idx`` are the segment pointer and per-entry
+    coordinate arrays (BSR row_ptr/col_idx, or CSC col_ptr/row_idx); ``blk``
+    maps a segment entry to its BSR block (None: the entry position itself).
+
+    Returns (grp_ptr, grp_bptr, ent, blk_list) with ent = coordinate |
+    (mask << 24).
+    """
+    ptr = [int(v) for v in ptr]
+    idx = [int(v) for v in idx]
+    order = [int(v) for v in order]
+    nseg = len(ptr) - 1
+    ngroups = (nseg + G - 1) // G
+    grp_ptr, grp_bptr, ent, blk_list = [0], [0], [], []
+    for g in range(ngroups):
+        members = order[g * G:(g + 1) * G]
+        coords = {}
+        for i, sgm in enumerate(members):
+            for j in range(ptr[sgm], ptr[sgm + 1]):
+                coords.setdefault(idx[j], {})[i] = j
+        for c in sorted(coords):
+            present = coords[c]
+            mask = 0
+            for i in sorted(present):
+                mask |= 1 << i
+                j = present[i]
+                blk_list.append(j if blk is None else int(blk[j]))
+            ent.append(c | (mask << 24))
+        grp_ptr.append(len(ent))
+        grp_bptr.append(len(blk_list))
+    i32 = lambda v: np.asarray(v, dtype=np.int64).astype(np.int32)
+    return i32(grp_ptr), i32(grp_bptr), i32(ent), i32(blk_list)
+
+
 def dw_group_ptr(col_ptr, group: int) -> np.ndarray:
     """Exclusive prefix over block columns of ceil(blocks_in_column / group):
     the weight-gradient kernel processes the blocks of one column in groups

@@ -89,14 +89,19 @@ bsl_status check_bsr(const bsl_bsr *W)
     if (W->N <= 0 || W->K <= 0 || W->N % W->b || W->K % W->b || W->nnz < 0) return BSL_ERR_INVALID_ARG;
     const int64_t R = W->N / W->b, C = W->K / W->b;
     if (W->nnz > R * C) return BSL_ERR_INVALID_ARG;
-    const void *ptrs[] = {W->row_ptr, W->col_ptr, W->row_order, W->col_order, W->dw_gptr, W->status};
+    if (R >= (1 << 24) || C >= (1 << 24)) return BSL_ERR_UNSUPPORTED;  // plan entries hold 24-bit coordinates
+    const void *ptrs[] = {W->row_ptr, W->col_ptr, W->row_order, W->col_order, W->dw_gptr, W->rgrp_ptr,
+                          W->rgrp_bptr, W->cgrp_ptr, W->cgrp_bptr, W->status};
     for (const void *p : ptrs)
         if (!p || !aligned(p, 4)) return BSL_ERR_INVALID_ARG;
     if (W->nnz > 0) {
-        const void *nz[] = {W->col_idx, W->row_idx, W->csc_to_bsr};
+        const void *nz[] = {W->col_idx, W->row_idx, W->csc_to_bsr, W->rgrp_ent, W->rgrp_blk, W->cgrp_ent,
+                            W->cgrp_blk};
         for (const void *p : nz)
             if (!p || !aligned(p, 4)) return BSL_ERR_INVALID_ARG;
         if (!W->values || !aligned(W->values, 16)) return BSL_ERR_INVALID_ARG;
+        if (!W->values_rg || !aligned(W->values_rg, 16) || !W->values_cg || !aligned(W->values_cg, 16))
+            return BSL_ERR_INVALID_ARG;
     }
     return BSL_OK;
 }

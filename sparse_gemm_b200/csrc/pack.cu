@@ -15,6 +15,12 @@
 //   k_fill_cols  one warp per block column: row_idx, csc_to_bsr
 //   k_gather     16-byte vector copy of every kept block into `values`
 //   k_order      rank of each row / column in the longest-first order
+//   k_group_plan one warp per group of G = 256/b rows (columns) in that order:
+//                merges the members' sorted block coordinates into the
+//                entry list of the tensor-core kernels (count pass, scan,
+//                fill pass)
+//   k_gather_mma the values again, in plan order and in the tensor core's
+//                swizzled shared-memory image (one copy per plan)
 #include "common.cuh"
 #include "internal.h"
 
@@ -212,6 +218,104 @@ __global__ void k_order(const int32_t *__restrict__ ptr, int32_t n, int32_t *__r
     if (id < n) order[rank] = id;
 }
 
+// One warp per group of G segments, consecutive in `order`: merges the
+// members' ascending coordinate lists (a warp-wide minimum per step).  The
+// count pass writes the group's entry and block counts to gptr[g+1] and
+// bptr[g+1]; after the scan turns them into offsets, the fill pass writes
+// entry = coordinate | (member mask << 24) and the BSR block of every
+// present member (`blkmap` maps a segment position to its BSR block; null:
+// the position itself).
+template <int G>
+__global__ void k_group_plan(const int32_t *__restrict__ seg_ptr, const int32_t *__restrict__ seg_idx,
+                             const int32_t *__restrict__ blkmap, const int32_t *__restrict__ order, int32_t nseg,
+                             int32_t ngroups, int32_t *__restrict__ gptr, int32_t *__restrict__ bptr,
+                             int32_t *__restrict__ ent, int32_t *__restrict__ blk, int32_t nnz, int fill)
+{
+    static_assert(G <= 8, "member mask is 8 bits");
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * kWarps + (threadIdx.x >> 5);
+    if (g >= ngroups) return;
+    const int mi = g * G + lane;
+    int cur = 0, end = 0;
+    if (lane < G && mi < nseg) {
+        const int sgm = order[mi];
+        cur = max(0, seg_ptr[sgm]);
+        end = min(nnz, seg_ptr[sgm + 1]);
+    }
+    const int e0 = fill ? gptr[g] : 0;
+    const int q0 = fill ? bptr[g] : 0;
+    int count = 0, nb = 0;
+    while (true) {
+        const int v = cur < end ? seg_idx[cur] : 0x7fffffff;
+        const int m = __reduce_min_sync(0xffffffffu, v);
+        if (m == 0x7fffffff) break;
+        const bool present = v == m;
+        const uint32_t mask = __ballot_sync(0xffffffffu, present);
+        if (fill) {
+            if (lane == 0 && e0 + count < nnz) ent[e0 + count] = m | static_cast<int32_t>(mask << 24);
+            const int pos = q0 + nb + __popc(mask & ((1u << lane) - 1u));
+            if (present && pos < nnz) blk[pos] = blkmap ? blkmap[cur] : cur;
+        }
+        nb += __popc(mask);
+        ++count;
+        if (present) ++cur;
+    }
+    if (!fill && lane == 0) {
+        gptr[g + 1] = count;
+        bptr[g + 1] = nb;
+    }
+}
+
+__global__ void __launch_bounds__(1024) k_scan_groups(int32_t *a, int32_t na, int32_t *b, int32_t nb_,
+                                                      int32_t *c, int32_t nc, int32_t *d, int32_t nd)
+{
+    __shared__ int sm[32];
+    scan_counts(a, na, nullptr, 1, sm);
+    scan_counts(b, nb_, nullptr, 1, sm);
+    scan_counts(c, nc, nullptr, 1, sm);
+    scan_counts(d, nd, nullptr, 1, sm);
+}
+
+// dst[i] = block map[i] of `values`, with the 16-byte chunks of each row
+// permuted as the 128-byte (b = 64) / 64-byte (b = 32) swizzle places them.
+__global__ void k_gather_mma(const uint4 *__restrict__ values, const int32_t *__restrict__ map,
+                             uint4 *__restrict__ dst, int32_t b, int32_t nnz)
+{
+    const int vpr = b / 8;
+    const int64_t per_block = static_cast<int64_t>(b) * vpr;
+    const int64_t total = per_block * nnz;
+    for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int i = static_cast<int>(t / per_block);
+        const int rem = static_cast<int>(t - static_cast<int64_t>(i) * per_block);
+        const int row = rem / vpr, ch = rem - row * vpr;
+        int src = map[i];
+        src = src < 0 ? 0 : (src >= nnz ? nnz - 1 : src);
+        const int pch = b == 64 ? (ch ^ (row & 7)) : (ch ^ ((row >> 1) & 3));
+        dst[(static_cast<int64_t>(i) * b + row) * vpr + pch] =
+            values[(static_cast<int64_t>(src) * b + row) * vpr + ch];
+    }
+}
+
+template <int G>
+void launch_group_plans(const bsl_bsr *o, cudaStream_t s)
+{
+    const int32_t R = o->N / o->b, C = o->K / o->b, nnz = o->nnz;
+    const int nrg = (R + G - 1) / G, ncg = (C + G - 1) / G;
+    const int rb = (nrg + kWarps - 1) / kWarps, cbk = (ncg + kWarps - 1) / kWarps;
+    for (int fill = 0; fill < 2; ++fill) {
+        k_group_plan<G><<<rb, kWarps * 32, 0, s>>>(o->row_ptr, o->col_idx, nullptr, o->row_order, R, nrg,
+                                                   o->rgrp_ptr, o->rgrp_bptr, o->rgrp_ent, o->rgrp_blk, nnz,
+                                                   fill);
+        k_group_plan<G><<<cbk, kWarps * 32, 0, s>>>(o->col_ptr, o->row_idx, o->csc_to_bsr, o->col_order, C, ncg,
+                                                    o->cgrp_ptr, o->cgrp_bptr, o->cgrp_ent, o->cgrp_blk, nnz,
+                                                    fill);
+        if (!fill)
+            k_scan_groups<<<1, 1024, 0, s>>>(o->rgrp_ptr, nrg, o->rgrp_bptr, nrg, o->cgrp_ptr, ncg, o->cgrp_bptr,
+                                             ncg);
+    }
+}
+
 }  // namespace
 
 bsl_status launch_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *row_ptr, cudaStream_t s)
@@ -245,6 +349,23 @@ bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cud
     }
     k_order<<<(R + 255) / 256, 256, 256 * sizeof(int32_t), s>>>(o->row_ptr, R, o->row_order);
     k_order<<<(C + 255) / 256, 256, 256 * sizeof(int32_t), s>>>(o->col_ptr, C, o->col_order);
+    if (nnz > 0) {
+        cudaMemsetAsync(o->rgrp_ent, 0, sizeof(int32_t) * nnz, s);
+        cudaMemsetAsync(o->rgrp_blk, 0, sizeof(int32_t) * nnz, s);
+        cudaMemsetAsync(o->cgrp_ent, 0, sizeof(int32_t) * nnz, s);
+        cudaMemsetAsync(o->cgrp_blk, 0, sizeof(int32_t) * nnz, s);
+    }
+    if (o->b == 64) launch_group_plans<4>(o, s);
+    else launch_group_plans<8>(o, s);
+    if (nnz > 0) {
+        const int64_t total = static_cast<int64_t>(nnz) * o->b * (o->b / 8);
+        const int64_t want = (total + 255) / 256;
+        const int grid = static_cast<int>(want < 8L * num_sms() ? want : 8L * num_sms());
+        k_gather_mma<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(o->values), o->rgrp_blk,
+                                          static_cast<uint4 *>(o->values_rg), o->b, nnz);
+        k_gather_mma<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(o->values), o->cgrp_blk,
+                                          static_cast<uint4 *>(o->values_cg), o->b, nnz);
+    }
     return cuda_status(cudaGetLastError());
 }
 

@@ -17,8 +17,11 @@
 // column); a column's last group may hold fewer than G blocks, and its
 // unused accumulator lanes are never stored.
 //
-// Roles as in spmm_tc.cu: warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..5 epilogue (TMEM -> bf16 -> 16-byte global stores).
+// Roles: warps 0..P-1 TMA producers (one thread cannot start copies fast
+// enough, so k-step i is issued by warp i % P; the stage ring is partitioned
+// so that slot i % STAGES is only ever filled by that warp), warp P TMEM
+// owner + MMA issuer, warps P+1..P+4 epilogue (TMEM -> bf16 -> 16-byte
+// global stores).
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,6 +36,9 @@ struct SddmmCfg {
     static constexpr int T_BYTES = MK * ROW_BYTES;       // one strip tile (64 x b)
     static constexpr int STAGE_BYTES = (G + 1) * T_BYTES;
     static constexpr int STAGES = 8;
+    static constexpr int P = 4;                          // producer warps (STAGES % P == 0)
+    static constexpr int THREADS = (P + 5) * 32;
+    static_assert(STAGES % P == 0, "each stage slot belongs to one producer warp");
     static constexpr int ACC = 2;
     static constexpr int TMEM_COLS = ACC * B;            // 64 or 128
     static constexpr uint32_t LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
@@ -68,7 +74,7 @@ __device__ __forceinline__ int group_column(const int32_t *gptr, int C, int g)
 }
 
 template <int B>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
     k_sddmm_tc(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmX,
                const SddmmArgs args)
 {
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_map(&tmDY);
         tma_prefetch_map(&tmX);
     }
-    if (warp == 1) {
+    if (warp == Cfg::P) {
         tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
@@ -114,42 +120,50 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem_base = *tmem_slot;
     const int ngroups = args.dw_gptr[args.C];
 
-    if (warp == 0) {
+    if (warp < Cfg::P) {
+        // k-step i (counted over all groups of this CTA) uses slot i % STAGES and
+        // is issued by warp i % P; the slot's previous fill, step i - STAGES,
+        // was issued by the same warp, so every wait is on the warp's own fills
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0, issued = 0, issued_par = 0;
+            uint32_t issued = 0, issued_par = 0;
             bool ok = true;
+            int i = 0;
             for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x) {
                 const int c = group_column(args.dw_gptr, args.C, g);
                 const int j0 = args.col_ptr[c] + (g - args.dw_gptr[c]) * Cfg::G;
                 const int cnt = min(Cfg::G, args.col_ptr[c + 1] - j0);
-                for (int ks = 0; ks < args.ksteps; ++ks) {
+                int rows[Cfg::G];
+#pragma unroll
+                for (int q = 0; q < Cfg::G; ++q) rows[q] = q < cnt ? args.row_idx[j0 + q] : 0;
+                for (int ks = 0; ks < args.ksteps; ++ks, ++i) {
+                    if (i % Cfg::P != warp) continue;
+                    const int stage = i % Cfg::STAGES;
+                    const uint32_t phase = (i / Cfg::STAGES) & 1;
                     if (!mbar_wait(&empty[stage], phase ^ 1, tmo, abort_flag)) {
                         ok = false;
                         break;
                     }
                     uint8_t *sa = stages + stage * Cfg::STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[stage], (cnt + 1) * Cfg::T_BYTES);
-                    for (int i = 0; i < cnt; ++i)
-                        tma_load_2d(sa + i * Cfg::T_BYTES, &tmDY, &full[stage], args.row_idx[j0 + i] * B,
-                                    ks * Cfg::MK);
+#pragma unroll
+                    for (int q = 0; q < Cfg::G; ++q)
+                        if (q < cnt)
+                            tma_load_2d(sa + q * Cfg::T_BYTES, &tmDY, &full[stage], rows[q] * B, ks * Cfg::MK);
                     tma_load_2d(sa + Cfg::G * Cfg::T_BYTES, &tmX, &full[stage], c * B, ks * Cfg::MK);
                     issued |= 1u << stage;
                     issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-                    if (++stage == Cfg::STAGES) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
                 }
             }
             if (!ok) {
                 *abort_flag = 1;
                 set_status(args.status, BSL_ERR_TIMEOUT);
             }
-            for (int s = 0; s < Cfg::STAGES; ++s)
-                if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_par >> s) & 1u, tmo, nullptr);
+            for (int sl = 0; sl < Cfg::STAGES; ++sl)
+                if (((issued >> sl) & 1u) && !mbar_wait(&full[sl], (issued_par >> sl) & 1u, tmo, nullptr))
+                    set_status(args.status, BSL_ERR_TIMEOUT);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == Cfg::P) {
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc_bf16(128, B, true, true);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
@@ -197,12 +211,12 @@ __global__ void __launch_bounds__(192, 1)
             }
             if (any) {
                 umma_commit(drain);
-                mbar_wait(drain, 0, tmo, nullptr);
+                if (!mbar_wait(drain, 0, tmo, nullptr)) set_status(args.status, BSL_ERR_TIMEOUT);
             }
         }
         __syncwarp();
     } else {
-        const int et = threadIdx.x - 64;
+        const int et = threadIdx.x - (Cfg::P + 1) * 32;
         const int q = warp & 3;
         const int l = q * 32 + lane;      // accumulator row = TMEM lane
         const int blk_in_group = l / B, u = l % B;
@@ -253,7 +267,7 @@ __global__ void __launch_bounds__(192, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == Cfg::P) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
@@ -268,7 +282,7 @@ bsl_status run(const CUtensorMap &dy, const CUtensorMap &x, const SddmmArgs &arg
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_status(e);
     const int grid = ngroups_max < num_sms() ? ngroups_max : num_sms();
-    kern<<<grid, 192, Cfg::SMEM_BYTES, s>>>(dy, x, args);
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(dy, x, args);
     return cuda_status(cudaGetLastError());
 }
 

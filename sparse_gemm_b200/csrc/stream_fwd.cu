@@ -10,12 +10,14 @@
 // Decomposition: the BSR block list [0, nnz) is cut into equal contiguous
 // shares, one per warp of a one-CTA-per-SM grid (block counts, not block
 // rows, are balanced).  Each warp streams its share through its own ring of
-// stages; a stage holds CH consecutive weight blocks (one 2-D TMA copy, rows
-// swizzled) and, for each of them, the matching slice X[0:MP, c*b:(c+1)*b]
-// (one 2-D TMA copy each, rows >= M zero-filled).  Both operands go to
-// registers with ldmatrix and are multiplied with mma.sync m16n8k16 (bf16
-// in, fp32 accumulate) as Y^T[n][m] = W_blk[n][:] . X[m][:]; the partial sum
-// of the current block row stays in registers:
+// stages, a stage holding CH consecutive weight blocks (one 2-D TMA copy,
+// rows swizzled; every warp issues its own copies, since one thread can
+// start only a few copies per microsecond).  The activation slice
+// X[0:MP, c*b:(c+1)*b] of a block is small and stays in L2: its mma.sync
+// fragments are read straight into registers, one block ahead of use.  The
+// weight block goes to registers with ldmatrix; mma.sync m16n8k16 (bf16 in,
+// fp32 accumulate) forms Y^T[n][m] = W_blk[n][:] . X[m][:], and the partial
+// sum of the current block row stays in registers:
 //   - a block row entirely inside the warp's share is rounded to bf16 and
 //     written to Y directly;
 //   - a block row cut by a share boundary leaves an fp32 partial in the
@@ -37,10 +39,9 @@ constexpr int kWarpSmem = 24 * 1024;  // ring bytes per warp
 template <int B, int MP>
 struct StreamCfg {
     static constexpr int ROW_BYTES = B * 2;
-    static constexpr int CH = B == 32 ? 2 : 1;          // weight blocks per stage
+    static constexpr int CH = B == 32 ? 4 : 1;          // weight blocks per stage (8 KB)
     static constexpr int W_BLK = B * ROW_BYTES;         // one weight block
-    static constexpr int X_TILE = MP * ROW_BYTES;       // one X slice (MP tokens x b)
-    static constexpr int STAGE_BYTES = CH * (W_BLK + X_TILE);
+    static constexpr int STAGE_BYTES = CH * W_BLK;
     static constexpr int STAGES = kWarpSmem / STAGE_BYTES;
     static constexpr int WARP_BYTES = STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = kStreamWarps * WARP_BYTES + kStreamWarps * STAGES * 8 + 1024;
@@ -49,10 +50,11 @@ struct StreamCfg {
 };
 
 struct StreamArgs {
+    const __nv_bfloat16 *X;
     __nv_bfloat16 *Y;
     float *ws;
     const int32_t *row_ptr, *col_idx;
-    int32_t M, N, R, C, nnz;
+    int32_t M, N, K, R, C, nnz;
     int32_t *status;
     uint64_t timeout_ns;
 };
@@ -66,18 +68,6 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
 __device__ __forceinline__ int share_begin(int gw, int GW, int nnz)
 {
     return static_cast<int>((static_cast<int64_t>(gw) * nnz) / GW);
-}
-
-// block row holding block p: last r with row_ptr[r] <= p
-__device__ __forceinline__ int row_of(const int32_t *row_ptr, int R, int p)
-{
-    int lo = 0, hi = R;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (row_ptr[mid] <= p) lo = mid;
-        else hi = mid;
-    }
-    return lo;
 }
 
 template <int B>
@@ -147,8 +137,7 @@ __device__ __forceinline__ void flush_row(const RowAcc<B, MP> &acc, const Stream
 
 template <int B, int MP>
 __global__ void __launch_bounds__(kStreamWarps * 32, 1)
-    k_stream_fwd(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                 const StreamArgs a)
+    k_stream_fwd(const __grid_constant__ CUtensorMap tmW, const StreamArgs a)
 {
     using Cfg = StreamCfg<B, MP>;
     extern __shared__ uint8_t smem_raw[];
@@ -172,8 +161,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
         for (int s = 0; s < Cfg::STAGES; ++s) mbar_init(&bars[s], 1);
         fence_barrier_init();
         for (int t = 0; t < nfirst; ++t) {
-            const int nv = min(Cfg::CH, q1 - (q0 + t * Cfg::CH));
-            mbar_arrive_expect_tx(&bars[t], Cfg::CH * Cfg::W_BLK + nv * Cfg::X_TILE);
+            mbar_arrive_expect_tx(&bars[t], Cfg::STAGE_BYTES);
             tma_load_2d(ring + t * Cfg::STAGE_BYTES, &tmW, &bars[t], 0, (q0 + t * Cfg::CH) * B);
         }
     }
@@ -187,22 +175,43 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
             cidx = p + lane < q1 ? a.col_idx[p + lane] : 0;
         }
         const int c = __shfl_sync(0xffffffffu, cidx, p - cbase);
-        return c >= 0 && c < a.C ? c : 0;
+        return c >= 0 && c < a.C ? c : -1;
     };
-    auto issue_x = [&](int t) {  // X slices of chunk t (lane 0 issues)
+    // mma.sync B fragments of block column c: X[j*8 + lane/4][c*b + kk*16 + 2*(lane%4) (+8)]
+    constexpr int KK = B / 16, NT = MP / 8;
+    const int g = lane >> 2, c2 = (lane & 3) * 2;
+    auto load_x = [&](int c, uint32_t (&f)[KK][NT][2]) {
 #pragma unroll
-        for (int cb = 0; cb < Cfg::CH; ++cb) {
-            const int p = q0 + t * Cfg::CH + cb;
-            const int c = col_of(p < q1 ? p : q1 - 1);
-            if (lane == 0 && p < q1)
-                tma_load_2d(ring + (t % Cfg::STAGES) * Cfg::STAGE_BYTES + Cfg::CH * Cfg::W_BLK + cb * Cfg::X_TILE,
-                            &tmX, &bars[t % Cfg::STAGES], c * B, 0);
-        }
+        for (int kk = 0; kk < KK; ++kk)
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int m = j * 8 + g;
+                if (c >= 0 && m < a.M) {
+                    const __nv_bfloat16 *xp =
+                        a.X + static_cast<int64_t>(m) * a.K + static_cast<int64_t>(c) * B + kk * 16 + c2;
+                    f[kk][j][0] = __ldg(reinterpret_cast<const uint32_t *>(xp));
+                    f[kk][j][1] = __ldg(reinterpret_cast<const uint32_t *>(xp + 8));
+                } else {
+                    f[kk][j][0] = 0u;
+                    f[kk][j][1] = 0u;
+                }
+            }
     };
-    for (int t = 0; t < nfirst; ++t) issue_x(t);
+    uint32_t xf[KK][NT][2];
+    load_x(col_of(q0), xf);
 
-    // block-row ends of the share, one per lane: rp = row_ptr[rbase + 1 + lane]
-    const int first_row = row_of(a.row_ptr, a.R, q0);
+    // first block row of the share: last r with row_ptr[r] <= q0, by a
+    // warp-parallel search (two or three rounds of one load per lane)
+    int lo = 0, hi = a.R;  // row_ptr[lo] <= q0 < row_ptr[hi]
+    while (hi - lo > 1) {
+        const int step = (hi - lo + 31) / 32;
+        const int probe = lo + lane * step;
+        const bool le = probe < hi && a.row_ptr[probe] <= q0;
+        const int last = 31 - __clz(__ballot_sync(0xffffffffu, le));  // lane 0 always qualifies
+        lo = lo + last * step;
+        hi = min(hi, lo + step);
+    }
+    const int first_row = lo;
     int rbase = first_row;
     int rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
     int r = first_row;
@@ -226,6 +235,9 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
         for (int cb = 0; cb < Cfg::CH; ++cb) {
             const int p = q0 + t * Cfg::CH + cb;
             if (p >= q1) break;
+            // fragments of the next block, one block ahead
+            uint32_t xn[KK][NT][2];
+            load_x(p + 1 < q1 ? col_of(p + 1) : -1, xn);
             while (p >= row_end) {  // leaving block row r
                 if (have) {
                     const bool direct = a.row_ptr[r] >= q0;  // row began inside the share too
@@ -241,20 +253,8 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                 row_end = __shfl_sync(0xffffffffu, rp, r - rbase);
             }
             have = true;
-            const uint32_t xaddr = stage_addr + Cfg::CH * Cfg::W_BLK + cb * Cfg::X_TILE;
 #pragma unroll
-            for (int kk = 0; kk < B / 16; ++kk) {
-                // B operand from the X slice (rows = tokens); one x4 covers
-                // (tile j, k lo), (j, k hi), (j+1, k lo), (j+1, k hi)
-                uint32_t bf[RowAcc<B, MP>::NT][2];
-#pragma unroll
-                for (int j = 0; j < RowAcc<B, MP>::NT; j += 2) {
-                    const int mi = lane >> 3;
-                    const int tok = (j + (mi >> 1)) * 8 + (lane & 7);
-                    const int chunk = kk * 2 + (mi & 1);
-                    ldmatrix_x4(xaddr + tok * Cfg::ROW_BYTES + swz_chunk<B>(chunk, tok) * 16, bf[j][0], bf[j][1],
-                                bf[j + 1][0], bf[j + 1][1]);
-                }
+            for (int kk = 0; kk < KK; ++kk) {
 #pragma unroll
                 for (int i = 0; i < RowAcc<B, MP>::MT; ++i) {
                     const int row = cb * B + i * 16 + (lane & 15);  // weight row inside the stage
@@ -262,21 +262,26 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                     uint32_t a0, a1, a2, a3;
                     ldmatrix_x4(stage_addr + row * Cfg::ROW_BYTES + swz_chunk<B>(chunk, row) * 16, a0, a1, a2, a3);
 #pragma unroll
-                    for (int j = 0; j < RowAcc<B, MP>::NT; ++j)
-                        mma_bf16_16816(acc.d[i][j], a0, a1, a2, a3, bf[j][0], bf[j][1]);
+                    for (int j = 0; j < NT; ++j)
+                        mma_bf16_16816(acc.d[i][j], a0, a1, a2, a3, xf[kk][j][0], xf[kk][j][1]);
                 }
             }
+#pragma unroll
+            for (int kk = 0; kk < KK; ++kk)
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    xf[kk][j][0] = xn[kk][j][0];
+                    xf[kk][j][1] = xn[kk][j][1];
+                }
         }
         __syncwarp();
         const int tn = t + Cfg::STAGES;
         if (tn < nchunks) {
             if (lane == 0) {
                 fence_async_smem();  // ldmatrix reads of this stage precede the next TMA write
-                const int nv = min(Cfg::CH, q1 - (q0 + tn * Cfg::CH));
-                mbar_arrive_expect_tx(&bars[s], Cfg::CH * Cfg::W_BLK + nv * Cfg::X_TILE);
+                mbar_arrive_expect_tx(&bars[s], Cfg::STAGE_BYTES);
                 tma_load_2d(ring + s * Cfg::STAGE_BYTES, &tmW, &bars[s], 0, (q0 + tn * Cfg::CH) * B);
             }
-            issue_x(tn);
             issued = tn + 1;
         }
     }
@@ -350,16 +355,18 @@ bsl_status run(const void *X, const void *values, int32_t K, const StreamArgs &a
     using Cfg = StreamCfg<B, MP>;
     const int grid = num_sms();
     if (a.nnz > 0) {
-        CUtensorMap mw, mx;
-        if (!make_map_2d(&mw, values, B, static_cast<uint64_t>(a.nnz) * B, 2 * B, B, Cfg::CH * B, 2 * B) ||
-            !make_map_2d(&mx, X, K, a.M, static_cast<uint64_t>(K) * 2, B, MP, 2 * B))
+        CUtensorMap mw;
+        if (!make_map_2d(&mw, values, B, static_cast<uint64_t>(a.nnz) * B, 2 * B, B, Cfg::CH * B, 2 * B))
             return BSL_ERR_CUDA;
         auto kern = k_stream_fwd<B, MP>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_status(e);
-        kern<<<grid, kStreamWarps * 32, Cfg::SMEM_BYTES, s>>>(mw, mx, a);
+        kern<<<grid, kStreamWarps * 32, Cfg::SMEM_BYTES, s>>>(mw, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
     }
+    // same shared-memory carveout as the main kernel: no reconfiguration between the two
+    cudaFuncSetAttribute(k_stream_fixup<B, MP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
     const int rows_per_cta = 8;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((a.R + rows_per_cta - 1) / rows_per_cta);
@@ -386,12 +393,14 @@ bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, void *Y
 {
     const int B = W->b;
     StreamArgs a;
+    a.X = static_cast<const __nv_bfloat16 *>(X);
     a.Y = static_cast<__nv_bfloat16 *>(Y);
     a.ws = static_cast<float *>(ws);
     a.row_ptr = W->row_ptr;
     a.col_idx = W->col_idx;
     a.M = M;
     a.N = W->N;
+    a.K = W->K;
     a.R = W->N / B;
     a.C = W->K / B;
     a.nnz = W->nnz;

@@ -39,8 +39,7 @@ def _bsr(**kw):
     import sparse_gemm_b200 as sg
     s = sg._BSR()
     s.N, s.K, s.b, s.nnz = kw.get("N", 256), kw.get("K", 256), kw.get("b", 32), kw.get("nnz", 4)
-    for name in ("row_ptr", "col_idx", "values", "col_ptr", "row_idx", "csc_to_bsr",
-                 "row_order", "col_order", "dw_gptr", "status"):
+    for name, _ in sg._BSR._fields_[4:]:
         setattr(s, name, kw.get(name, 4096))
     return s
 

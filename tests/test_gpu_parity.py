@@ -47,6 +47,24 @@ def check_pack(Wp, case, b):
     assert np.array_equal(Wp.row_order.cpu().numpy(), oracle.schedule_order(want["row_ptr"]))
     assert np.array_equal(Wp.col_order.cpu().numpy(), oracle.schedule_order(want["col_ptr"]))
     assert np.array_equal(Wp.dw_gptr.cpu().numpy(), oracle.dw_group_ptr(want["col_ptr"], 128 // b))
+    G = 256 // b
+    rplan = oracle.group_plan(want["row_ptr"], want["col_idx"], oracle.schedule_order(want["row_ptr"]), G)
+    cplan = oracle.group_plan(want["col_ptr"], want["row_idx"], oracle.schedule_order(want["col_ptr"]), G,
+                              blk=want["csc_to_bsr"])
+    for pre, plan in (("rgrp", rplan), ("cgrp", cplan)):
+        gp, gb, ent, blk = plan
+        assert np.array_equal(getattr(Wp, pre + "_ptr").cpu().numpy(), gp), pre
+        assert np.array_equal(getattr(Wp, pre + "_bptr").cpu().numpy(), gb), pre
+        assert np.array_equal(getattr(Wp, pre + "_ent")[:len(ent)].cpu().numpy(), ent), pre
+        assert np.array_equal(getattr(Wp, pre + "_blk")[:nnz].cpu().numpy(), blk), pre
+        # plan-ordered copy in the swizzled smem image: chunk j of row i at j ^ f(i)
+        vals = want["values"].reshape(nnz, b, b // 8, 8)[blk]
+        rows = np.arange(b)[:, None]
+        perm = np.arange(b // 8)[None, :] ^ ((rows & 7) if b == 64 else ((rows >> 1) & 3))
+        img = np.empty_like(vals)
+        img[:, rows, perm] = vals
+        got = bits(getattr(Wp, "values_" + pre[0] + "g")[:nnz]).reshape(nnz, b, b // 8, 8)
+        assert np.array_equal(got, img), pre
     assert sg.device_status(Wp) == 0
 
 

@@ -300,3 +300,37 @@ def test_pins_catch_planted_mistakes(oracle_lib, mutant):
     want = brute_forward(case["X"], case["W"], case["mask"].tolist(), b)
     assert np.array_equal(oracle.forward(case["X"], case["W"], case["mask"], b)[0], want)
     assert not np.array_equal(mutant(case["X"], case["W"], case["mask"], b), want)
+
+
+def test_group_plan_covers_every_block_once(oracle_lib):
+    """Each stored block appears exactly once, under its own coordinate and
+    member, and entries are strictly ascending inside a group."""
+    b, R, C, G = 4, 11, 9, 4
+    mask = synth.mask_uniform(R, C, 37, np.random.default_rng(31))
+    mask[5, :] = 0
+    W = synth.bf16_bits(np.random.default_rng(31).standard_normal((R * b, C * b), dtype=np.float32))
+    pk = oracle.pack(W, mask, b)
+    order = oracle.schedule_order(pk["row_ptr"])
+    gp, gb, ent, blk = oracle.group_plan(pk["row_ptr"], pk["col_idx"], order, G)
+    assert sorted(blk.tolist()) == list(range(pk["nnz"]))
+    seen = set()
+    for g in range(len(gp) - 1):
+        members = order[g * G:(g + 1) * G]
+        cols = [int(e) & 0xFFFFFF for e in ent[gp[g]:gp[g + 1]]]
+        assert cols == sorted(set(cols))
+        q = gb[g]
+        for e in ent[gp[g]:gp[g + 1]]:
+            c, m = int(e) & 0xFFFFFF, int(e) >> 24
+            for i in range(G):
+                if m >> i & 1:
+                    p = blk[q]
+                    q += 1
+                    r = members[i]
+                    assert pk["row_ptr"][r] <= p < pk["row_ptr"][r + 1] and pk["col_idx"][p] == c
+                    seen.add((r, c))
+        assert q == gb[g + 1]
+    assert seen == set(zip(*np.nonzero(mask)))
+    # transposed plan over the CSC index maps to the same blocks
+    corder = oracle.schedule_order(pk["col_ptr"])
+    gp, gb, ent, blk = oracle.group_plan(pk["col_ptr"], pk["row_idx"], corder, G, blk=pk["csc_to_bsr"])
+    assert sorted(blk.tolist()) == list(range(pk["nnz"]))
