@@ -87,7 +87,7 @@ typedef struct {
     int32_t *row_order;   /* [R] block rows by block count, largest first, ties lower id first */
     int32_t *col_order;   /* [C] block columns, same order rule */
     int32_t *dw_gptr;     /* [C+1] prefix over columns of ceil(col_count / (128/b)) (weight-gradient groups) */
-    /* Work plan of the tensor-core forward: block rows taken G = 256/b at a
+    /* Work plan of the tensor-core forward: block rows taken G = 128/b at a
      * time in row_order ("row groups", ceil(R/G) of them).  For each group
      * the members' block columns are merged into one ascending list of
      * entries; entry = block column | (member mask << 24), bit i set when the
@@ -112,6 +112,9 @@ typedef struct {
     void *values_rg;      /* bf16 [nnz][b][b] */
     void *values_cg;      /* bf16 [nnz][b][b] */
     int32_t *status;      /* [1] device status word; must be zeroed once at allocation */
+    int32_t *sched;       /* [8] work counters of the persistent tensor-core kernels; zeroed by
+                           * bsl_pack and left at zero by every kernel that uses them, so the
+                           * kernels of one weight must run in stream order (not concurrently) */
 } bsl_bsr;
 
 /* Human-readable name of a status code (static string). */

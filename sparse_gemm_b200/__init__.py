@@ -49,7 +49,7 @@ class _BSR(ctypes.Structure):
         (name, ctypes.c_void_p) for name in
         ("row_ptr", "col_idx", "values", "col_ptr", "row_idx", "csc_to_bsr", "row_order",
          "col_order", "dw_gptr", "rgrp_ptr", "rgrp_bptr", "rgrp_ent", "rgrp_blk", "cgrp_ptr",
-         "cgrp_bptr", "cgrp_ent", "cgrp_blk", "values_rg", "values_cg", "status")]
+         "cgrp_bptr", "cgrp_ent", "cgrp_blk", "values_rg", "values_cg", "status", "sched")]
 
 
 _lib = None
@@ -126,7 +126,7 @@ class BsrWeight:
         self.row_order = torch.empty(R, **i32)
         self.col_order = torch.empty(C, **i32)
         self.dw_gptr = torch.empty(C + 1, **i32)
-        G = 256 // b
+        G = 128 // b
         nrg, ncg = (R + G - 1) // G, (C + G - 1) // G
         self.rgrp_ptr = torch.empty(nrg + 1, **i32)
         self.rgrp_bptr = torch.empty(nrg + 1, **i32)
@@ -139,6 +139,7 @@ class BsrWeight:
         self.values_rg = torch.empty((max(nnz, 1), b, b), dtype=torch.bfloat16, device=device)
         self.values_cg = torch.empty((max(nnz, 1), b, b), dtype=torch.bfloat16, device=device)
         self.status = torch.zeros(1, **i32)
+        self.sched = torch.zeros(8, **i32)
         self._c = _BSR(self.N, self.K, self.b, self.nnz,
                        *[t.data_ptr() for t in (self.row_ptr, self.col_idx, self.values, self.col_ptr,
                                                 self.row_idx, self.csc_to_bsr, self.row_order,
@@ -146,7 +147,7 @@ class BsrWeight:
                                                 self.rgrp_bptr, self.rgrp_ent, self.rgrp_blk,
                                                 self.cgrp_ptr, self.cgrp_bptr, self.cgrp_ent,
                                                 self.cgrp_blk, self.values_rg, self.values_cg,
-                                                self.status)])
+                                                self.status, self.sched)])
 
     @property
     def R(self):

@@ -15,7 +15,7 @@
 //   k_fill_cols  one warp per block column: row_idx, csc_to_bsr
 //   k_gather     16-byte vector copy of every kept block into `values`
 //   k_order      rank of each row / column in the longest-first order
-//   k_group_plan one warp per group of G = 256/b rows (columns) in that order:
+//   k_group_plan one warp per group of G = 128/b rows (columns) in that order:
 //                merges the members' sorted block coordinates into the
 //                entry list of the tensor-core kernels (count pass, scan,
 //                fill pass)
@@ -355,8 +355,9 @@ bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cud
         cudaMemsetAsync(o->cgrp_ent, 0, sizeof(int32_t) * nnz, s);
         cudaMemsetAsync(o->cgrp_blk, 0, sizeof(int32_t) * nnz, s);
     }
-    if (o->b == 64) launch_group_plans<4>(o, s);
-    else launch_group_plans<8>(o, s);
+    if (o->b == 64) launch_group_plans<2>(o, s);
+    else launch_group_plans<4>(o, s);
+    cudaMemsetAsync(o->sched, 0, 8 * sizeof(int32_t), s);
     if (nnz > 0) {
         const int64_t total = static_cast<int64_t>(nnz) * o->b * (o->b / 8);
         const int64_t want = (total + 255) / 256;

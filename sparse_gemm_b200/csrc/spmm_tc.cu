@@ -14,37 +14,48 @@
 // Only stored blocks are touched; output blocks of segments without blocks
 // are written as zeros.
 //
-// Data flow.  On B200 the L2 -> SM fabric, not the tensor core, limits a
-// block-sparse product whose activation tile feeds one b-wide block: every
-// 128 x b activation tile would be fetched once per block.  So segments are
-// processed G = 256/b at a time ("groups", fixed by the pack in longest-
-// first order): for each group the pack merged the members' block
-// coordinates into ascending entries with a member mask.  A work unit is
-// (128-row tile of M, group); per entry the activation tile is fetched once
-// and the weight blocks of the present members follow it into a separate
-// ring, so each activation tile feeds every member that needs it.  Present
-// members that are consecutive in the group and whose blocks sit in
-// consecutive ring slots form a "run" whose blocks are stacked along N: one
-// tcgen05.mma of N = run * b per 16-wide K step, writing the members'
-// accumulator columns directly (runs are also split where a member is
+// Data flow.  On B200 the L2 -> SM fabric (about 20 TB/s in all), not the
+// tensor core, bounds a block-sparse product at low density: every
+// activation tile a block needs must cross it.  Reuse is raised both ways.
+// A work unit is (256-row tile of M, group of G = 128/b segments); the pack
+// fixed the groups (longest-first order) and merged the members' block
+// coordinates into ascending entries with a member mask.  Per entry one
+// 256 x b activation tile is fetched and feeds every present member, and
+// every weight block feeds both 128-row halves of the tile.  Present members
+// that are consecutive in the group and share their first-write status form
+// a "run" whose blocks are stacked along N: per 128-row half and 16-wide K
+// step one tcgen05.mma of N = run * b (runs are split where a member is
 // written for the first time in the unit, since that MMA must overwrite).
-// The accumulator of a unit is G*b = 256 fp32 columns of TMEM; two of them
+// A unit's accumulator is 2 x G*b = 256 fp32 columns of TMEM; two of them
 // let the epilogue of one unit overlap the MMAs of the next.
 //
-// Copies are issued from several warps: one thread can start only a few TMA
-// copies per microsecond, far below what the fabric delivers, so entry e is
-// issued by producer warp e % P.  The weight blocks of an entry sit
-// contiguously in the pack's plan-ordered copy of the values, stored in the
-// swizzled shared-memory image, so they arrive with one 1-D bulk copy into
-// consecutive W-ring slots (an entry never wraps around the ring).
+// Entry slots.  Each entry in flight owns one shared-memory slot: its
+// activation tile and room for G weight blocks.  The weight blocks of an
+// entry sit contiguously in the pack's plan-ordered copy of the values,
+// stored in the swizzled shared-memory image, so they arrive with one 1-D
+// bulk copy.  The producer also writes the entry's MMA runs (TMEM column,
+// block, instruction descriptor, overwrite flag) into a small slot header:
+// one issuing thread is the tensor core's only feeder, so it does nothing
+// per entry but wait, read the header and issue.  One thread starts only about four TMA copies per microsecond,
+// so entry e goes to slot e % S and its copies are issued by producer warp
+// e % P, which owns that slot alone (S a multiple of P): every slot is a
+// single-producer, single-consumer ring.
 //
-// Roles per CTA (persistent grid, one CTA per SM, units dealt round-robin,
-// m-tile-major so concurrent CTAs share activation rows in L2):
-//   warps 0..P-1   producers: TMA tile copy of the activation tile (X ring),
-//                  bulk copy of the entry's weight blocks (W ring)
+// Scheduling.  Units are taken from a per-weight atomic counter in the
+// order of decode_unit (heaviest first inside chunks of m-tiles), so the SMs
+// stay balanced under skewed block rows.  The first producer warp takes a
+// unit only when it starts issuing it (a CTA never sits on work another SM
+// could do) and publishes it to the other roles through a small ring in
+// shared memory.  The last CTA to stop taking units puts the counter back to
+// zero for the next launch, so launches on one weight must be ordered (one
+// stream, or events).
+//
+// Roles per CTA (persistent grid, one CTA per SM):
+//   warps 0..P-1   producers: TMA tile copy of the activation tile, bulk
+//                  copy of the entry's weight blocks, into the entry's slot
 //   warp P         TMEM owner; lane 0 issues the MMAs (bf16 in, fp32 in TMEM)
 //   warps P+1..P+4 epilogue: TMEM -> registers -> bf16 (RNE) -> swizzled smem
-//                  -> TMA store, one 128 x b chunk per member
+//                  -> TMA store; each warp its own 32 rows of every chunk
 // Every wait is bounded in time; on expiry the kernel records
 // BSL_ERR_TIMEOUT, lets its own copies and MMAs drain, frees TMEM and exits.
 #include "common.cuh"
@@ -55,41 +66,48 @@ namespace {
 
 template <int B>
 struct SpmmCfg {
-    static constexpr int BM = 128;                      // rows of M per tile (= MMA M)
-    static constexpr int G = 256 / B;                   // members per group
+    static constexpr int BM = 128;                      // rows of one MMA (M)
+    static constexpr int MSUB = 2;                      // MMA row blocks per unit
+    static constexpr int MT = BM * MSUB;                // rows of M per unit
+    static constexpr int G = 128 / B;                   // members per group
     static constexpr int ROW_BYTES = B * 2;             // one tile row: 64 B (b=32) or 128 B (b=64)
-    static constexpr int A_BYTES = BM * ROW_BYTES;      // activation tile
+    static constexpr int SUB_BYTES = BM * ROW_BYTES;    // one 128-row half of the activation tile
+    static constexpr int X_BYTES = MT * ROW_BYTES;      // activation tile
     static constexpr int W_BYTES = B * ROW_BYTES;       // weight block
+    static constexpr int SLOT_BYTES = X_BYTES + G * W_BYTES;
+    static constexpr int S = B == 64 ? 4 : 8;           // entry slots (= entries in flight)
+    static constexpr int S_LOG = B == 64 ? 2 : 3;
     static constexpr int P = 4;                         // producer warps
-    static constexpr int THREADS = (P + 5) * 32;        // producers, MMA warp, 4 epilogue warps
-    static constexpr int XS = B == 64 ? 5 : 10;         // activation ring slots (= entries in flight)
-    static constexpr int WS = B == 64 ? 12 : 48;        // weight ring slots
-    static constexpr int OUT_BYTES = BM * ROW_BYTES;    // epilogue staging chunk
-    static constexpr int OUT_BUFS = 2;
+    static constexpr int UR = 16;                       // unit-id ring
+    static constexpr int W_MMA = P;                     // then 4 epilogue warps
+    static constexpr int THREADS = (P + 5) * 32;
+    static constexpr int WARP_OUT = 32 * ROW_BYTES;     // one epilogue warp's staging chunk (32 rows)
+    static constexpr int OUT_BYTES = 4 * 2 * WARP_OUT;  // 4 warps x 2 chunks
     static constexpr int ACC = 2;                       // TMEM accumulators
-    static constexpr int ACC_COLS = G * B;              // 256
+    static constexpr int HALF_COLS = G * B;             // 128 columns per row block
+    static constexpr int ACC_COLS = MSUB * HALF_COLS;   // 256
     static constexpr int TMEM_COLS = ACC * ACC_COLS;    // 512
     static constexpr uint32_t LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t SBO = 8 * ROW_BYTES;      // stride of 8-row core-matrix groups
-    static constexpr int TABLE = 256;                   // unit descriptors cached per CTA
-    static constexpr int NUM_BARS = 2 * XS + 2 * ACC + 1;
-    static constexpr int SMEM_BYTES = XS * A_BYTES + WS * W_BYTES + OUT_BUFS * OUT_BYTES + TABLE * 20 +
-                                      P * (WS + XS + 1) * 4 + NUM_BARS * 8 + 32 + 1024;
+    static constexpr int NUM_BARS = 2 * S + 2 * ACC + 2 * UR + 1;
+    static constexpr int HDR_BYTES = S * (G * 8 + 8);   // per slot: run descriptors + run count
+    static constexpr int SMEM_BYTES =
+        S * SLOT_BYTES + OUT_BYTES + NUM_BARS * 8 + HDR_BYTES + UR * 4 + 64 + 1024;
+    static_assert((1 << S_LOG) == S && S % P == 0 && (P & (P - 1)) == 0, "slot ownership");
     static_assert(ACC_COLS == 256 && TMEM_COLS == 512, "TMEM layout");
     static_assert(G <= 8, "member mask is 8 bits");
-    static_assert(XS <= 32, "issue bookkeeping uses a 32-bit mask");
-    static_assert(WS >= G, "one entry's blocks must fit the weight ring");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct SpmmArgs {
-    int32_t M, nseg, ngroups, mtiles, nblk;
+    int32_t M, nseg, ngroups, mtiles, units;  // units = ngroups * mtiles
     const int32_t *seg_ptr;    // [nseg+1] blocks per segment (empty segments give zero output)
     const int32_t *seg_order;  // [nseg] longest first; group g = seg_order[g*G .. g*G+G-1]
     const int32_t *grp_ptr;    // [ngroups+1] entry range per group
     const int32_t *grp_bptr;   // [ngroups+1] block range per group
     const int32_t *grp_ent;    // entries: coordinate | (mask << 24)
     const uint8_t *grp_vals;   // weight blocks in plan order, swizzled smem image
+    int32_t *sched;            // [2] next unit, CTAs finished taking units (zero between launches)
     int32_t *status;
     uint64_t timeout_ns;
 };
@@ -108,15 +126,20 @@ __device__ __forceinline__ int swz_chunk(int chunk, int row)
     else return chunk ^ ((row >> 1) & 3);
 }
 
-// Unit i of this CTA: global unit u = blockIdx.x + i * gridDim.x, m-tile-major.
-// x = group, y = first row of the m-tile, z/w = entry range; first block in *bstart.
-__device__ __forceinline__ int4 unit_info(const SpmmArgs &a, int i, int *bstart)
+// Work order: m-tiles in chunks of CHUNK (the activation rows a chunk needs
+// stay in L2), and inside a chunk group-major, groups in longest-first
+// order, so every chunk starts with its heaviest units and ends with the
+// lightest: the SMs that finish first pick up the small units of the tail.
+constexpr int CHUNK = 8;
+__device__ __forceinline__ void decode_unit(const SpmmArgs &a, int ord, int *mt, int *g)
 {
-    const int u = blockIdx.x + i * gridDim.x;
-    const int mt = u / a.ngroups;
-    const int g = u - mt * a.ngroups;
-    *bstart = a.grp_bptr[g];
-    return make_int4(g, mt * 128, a.grp_ptr[g], a.grp_ptr[g + 1]);
+    const int per_chunk = CHUNK * a.ngroups;
+    const int ch = ord / per_chunk;
+    const int mt0 = ch * CHUNK;
+    const int nmt = min(CHUNK, a.mtiles - mt0);
+    const int r = ord - ch * per_chunk;
+    *g = r / nmt;
+    *mt = mt0 + (r - *g * nmt);
 }
 
 // Ring cursor: slot index + phase parity.
@@ -131,154 +154,200 @@ struct Ring {
     }
 };
 
+// Consumer side of the unit-id ring: the j-th unit id of this CTA (-1: no
+// more units).  Returns false if the wait ran out or the kernel aborted.
+template <int UR>
+__device__ __forceinline__ bool unit_take(uint64_t *ufull, uint64_t *uempty, const volatile int *uring, int j,
+                                          int *uid, uint64_t tmo, const volatile int *abort_flag)
+{
+    const int s = j % UR;
+    if (!mbar_wait(&ufull[s], (j / UR) & 1, tmo, abort_flag)) return false;
+    *uid = uring[s];
+    mbar_arrive(&uempty[s]);
+    return true;
+}
+
 template <int B, bool TRANS>
 __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
-    k_spmm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
-              const __grid_constant__ CUtensorMap tmO, const SpmmArgs args)
+    k_spmm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmO, const SpmmArgs args)
 {
     using Cfg = SpmmCfg<B>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *xring = smem;
-    uint8_t *wring = xring + Cfg::XS * Cfg::A_BYTES;
-    uint8_t *outbuf = wring + Cfg::WS * Cfg::W_BYTES;
-    int4 *table = reinterpret_cast<int4 *>(outbuf + Cfg::OUT_BUFS * Cfg::OUT_BYTES);
-    int *btable = reinterpret_cast<int *>(table + Cfg::TABLE);
-    int *wowner_all = btable + Cfg::TABLE;  // per producer warp: entry that last filled each weight slot
-    int *xlast_all = wowner_all + Cfg::P * Cfg::WS;  // per producer warp: last entry it issued per X slot
-    uint64_t *bars = reinterpret_cast<uint64_t *>(xlast_all + Cfg::P * Cfg::XS + (Cfg::P * Cfg::XS) % 2);
-    uint64_t *xfull = bars;   // all copies of an entry (activation tile + weight blocks)
-    uint64_t *xempty = xfull + Cfg::XS;  // MMAs of the entry done: its X slot and weight slots are free
-    uint64_t *tfull = xempty + Cfg::XS;
-    uint64_t *tempty = tfull + Cfg::ACC;
-    uint64_t *drain = tempty + Cfg::ACC;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint8_t *slots = smem;
+    uint8_t *outbuf = slots + Cfg::S * Cfg::SLOT_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + Cfg::OUT_BYTES);
+    uint64_t *full = bars;                 // the entry's copies landed in the slot
+    uint64_t *empty = full + Cfg::S;       // the entry's MMAs finished: the slot is free
+    uint64_t *tfull = empty + Cfg::S;      // accumulator complete
+    uint64_t *tempty = tfull + Cfg::ACC;   // accumulator read out
+    uint64_t *ufull = tempty + Cfg::ACC;   // unit id published
+    uint64_t *uempty = ufull + Cfg::UR;    // unit id read by every role
+    uint64_t *drain = uempty + Cfg::UR;
+    uint2 *hdr_run = reinterpret_cast<uint2 *>(drain + 1);  // [S][G] runs of the slot's entry
+    int *hdr_n = reinterpret_cast<int *>(hdr_run + Cfg::S * Cfg::G);  // [S] (padded to 8 bytes each)
+    volatile int *uring = reinterpret_cast<volatile int *>(hdr_n + 2 * Cfg::S);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(const_cast<int *>(uring + Cfg::UR));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_go = abort_flag + 1;
-    volatile int *turn = epi_go + 1;  // next entry whose producer may check slot reuse
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::XS; ++s) {
-            mbar_init(&xfull[s], 1);
-            mbar_init(&xempty[s], 1);
+        for (int s = 0; s < Cfg::S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
-        for (int s = 0; s < Cfg::P * Cfg::WS; ++s) wowner_all[s] = -1;
-        for (int s = 0; s < Cfg::P * Cfg::XS; ++s) xlast_all[s] = -1;
         for (int a = 0; a < Cfg::ACC; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 128);
         }
+        for (int u = 0; u < Cfg::UR; ++u) {
+            mbar_init(&ufull[u], 1);
+            mbar_init(&uempty[u], Cfg::P + 5);  // producers, MMA issuer, 4 epilogue warps
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        *epi_go = 0;
-        *turn = 0;
         fence_barrier_init();
         tma_prefetch_map(&tmA);
-        tma_prefetch_map(&tmW);
         tma_prefetch_map(&tmO);
     }
-    if (warp == Cfg::P) {
+    if (warp == Cfg::W_MMA) {
         tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
-    const int units = args.ngroups * args.mtiles;
-    const int nlocal = blockIdx.x < units ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int ncached = nlocal < Cfg::TABLE ? nlocal : Cfg::TABLE;
-    for (int i = threadIdx.x; i < ncached; i += blockDim.x) table[i] = unit_info(args, i, &btable[i]);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    auto unit = [&](int i, int *bstart) {
-        if (i < Cfg::TABLE) {
-            *bstart = btable[i];
-            return table[i];
-        }
-        return unit_info(args, i, bstart);
-    };
 
     if (warp < Cfg::P) {
         // ------------------------------------------------------------ producers
-        // Every producer warp walks all entries (ring cursors and slot owners
-        // stay identical across warps) and issues the copies of entries
-        // e % P == warp.  Entry e uses X slot e % XS; its copies complete on
-        // xfull of that slot, and the MMA warp's one commit per entry frees the
-        // X slot and the entry's weight slots.  A slot is refilled once the
-        // entry that last used it has completed (entries complete in order).
-        // The reuse checks run in entry order (`turn`), so each waits on a
-        // barrier at most one phase ahead of the entry it waits for; the
-        // copies themselves are then issued by the warps concurrently.
-        int *wowner = wowner_all + warp * Cfg::WS;
-        int *xlast = xlast_all + warp * Cfg::XS;
-        Ring xr;
-        uint32_t ws = 0;                 // weight ring cursor
-        int e = 0, done = -1;            // entries walked; highest entry known complete
+        // Every producer warp walks all entries of every unit (block offsets
+        // and first-write status are prefix sums over the unit) and issues the
+        // copies of the entries whose slot it owns.  Before the copies it
+        // writes the entry's MMA runs into the slot header, so the issuer only
+        // reads them; the expect_tx arrive publishes the header with the data.
+        // Slot reuse waits for the one MMA commit of the slot's previous
+        // entry, which this warp also issued, so the parity is unambiguous.
+        const int p = warp;
+        int e = 0;                  // entries walked so far (all units of this CTA)
+        int fills[Cfg::S / Cfg::P]; // fills issued per owned slot
+#pragma unroll
+        for (int i = 0; i < Cfg::S / Cfg::P; ++i) fills[i] = 0;
         bool ok = true;
-        for (int i = 0; i < nlocal && ok; ++i) {
-            int bcur;
-            const int4 ui = unit(i, &bcur);
-            for (int eb = ui.z; eb < ui.w && ok; eb += 32) {
-                const int el = eb + lane < ui.w ? args.grp_ent[eb + lane] : 0;
-                const int n = min(32, ui.w - eb);
-                for (int t = 0; t < n; ++t, ++e) {
+        for (int j = 0; ok; ++j) {
+            int uid = -1, good = 1;
+            if (lane == 0) {
+                if (p == 0) {
+                    // take the next unit only now that this warp starts it, so a CTA
+                    // never holds more than the units it is working on
+                    const int s = j % Cfg::UR;
+                    if (j >= Cfg::UR && !mbar_wait(&uempty[s], ((j / Cfg::UR) - 1) & 1, tmo, abort_flag)) {
+                        good = 0;
+                    } else {
+                        int ord = atomicAdd(args.sched, 1);
+                        if (ord >= args.units) ord = -1;
+                        uring[s] = ord;
+                        mbar_arrive(&ufull[s]);
+                    }
+                }
+                if (good) good = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag);
+            }
+            good = __shfl_sync(0xffffffffu, good, 0);
+            uid = __shfl_sync(0xffffffffu, uid, 0);
+            if (!good) {
+                ok = false;
+                break;
+            }
+            if (uid < 0) break;
+            int mt, g;
+            decode_unit(args, uid, &mt, &g);
+            const int m0 = mt * Cfg::MT;
+            const int z = args.grp_ptr[g], zend = args.grp_ptr[g + 1];
+            int bcur = args.grp_bptr[g];
+            uint32_t seen_carry = 0;  // members present in earlier chunks of this unit
+            for (int eb = z; eb < zend && ok; eb += 32) {
+                const int n = min(32, zend - eb);
+                const int el = lane < n ? args.grp_ent[eb + lane] : 0;
+                const uint32_t ml = static_cast<uint32_t>(el) >> 24;
+                const int kl = __popc(ml);
+                int incl = kl;       // inclusive prefix of block counts over the chunk
+                uint32_t orl = ml;   // inclusive prefix OR of member masks
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    const uint32_t w = __shfl_up_sync(0xffffffffu, orl, o);
+                    if (lane >= o) {
+                        incl += v;
+                        orl |= w;
+                    }
+                }
+                const int excl = incl - kl;
+                uint32_t seen_ex = __shfl_up_sync(0xffffffffu, orl, 1);
+                seen_ex = (lane == 0 ? 0u : seen_ex) | seen_carry;
+                const int total = __shfl_sync(0xffffffffu, incl, 31);
+                const uint32_t all_or = __shfl_sync(0xffffffffu, orl, 31);
+                for (int t = (p - e) & (Cfg::P - 1); t < n; t += Cfg::P) {
                     const uint32_t ent = static_cast<uint32_t>(__shfl_sync(0xffffffffu, el, t));
-                    const int coord = static_cast<int>(ent & 0xFFFFFFu);
-                    const uint32_t k = __popc(ent >> 24);
-                    if (ws + k > Cfg::WS) ws = 0;  // an entry's blocks never wrap
-                    int good = 1;
-                    if (lane == 0 && e % Cfg::P == warp) {
-                        // wait for this entry's turn (all earlier entries passed their checks)
-                        if (*turn != e) {
-                            const uint64_t t0 = globaltimer_ns();
-                            for (uint32_t spin = 1; *turn != e; ++spin) {
-                                // the clock is slow to read: look at it (and the abort flag) rarely
-                                if ((spin & 255u) == 0 && (*abort_flag || globaltimer_ns() - t0 > tmo)) {
-                                    good = 0;
-                                    break;
-                                }
-                            }
-                        }
-                        // entry e-1 passed its checks, which made entry e-1-XS complete, and
-                        // entries complete in order; so any remaining owner is at least
-                        // e - XS and its X-slot barrier is at most one phase ahead of it
-                        done = max(done, e - 1 - Cfg::XS);
-                        if (good && e >= Cfg::XS && e - Cfg::XS > done) {  // X slot: entry e - XS done
-                            good = mbar_wait(&xempty[xr.slot], xr.phase ^ 1, tmo, abort_flag);
-                            done = e - Cfg::XS;
-                        }
-                        for (uint32_t q = 0; q < k && good; ++q) {  // weight slots: last users done
-                            const int owner = wowner[ws + q];
-                            if (owner > done) {
-                                good = mbar_wait(&xempty[owner % Cfg::XS], (owner / Cfg::XS) & 1, tmo, abort_flag);
-                                done = owner;
-                            }
-                        }
+                    const int off = __shfl_sync(0xffffffffu, excl, t);
+                    const uint32_t sb = __shfl_sync(0xffffffffu, seen_ex, t);
+                    // the entry that reuses this slot next: pull its activation tile into L2
+                    const int tn = t + Cfg::S;
+                    const uint32_t entn = static_cast<uint32_t>(__shfl_sync(0xffffffffu, el, tn < n ? tn : 0));
+                    if (lane == 0) {
+                        const int ee = e + t;
+                        const int slot = ee & (Cfg::S - 1);
+                        const int use = ee >> Cfg::S_LOG;
+                        const uint32_t mask = ent >> 24;
+                        const uint32_t k = __popc(mask);
+                        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, tmo, abort_flag)) good = 0;
                         if (good) {
-                            __threadfence_block();
-                            *turn = e + 1;  // the next entry may check its slots
-                            uint64_t *bar = &xfull[xr.slot];
-                            mbar_arrive_expect_tx(bar, Cfg::A_BYTES + k * Cfg::W_BYTES);
-                            tma_load_2d(xring + xr.slot * Cfg::A_BYTES, &tmA, bar, coord * B, ui.y);
-                            if (k)
-                                bulk_load(wring + ws * Cfg::W_BYTES,
-                                          args.grp_vals + static_cast<int64_t>(bcur) * Cfg::W_BYTES,
-                                          k * Cfg::W_BYTES, bar);
-                            xlast[xr.slot] = e;
+                            // runs: consecutive present members with the same first-write
+                            // status; their blocks are consecutive in the slot
+                            uint2 *hr = hdr_run + slot * Cfg::G;
+                            int nr = 0, mbr = 0;
+                            uint32_t q = 0;
+                            while (mbr < Cfg::G) {
+                                if (!((mask >> mbr) & 1u)) {
+                                    ++mbr;
+                                    continue;
+                                }
+                                const int first = mbr;
+                                const uint32_t q0 = q;
+                                const uint32_t st = (sb >> mbr) & 1u;
+                                int len = 1;
+                                ++mbr;
+                                ++q;
+                                while (mbr < Cfg::G && ((mask >> mbr) & 1u) && ((sb >> mbr) & 1u) == st) {
+                                    ++len;
+                                    ++mbr;
+                                    ++q;
+                                }
+                                hr[nr++] = make_uint2(static_cast<uint32_t>(first * B) | (q0 << 8) | (st << 16),
+                                                      make_idesc_bf16(128, len * B, false, TRANS));
+                            }
+                            hdr_n[2 * slot] = nr;
+                            uint8_t *sp = slots + slot * Cfg::SLOT_BYTES;
+                            mbar_arrive_expect_tx(&full[slot], Cfg::X_BYTES + k * Cfg::W_BYTES);
+                            tma_load_2d(sp, &tmA, &full[slot], static_cast<int>(ent & 0xFFFFFFu) * B, m0);
+                            bulk_load(sp + Cfg::X_BYTES,
+                                      args.grp_vals + static_cast<int64_t>(bcur + off) * Cfg::W_BYTES,
+                                      k * Cfg::W_BYTES, &full[slot]);
+                            if (tn < n) tma_prefetch_2d(&tmA, static_cast<int>(entn & 0xFFFFFFu) * B, m0);
+#pragma unroll
+                            for (int i = 0; i < Cfg::S / Cfg::P; ++i)
+                                if (slot == p + i * Cfg::P) fills[i] = use + 1;
                         }
                     }
                     if (!__shfl_sync(0xffffffffu, good, 0)) {
                         ok = false;
                         break;
                     }
-                    if (lane == 0)
-                        for (uint32_t q = 0; q < k; ++q) wowner[ws + q] = e;
-                    ws += k;
-                    bcur += static_cast<int>(k);
-                    xr.next(Cfg::XS);
                 }
+                bcur += total;
+                seen_carry |= all_or;
+                e += n;
             }
         }
         if (lane == 0) {
@@ -286,100 +355,92 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                 *abort_flag = 1;
                 set_status(args.status, BSL_ERR_TIMEOUT);
             }
-            // every copy this warp issued must land before the CTA's smem is released.
-            // If entry x + XS passed its reuse check, x was consumed already; otherwise
-            // x is the last fill of its slot and the parity wait is unambiguous.
-            for (int sl = 0; sl < Cfg::XS; ++sl) {
-                const int x = xlast[sl];
-                if (x >= 0 && *turn <= x + Cfg::XS && !mbar_wait(&xfull[sl], (x / Cfg::XS) & 1, tmo, nullptr))
+            if (p == 0) {
+                // the last CTA to stop taking units resets the counter for the next launch
+                __threadfence();
+                if (atomicAdd(args.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+                    atomicExch(args.sched, 0);
+                    atomicExch(args.sched + 1, 0);
+                }
+            }
+            // every copy this warp issued lands before the CTA's smem is released
+            // (the last fill of a slot is the newest phase of its barrier)
+#pragma unroll
+            for (int i = 0; i < Cfg::S / Cfg::P; ++i) {
+                const int slot = p + i * Cfg::P;
+                if (fills[i] > 0 && !mbar_wait(&full[slot], (fills[i] - 1) & 1, tmo, nullptr))
                     set_status(args.status, BSL_ERR_TIMEOUT);
             }
         }
         __syncwarp();
-    } else if (warp == Cfg::P) {
+    } else if (warp == Cfg::W_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        // The warp walks the entries (cached 32 at a time); lane 0 waits and issues.
-        Ring xr, ar;
-        uint32_t ws = 0;  // weight ring cursor (same allocation rule as the producers)
-        bool ok = true, any = false;
-        for (int i = 0; i < nlocal && ok; ++i) {
-            int bdummy;
-            const int4 ui = unit(i, &bdummy);
-            int good = 1;
-            if (lane == 0) good = mbar_wait(&tempty[ar.slot], ar.phase ^ 1, tmo, abort_flag);
-            if (!__shfl_sync(0xffffffffu, good, 0)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t d0 = tmem_base + ar.slot * Cfg::ACC_COLS;
-            uint32_t seen = 0;  // members already written in this unit
-            for (int eb = ui.z; eb < ui.w && ok; eb += 32) {
-                const int el = eb + lane < ui.w ? args.grp_ent[eb + lane] : 0;
-                const int n = min(32, ui.w - eb);
-                for (int t = 0; t < n; ++t) {
-                    const uint32_t mask = static_cast<uint32_t>(__shfl_sync(0xffffffffu, el, t)) >> 24;
-                    const uint32_t k = __popc(mask);
-                    if (ws + k > Cfg::WS) ws = 0;
-                    if (lane == 0) {
-                        good = mbar_wait(&xfull[xr.slot], xr.phase, tmo, abort_flag);
-                        if (good) {
-                            tc_fence_after();
-                            const uint32_t a0 = smem_u32(xring + xr.slot * Cfg::A_BYTES);
-                            // runs: consecutive present members with the same first-write
-                            // status (their blocks sit in consecutive slots)
-                            uint32_t slot = ws;
-                            int mbr = 0;
-                            while (mbr < Cfg::G) {
-                                if (!((mask >> mbr) & 1u)) {
-                                    ++mbr;
-                                    continue;
-                                }
-                                const int first = mbr;
-                                const uint32_t first_slot = slot;
-                                const uint32_t st = (seen >> mbr) & 1u;
-                                int len = 1;
-                                ++mbr;
-                                ++slot;
-                                while (mbr < Cfg::G && ((mask >> mbr) & 1u) && ((seen >> mbr) & 1u) == st) {
-                                    ++len;
-                                    ++mbr;
-                                    ++slot;
-                                }
-                                const uint32_t idesc = make_idesc_bf16(128, len * B, false, TRANS);
-                                const uint32_t w0 = smem_u32(wring + first_slot * Cfg::W_BYTES);
-#pragma unroll
-                                for (int kk = 0; kk < B / 16; ++kk) {
-                                    const uint64_t ad = make_sdesc(a0 + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT);
-                                    const uint64_t wd =
-                                        TRANS ? make_sdesc(w0 + kk * 16 * Cfg::ROW_BYTES, Cfg::W_BYTES, Cfg::SBO,
-                                                           Cfg::LAYOUT)
-                                              : make_sdesc(w0 + kk * 32, 16, Cfg::SBO, Cfg::LAYOUT);
-                                    umma_bf16(d0 + first * B, ad, wd, idesc, (kk > 0 || st) ? 1u : 0u);
-                                }
-                            }
-                            // the entry's X slot and weight slots are free once these MMAs finish
-                            umma_commit(&xempty[xr.slot]);
-                            any = true;
-                        }
-                    }
-                    if (!__shfl_sync(0xffffffffu, good, 0)) {
+        // Lane 0 alone: per entry one wait, the header's runs (per 128-row
+        // half and 16-wide K step one MMA each), one commit that frees the slot.
+        if (lane == 0) {
+            Ring ar;
+            int e = 0;
+            bool ok = true, any = false;
+            const uint32_t sbase = smem_u32(slots);
+            const uint64_t xdesc0 = make_sdesc(sbase, 16, Cfg::SBO, Cfg::LAYOUT);
+            const uint64_t wdesc0 = TRANS ? make_sdesc(sbase + Cfg::X_BYTES, Cfg::W_BYTES, Cfg::SBO, Cfg::LAYOUT)
+                                          : make_sdesc(sbase + Cfg::X_BYTES, 16, Cfg::SBO, Cfg::LAYOUT);
+            const uint32_t xlo0 = static_cast<uint32_t>(xdesc0), xhi = static_cast<uint32_t>(xdesc0 >> 32);
+            const uint32_t wlo0 = static_cast<uint32_t>(wdesc0), whi = static_cast<uint32_t>(wdesc0 >> 32);
+            // descriptor address units (16 bytes) per 16-wide K step of the weight operand
+            constexpr uint32_t KSTEP_W = TRANS ? (16 * Cfg::ROW_BYTES) >> 4 : 2;
+            constexpr uint32_t SUB_LO = Cfg::SUB_BYTES >> 4;
+            for (int j = 0;; ++j) {
+                int uid = -1;
+                if (!unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (uid < 0) break;
+                int mt, g;
+                decode_unit(args, uid, &mt, &g);
+                const bool two = args.M - mt * Cfg::MT > Cfg::BM;  // second 128-row half in range
+                const int z = args.grp_ptr[g], zend = args.grp_ptr[g + 1];
+                if (!mbar_wait(&tempty[ar.slot], ar.phase ^ 1, tmo, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + ar.slot * Cfg::ACC_COLS;
+                for (int t = z; t < zend; ++t, ++e) {
+                    const int slot = e & (Cfg::S - 1);
+                    if (!mbar_wait(&full[slot], (e >> Cfg::S_LOG) & 1, tmo, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    seen |= mask;
-                    xr.next(Cfg::XS);
-                    ws += k;
+                    tc_fence_after();
+                    const uint32_t soff = static_cast<uint32_t>(slot) * (Cfg::SLOT_BYTES >> 4);
+                    const uint32_t xlo = xlo0 + soff, wlo = wlo0 + soff;
+                    const int nr = hdr_n[2 * slot];
+                    for (int r = 0; r < nr; ++r) {
+                        const uint2 h = hdr_run[slot * Cfg::G + r];
+                        const uint32_t dcol = d0 + (h.x & 0xFFu);
+                        const uint32_t blo = wlo + ((h.x >> 8) & 0xFFu) * (Cfg::W_BYTES >> 4);
+                        const uint32_t st = h.x >> 16;
+#pragma unroll
+                        for (int kk = 0; kk < B / 16; ++kk)
+                            umma_bf16_lo(dcol, xlo + kk * 2, xhi, blo + kk * KSTEP_W, whi, h.y, kk ? 1u : st);
+                        if (two) {
+#pragma unroll
+                            for (int kk = 0; kk < B / 16; ++kk)
+                                umma_bf16_lo(dcol + Cfg::HALF_COLS, xlo + SUB_LO + kk * 2, xhi, blo + kk * KSTEP_W,
+                                             whi, h.y, kk ? 1u : st);
+                        }
+                    }
+                    // the slot is free once these MMAs finish
+                    umma_commit(&empty[slot]);
+                    any = true;
                 }
-            }
-            if (!ok) break;
-            if (lane == 0) {
-                if (ui.w > ui.z) umma_commit(&tfull[ar.slot]);
+                if (!ok) break;
+                if (zend > z) umma_commit(&tfull[ar.slot]);
                 else mbar_arrive(&tfull[ar.slot]);
+                ar.next(Cfg::ACC);
             }
-            ar.next(Cfg::ACC);
-        }
-        if (lane == 0) {
             if (!ok) {
                 *abort_flag = 1;
                 set_status(args.status, BSL_ERR_TIMEOUT);
@@ -392,15 +453,32 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        const int et = threadIdx.x - (Cfg::P + 1) * 32;  // 0..127
-        const int q = warp & 3;           // TMEM lane quarter this warp may access
-        const int row = q * 32 + lane;    // tile row = TMEM lane
+        // Each warp drains its own 32 TMEM lanes (tile rows) of every chunk
+        // and writes them with its own TMA stores (two staging chunks per
+        // warp), so the four epilogue warps never wait on one another.
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        uint8_t *wbuf = outbuf + q * 2 * Cfg::WARP_OUT;
         Ring ar;
         uint32_t ob = 0;
-        for (int i = 0; i < nlocal; ++i) {
-            int bdummy;
-            const int4 ui = unit(i, &bdummy);
-            const int g = ui.x, m0 = ui.y;
+        bool ok = true;
+        for (int j = 0;; ++j) {
+            int uid = -1, go = 1;
+            if (lane == 0) {
+                go = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag);
+                if (go && uid >= 0) go = mbar_wait(&tfull[ar.slot], ar.phase, tmo, abort_flag);
+            }
+            go = __shfl_sync(0xffffffffu, go, 0);
+            uid = __shfl_sync(0xffffffffu, uid, 0);
+            if (!go) {
+                ok = false;
+                break;
+            }
+            if (uid < 0) break;
+            tc_fence_after();
+            int mt, g;
+            decode_unit(args, uid, &mt, &g);
+            const int m0 = mt * Cfg::MT;
+            const int nsub = args.M - m0 > Cfg::BM ? 2 : 1;
             // members of the group and whether they hold any block (lane i < G)
             const int mi = g * Cfg::G + lane;
             int mseg = -1, mnz = 0;
@@ -408,80 +486,78 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                 mseg = args.seg_order[mi];
                 mnz = args.seg_ptr[mseg + 1] > args.seg_ptr[mseg];
             }
-            if (et == 0) {
-                const bool go = mbar_wait(&tfull[ar.slot], ar.phase, tmo, abort_flag);
-                if (!go) {
-                    *abort_flag = 1;
-                    set_status(args.status, BSL_ERR_TIMEOUT);
-                }
-                *epi_go = go ? 1 : 0;
-            }
-            named_bar_sync(1, 128);
-            if (!*epi_go) break;
-            tc_fence_after();
-            for (int mbr = 0; mbr < Cfg::G; ++mbr) {
-                const int seg = __shfl_sync(0xffffffffu, mseg, mbr);
-                const int nz = __shfl_sync(0xffffffffu, mnz, mbr);
-                if (seg < 0) break;
-                uint32_t v[B];
-                if (nz) {
-                    const uint32_t taddr =
-                        tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ar.slot * Cfg::ACC_COLS + mbr * B;
+            for (int s = 0; s < nsub; ++s) {
+                const int r0 = m0 + s * Cfg::BM + q * 32;  // first output row of this warp
+                if (r0 >= args.M) continue;
+                for (int mbr = 0; mbr < Cfg::G; ++mbr) {
+                    const int seg = __shfl_sync(0xffffffffu, mseg, mbr);
+                    const int nz = __shfl_sync(0xffffffffu, mnz, mbr);
+                    if (seg < 0) break;
+                    uint32_t v[B];
+                    if (nz) {
+                        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                               ar.slot * Cfg::ACC_COLS + s * Cfg::HALF_COLS + mbr * B;
 #pragma unroll
-                    for (int c = 0; c < B / 16; ++c)
-                        tmem_ld16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
-                    tmem_wait_ld();
-                } else {
+                        for (int c = 0; c < B / 16; ++c)
+                            tmem_ld16(taddr + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[c * 16]));
+                        tmem_wait_ld();
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < B; ++c) v[c] = 0u;
-                }
-                if (et == 0) bulk_wait_group_read<Cfg::OUT_BUFS - 1>();  // staging chunk `ob` is free
-                named_bar_sync(1, 128);
-                uint8_t *dst = outbuf + ob * Cfg::OUT_BYTES + row * Cfg::ROW_BYTES;
+                        for (int c = 0; c < B; ++c) v[c] = 0u;
+                    }
+                    if (lane == 0) bulk_wait_group_read<1>();  // staging chunk `ob` was read out
+                    __syncwarp();
+                    uint8_t *dst = wbuf + ob * Cfg::WARP_OUT + lane * Cfg::ROW_BYTES;
 #pragma unroll
-                for (int c = 0; c < B / 8; ++c) {
-                    uint4 pk;
-                    pk.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-                    pk.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-                    pk.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-                    pk.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-                    *reinterpret_cast<uint4 *>(dst + swz_chunk<B>(c, row) * 16) = pk;
+                    for (int c = 0; c < B / 8; ++c) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
+                        pk.y = pack_bf16x2(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
+                        pk.z = pack_bf16x2(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
+                        pk.w = pack_bf16x2(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
+                        *reinterpret_cast<uint4 *>(dst + swz_chunk<B>(c, lane) * 16) = pk;
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmO, wbuf + ob * Cfg::WARP_OUT, seg * B, r0);
+                        bulk_commit_group();
+                    }
+                    ob ^= 1;
                 }
-                fence_async_smem();
-                named_bar_sync(1, 128);
-                if (et == 0) {
-                    tma_store_2d(&tmO, outbuf + ob * Cfg::OUT_BYTES, seg * B, m0);
-                    bulk_commit_group();
-                }
-                ob ^= 1;
             }
             // every TMEM read of this accumulator is complete (each was waited)
             tc_fence_before();
             mbar_arrive(&tempty[ar.slot]);
             ar.next(Cfg::ACC);
         }
-        if (et == 0) bulk_wait_group<0>();
+        if (lane == 0) {
+            if (!ok) {
+                *abort_flag = 1;
+                set_status(args.status, BSL_ERR_TIMEOUT);
+            }
+            bulk_wait_group<0>();
+        }
+        __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == Cfg::P) {
+    if (warp == Cfg::W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
 }
 
 template <int B, bool TRANS>
-bsl_status run(const CUtensorMap &a, const CUtensorMap &w, const CUtensorMap &o, const SpmmArgs &args,
-               cudaStream_t s)
+bsl_status run(const CUtensorMap &a, const CUtensorMap &o, const SpmmArgs &args, cudaStream_t s)
 {
     using Cfg = SpmmCfg<B>;
     auto kern = k_spmm_tc<B, TRANS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_status(e);
-    const int units = args.ngroups * args.mtiles;
-    const int grid = units < num_sms() ? units : num_sms();
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(a, w, o, args);
+    const int grid = args.units < num_sms() ? args.units : num_sms();
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(a, o, args);
     return cuda_status(cudaGetLastError());
 }
 
@@ -493,28 +569,28 @@ bsl_status launch_spmm_tc(const void *A, int32_t M, int32_t a_cols, const bsl_bs
     const int B = W->b;
     if (W->nnz == 0)
         return cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(M) * out_cols * 2, s));
-    CUtensorMap ma, mw, mo;
-    if (!make_map_2d(&ma, A, a_cols, M, static_cast<uint64_t>(a_cols) * 2, B, 128, 2 * B) ||
-        !make_map_2d(&mw, W->values, B, static_cast<uint64_t>(W->nnz) * B, 2 * B, B, B, 2 * B) ||
-        !make_map_2d(&mo, out, out_cols, M, static_cast<uint64_t>(out_cols) * 2, B, 128, 2 * B))
+    CUtensorMap ma, mo;
+    if (!make_map_2d(&ma, A, a_cols, M, static_cast<uint64_t>(a_cols) * 2, B, 256, 2 * B) ||
+        !make_map_2d(&mo, out, out_cols, M, static_cast<uint64_t>(out_cols) * 2, B, 32, 2 * B))
         return BSL_ERR_CUDA;
-    const int G = 256 / B;
+    const int G = 128 / B;
     SpmmArgs args;
     args.M = M;
-    args.mtiles = (M + 127) / 128;
+    args.mtiles = (M + 255) / 256;
     args.nseg = transposed ? W->K / B : W->N / B;
     args.ngroups = (args.nseg + G - 1) / G;
-    args.nblk = W->nnz;
+    args.units = args.ngroups * args.mtiles;
     args.seg_ptr = transposed ? W->col_ptr : W->row_ptr;
     args.seg_order = transposed ? W->col_order : W->row_order;
     args.grp_ptr = transposed ? W->cgrp_ptr : W->rgrp_ptr;
     args.grp_bptr = transposed ? W->cgrp_bptr : W->rgrp_bptr;
     args.grp_ent = transposed ? W->cgrp_ent : W->rgrp_ent;
     args.grp_vals = static_cast<const uint8_t *>(transposed ? W->values_cg : W->values_rg);
+    args.sched = W->sched + (transposed ? 2 : 0);
     args.status = W->status;
     args.timeout_ns = wait_timeout_ns();
-    if (B == 64) return transposed ? run<64, true>(ma, mw, mo, args, s) : run<64, false>(ma, mw, mo, args, s);
-    return transposed ? run<32, true>(ma, mw, mo, args, s) : run<32, false>(ma, mw, mo, args, s);
+    if (B == 64) return transposed ? run<64, true>(ma, mo, args, s) : run<64, false>(ma, mo, args, s);
+    return transposed ? run<32, true>(ma, mo, args, s) : run<32, false>(ma, mo, args, s);
 }
 
 }  // namespace bsl

@@ -47,7 +47,7 @@ def check_pack(Wp, case, b):
     assert np.array_equal(Wp.row_order.cpu().numpy(), oracle.schedule_order(want["row_ptr"]))
     assert np.array_equal(Wp.col_order.cpu().numpy(), oracle.schedule_order(want["col_ptr"]))
     assert np.array_equal(Wp.dw_gptr.cpu().numpy(), oracle.dw_group_ptr(want["col_ptr"], 128 // b))
-    G = 256 // b
+    G = 128 // b
     rplan = oracle.group_plan(want["row_ptr"], want["col_idx"], oracle.schedule_order(want["row_ptr"]), G)
     cplan = oracle.group_plan(want["col_ptr"], want["row_idx"], oracle.schedule_order(want["col_ptr"]), G,
                               blk=want["csc_to_bsr"])
