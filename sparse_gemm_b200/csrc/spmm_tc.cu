@@ -90,7 +90,8 @@ struct SpmmCfg {
     static constexpr uint32_t LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t SBO = 8 * ROW_BYTES;      // stride of 8-row core-matrix groups
     static constexpr int NUM_BARS = 2 * S + 2 * ACC + 2 * UR + 1;
-    static constexpr int HDR_BYTES = S * (G * 8 + 8);   // per slot: run descriptors + run count
+    static constexpr int HDR_V4 = (G + 1) / 2;          // 16-byte header words per slot (two runs each)
+    static constexpr int HDR_BYTES = S * HDR_V4 * 16;
     static constexpr int SMEM_BYTES =
         S * SLOT_BYTES + OUT_BYTES + NUM_BARS * 8 + HDR_BYTES + UR * 4 + 64 + 1024;
     static_assert((1 << S_LOG) == S && S % P == 0 && (P & (P - 1)) == 0, "slot ownership");
@@ -184,9 +185,12 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
     uint64_t *ufull = tempty + Cfg::ACC;   // unit id published
     uint64_t *uempty = ufull + Cfg::UR;    // unit id read by every role
     uint64_t *drain = uempty + Cfg::UR;
-    uint2 *hdr_run = reinterpret_cast<uint2 *>(drain + 1);  // [S][G] runs of the slot's entry
-    int *hdr_n = reinterpret_cast<int *>(hdr_run + Cfg::S * Cfg::G);  // [S] (padded to 8 bytes each)
-    volatile int *uring = reinterpret_cast<volatile int *>(hdr_n + 2 * Cfg::S);
+    // [S][HDR_V4] MMA runs of the slot's entry, two per 16-byte word: run r is
+    // (x, y) = (.x, .y) or (.z, .w) of word r / 2 with x = TMEM column | weight
+    // block offset (16-byte units) << 8 | run count (run 0 only) << 24 |
+    // overwrite-free flag << 28 and y = the instruction descriptor
+    uint4 *hdr = reinterpret_cast<uint4 *>((reinterpret_cast<uintptr_t>(drain + 1) + 15) & ~uintptr_t(15));
+    volatile int *uring = reinterpret_cast<volatile int *>(hdr + Cfg::S * Cfg::HDR_V4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(const_cast<int *>(uring + Cfg::UR));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                         if (good) {
                             // runs: consecutive present members with the same first-write
                             // status; their blocks are consecutive in the slot
-                            uint2 *hr = hdr_run + slot * Cfg::G;
+                            uint2 *hr = reinterpret_cast<uint2 *>(hdr + slot * Cfg::HDR_V4);
                             int nr = 0, mbr = 0;
                             uint32_t q = 0;
                             while (mbr < Cfg::G) {
@@ -324,10 +328,11 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                                     ++mbr;
                                     ++q;
                                 }
-                                hr[nr++] = make_uint2(static_cast<uint32_t>(first * B) | (q0 << 8) | (st << 16),
+                                hr[nr++] = make_uint2(static_cast<uint32_t>(first * B) |
+                                                          ((q0 * (Cfg::W_BYTES >> 4)) << 8) | (st << 28),
                                                       make_idesc_bf16(128, len * B, false, TRANS));
                             }
-                            hdr_n[2 * slot] = nr;
+                            hr[0].x |= static_cast<uint32_t>(nr) << 24;
                             uint8_t *sp = slots + slot * Cfg::SLOT_BYTES;
                             mbar_arrive_expect_tx(&full[slot], Cfg::X_BYTES + k * Cfg::W_BYTES);
                             tma_load_2d(sp, &tmA, &full[slot], static_cast<int>(ent & 0xFFFFFFu) * B, m0);
@@ -409,27 +414,38 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                 const uint32_t d0 = tmem_base + ar.slot * Cfg::ACC_COLS;
                 for (int t = z; t < zend; ++t, ++e) {
                     const int slot = e & (Cfg::S - 1);
+                    // the copies are ordered before the MMAs by the barrier itself (both
+                    // are async-proxy accesses), so no tcgen05 fence is needed here
                     if (!mbar_wait(&full[slot], (e >> Cfg::S_LOG) & 1, tmo, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
                     const uint32_t soff = static_cast<uint32_t>(slot) * (Cfg::SLOT_BYTES >> 4);
                     const uint32_t xlo = xlo0 + soff, wlo = wlo0 + soff;
-                    const int nr = hdr_n[2 * slot];
-                    for (int r = 0; r < nr; ++r) {
-                        const uint2 h = hdr_run[slot * Cfg::G + r];
-                        const uint32_t dcol = d0 + (h.x & 0xFFu);
-                        const uint32_t blo = wlo + ((h.x >> 8) & 0xFFu) * (Cfg::W_BYTES >> 4);
-                        const uint32_t st = h.x >> 16;
+                    const uint4 *hs = hdr + slot * Cfg::HDR_V4;
+                    const uint4 h0 = hs[0];
+                    const int nr = static_cast<int>((h0.x >> 24) & 0xFu);
+                    auto issue_run = [&](uint32_t x, uint32_t y) {
+                        const uint32_t dcol = d0 + (x & 0xFFu);
+                        const uint32_t blo = wlo + ((x >> 8) & 0xFFFFu);
+                        const uint32_t st = x >> 28;
 #pragma unroll
                         for (int kk = 0; kk < B / 16; ++kk)
-                            umma_bf16_lo(dcol, xlo + kk * 2, xhi, blo + kk * KSTEP_W, whi, h.y, kk ? 1u : st);
+                            umma_bf16_lo(dcol, xlo + kk * 2, xhi, blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
                         if (two) {
 #pragma unroll
                             for (int kk = 0; kk < B / 16; ++kk)
                                 umma_bf16_lo(dcol + Cfg::HALF_COLS, xlo + SUB_LO + kk * 2, xhi, blo + kk * KSTEP_W,
-                                             whi, h.y, kk ? 1u : st);
+                                             whi, y, kk ? 1u : st);
+                        }
+                    };
+                    issue_run(h0.x, h0.y);
+                    if (nr > 1) issue_run(h0.z, h0.w);
+                    if constexpr (Cfg::HDR_V4 > 1) {
+                        if (nr > 2) {
+                            const uint4 h1 = hs[1];
+                            issue_run(h1.x, h1.y);
+                            if (nr > 3) issue_run(h1.z, h1.w);
                         }
                     }
                     // the slot is free once these MMAs finish
