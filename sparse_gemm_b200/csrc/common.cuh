@@ -69,8 +69,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that may suspend the thread (no instructions issued) until the
+// phase completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the barrier phase with the given parity has completed.
 // Returns false when `timeout_ns` elapsed or another role raised `abort`.
+// A waiting thread sleeps inside try_wait (suspend hint) rather than
+// spinning, so it takes no issue slots from the warps that share its
+// scheduler; the clock and the abort flag are looked at between sleeps.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
                                           const volatile int *abort)
 {
@@ -79,8 +97,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     const uint64_t t0 = globaltimer_ns();
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 128; ++i)  // try_wait suspends briefly; the clock is read rarely
-            if (mbar_try_wait(a, parity)) return true;
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait_suspend(a, parity, 2000u)) return true;
         if (abort && *abort) return false;
         if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
