@@ -197,8 +197,11 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                 }
             }
     };
-    uint32_t xf[KK][NT][2];
-    load_x(col_of(q0), xf);
+    // fragments of a whole stage are loaded one stage ahead (CH blocks in
+    // flight), so the L2 latency is paid once per stage, not once per block
+    uint32_t xf[Cfg::CH][KK][NT][2];
+#pragma unroll
+    for (int cb = 0; cb < Cfg::CH; ++cb) load_x(q0 + cb < q1 ? col_of(q0 + cb) : -1, xf[cb]);
 
     // first block row of the share: last r with row_ptr[r] <= q0, by a
     // warp-parallel search (two or three rounds of one load per lane)
@@ -231,13 +234,16 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
             break;
         }
         const uint32_t stage_addr = smem_u32(ring + s * Cfg::STAGE_BYTES);
+        uint32_t xn[Cfg::CH][KK][NT][2];  // the next stage's fragments
+#pragma unroll
+        for (int cb = 0; cb < Cfg::CH; ++cb) {
+            const int pn = q0 + (t + 1) * Cfg::CH + cb;
+            load_x(pn < q1 ? col_of(pn) : -1, xn[cb]);
+        }
 #pragma unroll
         for (int cb = 0; cb < Cfg::CH; ++cb) {
             const int p = q0 + t * Cfg::CH + cb;
             if (p >= q1) break;
-            // fragments of the next block, one block ahead
-            uint32_t xn[KK][NT][2];
-            load_x(p + 1 < q1 ? col_of(p + 1) : -1, xn);
             while (p >= row_end) {  // leaving block row r
                 if (have) {
                     const bool direct = a.row_ptr[r] >= q0;  // row began inside the share too
@@ -263,17 +269,19 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                     ldmatrix_x4(stage_addr + row * Cfg::ROW_BYTES + swz_chunk<B>(chunk, row) * 16, a0, a1, a2, a3);
 #pragma unroll
                     for (int j = 0; j < NT; ++j)
-                        mma_bf16_16816(acc.d[i][j], a0, a1, a2, a3, xf[kk][j][0], xf[kk][j][1]);
+                        mma_bf16_16816(acc.d[i][j], a0, a1, a2, a3, xf[cb][kk][j][0], xf[cb][kk][j][1]);
                 }
             }
+        }
+#pragma unroll
+        for (int cb = 0; cb < Cfg::CH; ++cb)
 #pragma unroll
             for (int kk = 0; kk < KK; ++kk)
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
-                    xf[kk][j][0] = xn[kk][j][0];
-                    xf[kk][j][1] = xn[kk][j][1];
+                    xf[cb][kk][j][0] = xn[cb][kk][j][0];
+                    xf[cb][kk][j][1] = xn[cb][kk][j][1];
                 }
-        }
         __syncwarp();
         const int tn = t + Cfg::STAGES;
         if (tn < nchunks) {
@@ -319,15 +327,15 @@ __global__ void k_stream_fixup(const StreamArgs a, int GW)
 #pragma unroll
     for (int e = 0; e < PER; ++e) sum[e] = 0.f;
     if (end > beg) {
-        // warp share holding block p: last gw with share_begin(gw) <= p
+        // warp share holding block p: the last gw with share_begin(gw) <= p.
+        // share_begin(gw) = floor(gw * nnz / GW), so gw is within one of
+        // floor(p * GW / nnz); step to the exact one.
         auto warp_of = [&](int p) {
-            int lo = 0, hi = GW;
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (share_begin(mid, GW, a.nnz) <= p) lo = mid;
-                else hi = mid;
-            }
-            return lo;
+            int w = static_cast<int>((static_cast<int64_t>(p) * GW) / a.nnz);
+            w = w < 0 ? 0 : (w > GW - 1 ? GW - 1 : w);
+            while (w > 0 && share_begin(w, GW, a.nnz) > p) --w;
+            while (w + 1 < GW && share_begin(w + 1, GW, a.nnz) <= p) ++w;
+            return w;
         };
         const int w0 = warp_of(beg), w1 = warp_of(end - 1);
         if (w0 == w1) return;  // written directly by its warp
