@@ -380,91 +380,96 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         __syncwarp();
     } else if (warp == Cfg::W_MMA) {
         // ------------------------------------------------------------ MMA issuer
-        // Lane 0 alone: per entry one wait, the header's runs (per 128-row
-        // half and 16-wide K step one MMA each), one commit that frees the slot.
-        if (lane == 0) {
-            Ring ar;
-            int e = 0;
-            bool ok = true, any = false;
-            const uint32_t sbase = smem_u32(slots);
-            const uint64_t xdesc0 = make_sdesc(sbase, 16, Cfg::SBO, Cfg::LAYOUT);
-            const uint64_t wdesc0 = TRANS ? make_sdesc(sbase + Cfg::X_BYTES, Cfg::W_BYTES, Cfg::SBO, Cfg::LAYOUT)
-                                          : make_sdesc(sbase + Cfg::X_BYTES, 16, Cfg::SBO, Cfg::LAYOUT);
-            const uint32_t xlo0 = static_cast<uint32_t>(xdesc0), xhi = static_cast<uint32_t>(xdesc0 >> 32);
-            const uint32_t wlo0 = static_cast<uint32_t>(wdesc0), whi = static_cast<uint32_t>(wdesc0 >> 32);
-            // descriptor address units (16 bytes) per 16-wide K step of the weight operand
-            constexpr uint32_t KSTEP_W = TRANS ? (16 * Cfg::ROW_BYTES) >> 4 : 2;
-            constexpr uint32_t SUB_LO = Cfg::SUB_BYTES >> 4;
-            for (int j = 0;; ++j) {
-                int uid = -1;
-                if (!unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag)) {
+        // The whole warp runs the loop converged (waits, header reads); the
+        // MMAs and commits are issued by lane 0 (a predicate).  Per entry: one
+        // wait, the header's runs (per 128-row half and 16-wide K step one
+        // MMA each), one commit that frees the slot.
+        Ring ar;
+        int e = 0;
+        bool ok = true, any = false;
+        const uint32_t lead = lane == 0 ? 1u : 0u;
+        const uint32_t sbase = smem_u32(slots);
+        const uint64_t xdesc0 = make_sdesc(sbase, 16, Cfg::SBO, Cfg::LAYOUT);
+        const uint64_t wdesc0 = TRANS ? make_sdesc(sbase + Cfg::X_BYTES, Cfg::W_BYTES, Cfg::SBO, Cfg::LAYOUT)
+                                      : make_sdesc(sbase + Cfg::X_BYTES, 16, Cfg::SBO, Cfg::LAYOUT);
+        const uint32_t xlo0 = static_cast<uint32_t>(xdesc0), xhi = static_cast<uint32_t>(xdesc0 >> 32);
+        const uint32_t wlo0 = static_cast<uint32_t>(wdesc0), whi = static_cast<uint32_t>(wdesc0 >> 32);
+        // descriptor address units (16 bytes) per 16-wide K step of the weight operand
+        constexpr uint32_t KSTEP_W = TRANS ? (16 * Cfg::ROW_BYTES) >> 4 : 2;
+        constexpr uint32_t SUB_LO = Cfg::SUB_BYTES >> 4;
+        for (int j = 0;; ++j) {
+            int uid = -1, good = 1;
+            if (lane == 0) good = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag);
+            good = __shfl_sync(0xffffffffu, good, 0);
+            uid = __shfl_sync(0xffffffffu, uid, 0);
+            if (!good) {
+                ok = false;
+                break;
+            }
+            if (uid < 0) break;
+            int mt, g;
+            decode_unit(args, uid, &mt, &g);
+            const bool two = args.M - mt * Cfg::MT > Cfg::BM;  // second 128-row half in range
+            const int z = args.grp_ptr[g], zend = args.grp_ptr[g + 1];
+            if (__any_sync(0xffffffffu, !mbar_wait(&tempty[ar.slot], ar.phase ^ 1, tmo, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d0 = tmem_base + ar.slot * Cfg::ACC_COLS;
+            for (int t = z; t < zend; ++t, ++e) {
+                const int slot = e & (Cfg::S - 1);
+                // the copies are ordered before the MMAs by the barrier itself (both
+                // are async-proxy accesses), so no tcgen05 fence is needed here
+                if (__any_sync(0xffffffffu, !mbar_wait(&full[slot], (e >> Cfg::S_LOG) & 1, tmo, abort_flag))) {
                     ok = false;
                     break;
                 }
-                if (uid < 0) break;
-                int mt, g;
-                decode_unit(args, uid, &mt, &g);
-                const bool two = args.M - mt * Cfg::MT > Cfg::BM;  // second 128-row half in range
-                const int z = args.grp_ptr[g], zend = args.grp_ptr[g + 1];
-                if (!mbar_wait(&tempty[ar.slot], ar.phase ^ 1, tmo, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t d0 = tmem_base + ar.slot * Cfg::ACC_COLS;
-                for (int t = z; t < zend; ++t, ++e) {
-                    const int slot = e & (Cfg::S - 1);
-                    // the copies are ordered before the MMAs by the barrier itself (both
-                    // are async-proxy accesses), so no tcgen05 fence is needed here
-                    if (!mbar_wait(&full[slot], (e >> Cfg::S_LOG) & 1, tmo, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t soff = static_cast<uint32_t>(slot) * (Cfg::SLOT_BYTES >> 4);
-                    const uint32_t xlo = xlo0 + soff, wlo = wlo0 + soff;
-                    const uint4 *hs = hdr + slot * Cfg::HDR_V4;
-                    const uint4 h0 = hs[0];
-                    const int nr = static_cast<int>((h0.x >> 24) & 0xFu);
-                    auto issue_run = [&](uint32_t x, uint32_t y) {
-                        const uint32_t dcol = d0 + (x & 0xFFu);
-                        const uint32_t blo = wlo + ((x >> 8) & 0xFFFFu);
-                        const uint32_t st = x >> 28;
+                const uint32_t soff = static_cast<uint32_t>(slot) * (Cfg::SLOT_BYTES >> 4);
+                const uint32_t xlo = xlo0 + soff, wlo = wlo0 + soff;
+                const uint4 *hs = hdr + slot * Cfg::HDR_V4;
+                const uint4 h0 = hs[0];
+                const int nr = static_cast<int>((h0.x >> 24) & 0xFu);
+                auto issue_run = [&](uint32_t x, uint32_t y) {
+                    const uint32_t dcol = d0 + (x & 0xFFu);
+                    const uint32_t blo = wlo + ((x >> 8) & 0xFFFFu);
+                    const uint32_t st = x >> 28;
+#pragma unroll
+                    for (int kk = 0; kk < B / 16; ++kk)
+                        umma_bf16_lo_lead(lead, dcol, xlo + kk * 2, xhi, blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
+                    if (two) {
 #pragma unroll
                         for (int kk = 0; kk < B / 16; ++kk)
-                            umma_bf16_lo(dcol, xlo + kk * 2, xhi, blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
-                        if (two) {
-#pragma unroll
-                            for (int kk = 0; kk < B / 16; ++kk)
-                                umma_bf16_lo(dcol + Cfg::HALF_COLS, xlo + SUB_LO + kk * 2, xhi, blo + kk * KSTEP_W,
-                                             whi, y, kk ? 1u : st);
-                        }
-                    };
-                    issue_run(h0.x, h0.y);
-                    if (nr > 1) issue_run(h0.z, h0.w);
-                    if constexpr (Cfg::HDR_V4 > 1) {
-                        if (nr > 2) {
-                            const uint4 h1 = hs[1];
-                            issue_run(h1.x, h1.y);
-                            if (nr > 3) issue_run(h1.z, h1.w);
-                        }
+                            umma_bf16_lo_lead(lead, dcol + Cfg::HALF_COLS, xlo + SUB_LO + kk * 2, xhi,
+                                               blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
                     }
-                    // the slot is free once these MMAs finish
-                    umma_commit(&empty[slot]);
-                    any = true;
+                };
+                issue_run(h0.x, h0.y);
+                if (nr > 1) issue_run(h0.z, h0.w);
+                if constexpr (Cfg::HDR_V4 > 1) {
+                    if (nr > 2) {
+                        const uint4 h1 = hs[1];
+                        issue_run(h1.x, h1.y);
+                        if (nr > 3) issue_run(h1.z, h1.w);
+                    }
                 }
-                if (!ok) break;
-                if (zend > z) umma_commit(&tfull[ar.slot]);
-                else mbar_arrive(&tfull[ar.slot]);
-                ar.next(Cfg::ACC);
+                // the slot is free once these MMAs finish
+                umma_commit_lead(lead, &empty[slot]);
+                any = true;
             }
-            if (!ok) {
-                *abort_flag = 1;
-                set_status(args.status, BSL_ERR_TIMEOUT);
-            }
-            if (any) {  // all MMAs of this thread complete before TMEM is freed
-                umma_commit(drain);
-                if (!mbar_wait(drain, 0, tmo, nullptr)) set_status(args.status, BSL_ERR_TIMEOUT);
-            }
+            if (!ok) break;
+            if (zend > z) umma_commit_lead(lead, &tfull[ar.slot]);
+            else if (lane == 0) mbar_arrive(&tfull[ar.slot]);
+            __syncwarp();
+            ar.next(Cfg::ACC);
+        }
+        if (lane == 0 && !ok) {
+            *abort_flag = 1;
+            set_status(args.status, BSL_ERR_TIMEOUT);
+        }
+        if (any) {  // all MMAs of lane 0 complete before TMEM is freed
+            umma_commit_lead(lead, drain);
+            if (lane == 0 && !mbar_wait(drain, 0, tmo, nullptr)) set_status(args.status, BSL_ERR_TIMEOUT);
         }
         __syncwarp();
     } else {
