@@ -224,6 +224,27 @@ def cpu_sample(w: synth.Workload, inp: dict, budget_s: float, kinds: list[str]):
     return done_eff, secs, "; ".join(desc), nthreads
 
 
+# ----------------------------------------------------------------------------- ranks
+# The layer is not sharded: under torchrun every rank runs the whole workload
+# on its own GPU (replicas) and the job's throughput is all ranks' work over
+# the slowest rank's time.  Every rank calls these in the same order.
+
+def max_over_ranks(x, world, device=None):
+    """The largest value of `x` over all ranks (the slowest rank's time)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world, flops_per_step, steps, total_ms):
+    """Weak scaling: TFLOP/s of all ranks' steps over the slowest rank's time."""
+    return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def run_gpu(args):
@@ -368,14 +389,11 @@ def run_gpu(args):
             per_kernel = {"fwd": total_ms / K}
     else:
         per_kernel = {k: total_ms / K / len(kinds) for k in kinds}
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
 
     alg = algorithmic(w, w.nnz)
     flops_step = sum(alg[k]["flops"] for k in kinds)
-    value = world * flops_step * K / (total_ms * 1e-3) / 1e12
+    value = whole_job_value(world, flops_step, K, total_ms)
     ms_per_step = total_ms / K
 
     # dominant kernel + its roofline
@@ -450,10 +468,7 @@ def run_gpu(args):
     ev1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = ev0.elapsed_time(ev1) / ke
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     h2d = X0.numel() * 2 + (dY0.numel() * 2 if train else 0)
     d2h = Y.numel() * 2 + ((dX.numel() + dWv.numel()) * 2 if train else 0)
 
@@ -487,7 +502,7 @@ def run_gpu(args):
         "roofline": roof,
         "dense_cublas_ms_per_step": round(dense_ms, 5),
         "speedup_vs_dense": round(dense_ms / ms_per_step, 3),
-        "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        "e2e": {"value": round(whole_job_value(world, flops_step, 1, e2e_ms), 3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4), "timing": "eager public API calls"},
         "gpu_launches": K * launches_per_step,
