@@ -52,8 +52,8 @@ TRAFFIC = {
                            "src_sha": "d3cf5686545cfe03", "profile": "profiles/k_spmm_tc_fwd_large_fwd.md"},
     ("enc_train_d1.0", "dx"): {"bytes": 29933824, "files": ["spmm_tc.cu", "common.cuh"],
                                "src_sha": "d3cf5686545cfe03", "profile": "profiles/k_spmm_tc_dx_enc_train_d1.md"},
-    ("enc_train_d1.0", "dw"): {"bytes": 31499520, "files": ["sddmm_tc.cu", "common.cuh"],
-                               "src_sha": "630c4a3c2b34703f", "profile": "profiles/k_sddmm_tc_dw_enc_train_d1.md"},
+    ("enc_train_d1.0", "dw"): {"bytes": 31499008, "files": ["sddmm_tc.cu", "common.cuh"],
+                               "src_sha": "f5ed79d6a8ecbef4", "profile": "profiles/k_sddmm_tc_dw_enc_train_d1.md"},
     # k_stream_fwd alone (the fix-up kernel reads and writes well under 1 MB)
     ("decode_fwd", "fwd"): {"bytes": 22754560, "files": ["stream_fwd.cu", "common.cuh"],
                             "src_sha": "4ced2e66adbec8a4", "profile": "profiles/k_stream_fwd_decode_fwd.md"},

@@ -10,9 +10,9 @@
 //
 // MMA shape: the blocks of one block column c share the X strip X[:, c-block],
 // so a work unit ("group") stacks G = 128/b blocks of the same column along
-// MMA M: A = [dY[:, r_1-block] | ... | dY[:, r_G-block]]^T (128 x 64 rows of
+// MMA M: A = [dY[:, r_1-block] | ... | dY[:, r_G-block]]^T (128 x 128 rows of
 // M per stage, MN-major in smem: the dY tiles are loaded untransposed),
-// B = X[:, c-block]^T (b x 64, MN-major), D = 128 x b fp32 in TMEM.  Groups
+// B = X[:, c-block]^T (b x 128, MN-major), D = 128 x b fp32 in TMEM.  Groups
 // are listed per column by the pack's dw_gptr prefix (ceil(count/G) per
 // column); a column's last group may hold fewer than G blocks, and its
 // unused accumulator lanes are never stored.
@@ -28,14 +28,18 @@
 namespace bsl {
 namespace {
 
+// Rows of M per stage: copies are the bottleneck of this kernel (one thread
+// starts only about four per microsecond), so each copy moves a tall strip.
+constexpr int kSddmmRows = 128;
+
 template <int B>
 struct SddmmCfg {
     static constexpr int G = 128 / B;                    // blocks stacked along MMA M
-    static constexpr int MK = 64;                        // rows of M reduced per stage
+    static constexpr int MK = kSddmmRows;                // rows of M reduced per stage
     static constexpr int ROW_BYTES = B * 2;
-    static constexpr int T_BYTES = MK * ROW_BYTES;       // one strip tile (64 x b)
+    static constexpr int T_BYTES = MK * ROW_BYTES;       // one strip tile (MK x b)
     static constexpr int STAGE_BYTES = (G + 1) * T_BYTES;
-    static constexpr int STAGES = 8;
+    static constexpr int STAGES = 4;
     static constexpr int P = 4;                          // producer warps (STAGES % P == 0)
     static constexpr int THREADS = (P + 5) * 32;
     static_assert(STAGES % P == 0, "each stage slot belongs to one producer warp");
@@ -293,13 +297,13 @@ bsl_status launch_sddmm_tc(const void *dY, const void *X, int32_t M, const bsl_b
     const int B = W->b;
     if (W->nnz == 0) return BSL_OK;
     CUtensorMap mdy, mx;
-    if (!make_map_2d(&mdy, dY, W->N, M, static_cast<uint64_t>(W->N) * 2, B, 64, 2 * B) ||
-        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, B, 64, 2 * B))
+    if (!make_map_2d(&mdy, dY, W->N, M, static_cast<uint64_t>(W->N) * 2, B, kSddmmRows, 2 * B) ||
+        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, B, kSddmmRows, 2 * B))
         return BSL_ERR_CUDA;
     SddmmArgs args;
     args.M = M;
     args.C = W->K / B;
-    args.ksteps = (M + 63) / 64;
+    args.ksteps = (M + kSddmmRows - 1) / kSddmmRows;
     args.col_ptr = W->col_ptr;
     args.row_idx = W->row_idx;
     args.csc_to_bsr = W->csc_to_bsr;
