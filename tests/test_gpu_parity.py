@@ -251,6 +251,29 @@ def test_results_are_deterministic():
         assert torch.equal(u.view(torch.int16), v.view(torch.int16))
 
 
+def test_work_counters_return_to_zero():
+    """The persistent kernels take units from counters in the packed weight;
+    after every launch (any M, ragged or not, forward and input gradient,
+    repeated) the counters are back at zero and results are unchanged."""
+    case = synth.random_case(700, 1024, 768, 64, 120, 44)
+    Wp = pack_dev(case, 64)
+    assert torch.count_nonzero(Wp.sched).item() == 0
+    X, dY = to_dev(case["X"]), to_dev(case["dY"])
+    first = None
+    for M in (700, 256, 1, 700):
+        y = sg.forward_tc(X[:M].contiguous(), Wp)
+        dx = sg.backward_input(dY[:M].contiguous(), Wp)
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(Wp.sched).item() == 0, M
+        if M == 700:
+            if first is None:
+                first = (y.clone(), dx.clone())
+            else:
+                assert torch.equal(y.view(torch.int16), first[0].view(torch.int16))
+                assert torch.equal(dx.view(torch.int16), first[1].view(torch.int16))
+    assert sg.device_status(Wp) == 0
+
+
 def test_density_one_matches_cublas():
     M, N, K, b = 512, 1024, 768, 64
     case = synth.random_case(M, N, K, b, (N // b) * (K // b), 43)
