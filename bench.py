@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -49,14 +50,14 @@ L2_BYTES_DEFAULT = 126 * 2 ** 20
 # entry is only used while the kernel source still hashes to `src_sha`.
 TRAFFIC = {
     ("large_fwd", "fwd"): {"bytes": 292852736, "files": ["spmm_tc.cu", "common.cuh"],
-                           "src_sha": "d3cf5686545cfe03", "profile": "profiles/k_spmm_tc_fwd_large_fwd.md"},
+                           "src_sha": "7041d64ad13d53e9", "profile": "profiles/k_spmm_tc_fwd_large_fwd.md"},
     ("enc_train_d1.0", "dx"): {"bytes": 29933824, "files": ["spmm_tc.cu", "common.cuh"],
-                               "src_sha": "d3cf5686545cfe03", "profile": "profiles/k_spmm_tc_dx_enc_train_d1.md"},
+                               "src_sha": "7041d64ad13d53e9", "profile": "profiles/k_spmm_tc_dx_enc_train_d1.md"},
     ("enc_train_d1.0", "dw"): {"bytes": 31499008, "files": ["sddmm_tc.cu", "common.cuh"],
-                               "src_sha": "f5ed79d6a8ecbef4", "profile": "profiles/k_sddmm_tc_dw_enc_train_d1.md"},
+                               "src_sha": "b597a71c38505806", "profile": "profiles/k_sddmm_tc_dw_enc_train_d1.md"},
     # k_stream_fwd alone (the fix-up kernel reads and writes well under 1 MB)
     ("decode_fwd", "fwd"): {"bytes": 22754560, "files": ["stream_fwd.cu", "common.cuh"],
-                            "src_sha": "4ced2e66adbec8a4", "profile": "profiles/k_stream_fwd_decode_fwd.md"},
+                            "src_sha": "fa4f48f3f5bf4d99", "profile": "profiles/k_stream_fwd_decode_fwd.md"},
 }
 
 
@@ -76,10 +77,16 @@ def peaks():
 
 
 def src_sha(*names):
+    """Hash of the kernel sources with comments and blank lines removed, so a
+    traffic figure stays tied to the code it was measured on, not its prose."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "sparse_gemm_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "sparse_gemm_b200", "csrc", n), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+        h.update("\n".join(lines).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,9 +14,9 @@
 // Only stored blocks are touched; output blocks of segments without blocks
 // are written as zeros.
 //
-// Data flow.  On B200 the L2 -> SM fabric (about 20 TB/s in all), not the
-// tensor core, bounds a block-sparse product at low density: every
-// activation tile a block needs must cross it.  Reuse is raised both ways.
+// Data flow.  At low density each stored block needs a whole activation
+// tile, so tile traffic (L2 -> shared memory) and the count of narrow MMAs,
+// not tensor-core arithmetic, set the pace; reuse is raised both ways.
 // A work unit is (256-row tile of M, group of G = 128/b segments); the pack
 // fixed the groups (longest-first order) and merged the members' block
 // coordinates into ascending entries with a member mask.  Per entry one
@@ -35,11 +35,12 @@
 // stored in the swizzled shared-memory image, so they arrive with one 1-D
 // bulk copy.  The producer also writes the entry's MMA runs (TMEM column,
 // block, instruction descriptor, overwrite flag) into a small slot header:
-// one issuing thread is the tensor core's only feeder, so it does nothing
-// per entry but wait, read the header and issue.  One thread starts only about four TMA copies per microsecond,
-// so entry e goes to slot e % S and its copies are issued by producer warp
-// e % P, which owns that slot alone (S a multiple of P): every slot is a
-// single-producer, single-consumer ring.
+// the MMA pipe barely runs ahead of the thread that issues it, so that
+// thread does nothing per entry but wait, read the header and issue.  One
+// thread starts only about four TMA copies per microsecond, so entry e goes
+// to slot e % S and its copies are issued by producer warp e % P, which owns
+// that slot alone (S a multiple of P): every slot is a single-producer,
+// single-consumer ring.
 //
 // Scheduling.  Units are taken from a per-weight atomic counter in the
 // order of decode_unit (heaviest first inside chunks of m-tiles), so the SMs
@@ -53,7 +54,8 @@
 // Roles per CTA (persistent grid, one CTA per SM):
 //   warps 0..P-1   producers: TMA tile copy of the activation tile, bulk
 //                  copy of the entry's weight blocks, into the entry's slot
-//   warp P         TMEM owner; lane 0 issues the MMAs (bf16 in, fp32 in TMEM)
+//   warp P         TMEM owner; runs converged, lane 0 issues the MMAs and commits
+//                  (bf16 in, fp32 accumulators in TMEM)
 //   warps P+1..P+4 epilogue: TMEM -> registers -> bf16 (RNE) -> swizzled smem
 //                  -> TMA store; each warp its own 32 rows of every chunk
 // Every wait is bounded in time; on expiry the kernel records
