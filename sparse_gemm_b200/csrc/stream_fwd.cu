@@ -14,7 +14,8 @@
 // rows swizzled; every warp issues its own copies, since one thread can
 // start only a few copies per microsecond).  The activation slice
 // X[0:MP, c*b:(c+1)*b] of a block is small and stays in L2: its mma.sync
-// fragments are read straight into registers, one block ahead of use.  The
+// fragments are read straight into registers, a whole stage of blocks ahead
+// of use (the L2 latency is paid once per stage, not per block).  The
 // weight block goes to registers with ldmatrix; mma.sync m16n8k16 (bf16 in,
 // fp32 accumulate) forms Y^T[n][m] = W_blk[n][:] . X[m][:], and the partial
 // sum of the current block row stays in registers:
