@@ -123,7 +123,7 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2-D tiled load (no multicast) into this CTA's shared memory; completion is
+// 2-D tiled load into this CTA's own shared memory; completion is
 // signalled on `bar` as transaction bytes.  x is the innermost coordinate.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t x,
                                             int32_t y)
