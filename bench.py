@@ -231,6 +231,38 @@ def cpu_sample(w: synth.Workload, inp: dict, budget_s: float, kinds: list[str]):
     return done_eff, secs, "; ".join(desc), nthreads
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_sample_blockskip(w: synth.Workload, inp: dict, budget_s: float):
+    """Time the oracle's block-skipping forward (only the stored blocks'
+    work) on a bounded sample of token rows; flops counted are the effective
+    2*b*b per stored block and token.  Returns (flops, seconds, description)."""
+    import oracle
+    oracle.build()
+    Xd = oracle.widen(inp["X"])
+    Wt = oracle.dense_weight(inp["W"], inp["mask"], w.b)
+    nthreads = oracle.num_threads()
+    probe = np.arange(min(nthreads, w.M))
+    t0 = time.perf_counter()
+    oracle.forward_blockskip(None, None, inp["mask"], w.b, rows=probe, Xd=Xd, Wt=Wt)
+    t1 = time.perf_counter() - t0
+    n = int(min(w.M, max(1, budget_s / max(t1, 1e-6)) * len(probe)))
+    n = max(1, min(n, w.M))
+    rows = np.random.default_rng(1).choice(w.M, size=n, replace=False)
+    t0 = time.perf_counter()
+    oracle.forward_blockskip(None, None, inp["mask"], w.b, rows=rows, Xd=Xd, Wt=Wt)
+    dt = time.perf_counter() - t0
+    return 2.0 * n * w.b * w.b * w.nnz, dt, f"fwd: {n} of {w.M} token rows"
+
+
 # ----------------------------------------------------------------------------- ranks
 # The layer is not sharded: under torchrun every rank runs the whole workload
 # on its own GPU (replicas) and the job's throughput is all ranks' work over
@@ -345,18 +377,31 @@ def run_gpu(args):
         torch.cuda.synchronize()
         return g
 
-    def replay_ms(g):
+    def replay_times(g, reps):
+        """`reps` timed replays of a K-step graph, each bracketed by a
+        synchronize (and a barrier across ranks) on both sides."""
         g.replay()                      # untimed: first replay uploads the graph
         torch.cuda.synchronize()
-        ev0.record(stream)
-        g.replay()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        return ev0.elapsed_time(ev1)
+        out = []
+        for _ in range(reps):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            g.replay()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            out.append(ev0.elapsed_time(ev1))
+        return out
+
+    def replay_ms(g, reps=None):
+        return statistics.median(replay_times(g, reps or args.replays))
 
     timing = "cuda-graph"
     try:
         g_step = capture(step)
+        # the same K steps on one input copy: operands stay in L2 between steps
+        g_warm = capture(lambda i: step(0))
         kernel_graphs = {}
         if train:
             kernel_graphs["fwd"] = capture(lambda i: sg.forward(Xs[i % ncopy], Wps[i % ncopy], out=Y, workspace=ws))
@@ -372,8 +417,10 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    step_times = None
     if timing == "cuda-graph":
-        total_ms = replay_ms(g_step)
+        step_times = replay_times(g_step, args.replays)
+        total_ms = statistics.median(step_times)
     else:
         ev0.record(stream)
         for i in range(K):
@@ -383,6 +430,7 @@ def run_gpu(args):
         total_ms = ev0.elapsed_time(ev1)
     if world > 1:
         dist.barrier()
+    warm_ms = statistics.median(replay_times(g_warm, args.replays)) if timing == "cuda-graph" else None
     # keep the GPU busy inside the clock window for at least ~0.5 s
     t_end = time.time() + 0.5
     while timing == "cuda-graph" and time.time() < t_end:
@@ -397,6 +445,11 @@ def run_gpu(args):
     else:
         per_kernel = {k: total_ms / K / len(kinds) for k in kinds}
     total_ms = max_over_ranks(total_ms, world, dev)
+    spread = None
+    if step_times:
+        spread = {"replays": len(step_times), "min_ms_per_step": round(min(step_times) / K, 5),
+                  "max_ms_per_step": round(max(step_times) / K, 5),
+                  "median_ms_per_step": round(statistics.median(step_times) / K, 5)}
 
     alg = algorithmic(w, w.nnz)
     flops_step = sum(alg[k]["flops"] for k in kinds)
@@ -535,9 +588,13 @@ def run_gpu(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        done, secs, desc, nthr = cpu_sample(w, inp, args.cpu_budget, kinds)
+        done, secs, desc, nthr = cpu_sample(w, inp, args.cpu_budget * 2 / 3, kinds)
         cpu = {"value": round(done / secs / 1e12, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
-               "sample": desc + f" ({secs:.1f} s, fp64 dense-with-zeros loops)"}
+               "sample": desc + f" ({secs:.1f} s, fp64 dense-with-zeros loops)",
+               "cpu_model": cpu_model()}
+        bdone, bsecs, bdesc = cpu_sample_blockskip(w, inp, args.cpu_budget / 3)
+        cpu["block_skipping"] = {"value": round(bdone / bsecs / 1e12, 8), "unit": UNIT,
+                                 "sample": bdesc + f" ({bsecs:.1f} s, fp64 loops over the stored blocks only)"}
 
     if world > 1:
         dist.destroy_process_group()
@@ -556,6 +613,11 @@ def run_gpu(args):
             "pack_ms": round(statistics.median(pack_ms), 4),
             "timing": timing,
         },
+        "timing_spread": spread,
+        "warm_l2": ({"ms_per_step": round(warm_ms / K, 5),
+                     "value": round(whole_job_value(1, flops_step, K, warm_ms), 3),
+                     "note": "same K steps on one input copy (operands stay in L2); not the headline"}
+                    if warm_ms else None),
         "kernels_ms": {k: round(v, 5) for k, v in per_kernel.items()},
         "roofline": roof,
         "dense_cublas_ms_per_step": round(dense_ms, 5),
@@ -603,7 +665,8 @@ def run_reference(args):
         "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "b": w.b, "nnz": w.nnz,
                    "density": round(w.nnz / (w.R * w.C), 5), "mask": w.mask_kind, "seed": w.seed},
         "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
-                         "sample": descs[0] + " per step"},
+                         "sample": descs[0] + " per step (fp64 dense-with-zeros loops)",
+                         "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -653,6 +716,8 @@ def main():
     ap.add_argument("--reference-budget", type=float, default=120.0)
     ap.add_argument("--kernel-only", choices=["fwd", "dx", "dw"], default=None)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--replays", type=int, default=15,
+                    help="timed replays of the K-step graph; the median is reported")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

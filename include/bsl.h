@@ -173,18 +173,24 @@ BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W
  * of this entry point; it exists only for such callers.
  *
  * The scratch is a fixed array of BSL_NOALLOC_SCRATCH_BYTES in libbsl's own
- * device memory, reserved on every GPU that loads the library until the
- * process exits.  The entry point allocates nothing and calls no
- * cudaMalloc / cudaFree.  It returns BSL_ERR_SCRATCH_TOO_SMALL, launching
+ * device memory.  The CUDA runtime loads the array, like the library's
+ * kernels, the first time it is used on a device: the first call of this
+ * entry point on each device takes those 16 MiB from the device and fails
+ * with BSL_ERR_CUDA if the device has no room left, so make one call at
+ * start-up, before the memory budget is spent.  From then on the device keeps
+ * the array until the process exits.  The entry point allocates nothing
+ * itself and calls no cudaMalloc / cudaFree.  It returns BSL_ERR_SCRATCH_TOO_SMALL, launching
  * nothing, when the call would need more scratch than that (the need is
  * bsl_forward_workspace_bytes(M, W) = SMs x 8 warps x 2 x b x M' x 4 bytes,
  * M' = 16 for M <= 16, else 32; on a 148-SM B200 that is 4.8 MB for b = 32,
  * M <= 16, and 9.7 MB for b = 32, M <= 32 or b = 64, M <= 16, which fit;
  * b = 64 with M > 16 needs 19.4 MB and is rejected).
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress), so make that first call outside any stream
- * capture.  Every call on a device shares the one array, which keeps the
+ * The first call on each device also looks up the array's device address
+ * (cudaGetSymbolAddress) and keeps it for the life of the process, so make
+ * that first call outside any stream capture; calls after the device's
+ * primary context was destroyed and re-created (cudaDeviceReset) are not
+ * supported.  Every call on a device shares the one array, which keeps the
  * previous call's contents; nothing in it has to start at zero (each call
  * writes every partial sum before reading it).  Calls whose kernels overlap
  * on the GPU (different streams without ordering between them) race on the

@@ -57,6 +57,8 @@ def _load():
         lib.bsl_oracle_dense_weight.argtypes = [_i64, _i64, _i64, _p, _p, _p]
         lib.bsl_oracle_widen.argtypes = [_i64, _p, _p]
         lib.bsl_oracle_forward_rows.argtypes = [_i64, _i64, _i64, _p, _p, _p, _i64, _p, _p]
+        lib.bsl_oracle_forward_rows_blockskip.argtypes = [_i64, _i64, _i64, _i64, _p, _p, _p, _p,
+                                                          _i64, _p, _p]
         lib.bsl_oracle_backward_input_rows.argtypes = [_i64, _i64, _i64, _p, _p, _p, _i64, _p, _p]
         lib.bsl_oracle_backward_weight_blocks.argtypes = [_i64, _i64, _i64, _i64, _p, _p,
                                                           _p, _p, _i64, _p, _p]
@@ -102,11 +104,15 @@ def _rows(rows, M):
     return rows
 
 
-def forward(X, W, mask, b, rows=None, *, Xd=None, Wt=None):
-    """Y[rows] = X[rows] Wt^T in fp64, and sum_k |x w| per output.
+def forward(X, W, mask, b, rows=None, *, Xd=None, Wt=None, bias=None):
+    """Y[rows] = X[rows] Wt^T (+ bias) in fp64, and sum_k |x w| (+ |bias|) per output.
 
     ``X``/``W`` are bf16 bit arrays; ``Xd``/``Wt`` may pass already widened
-    operands to skip the conversion.  Returns (Y, Yabs), shape [len(rows), N].
+    operands to skip the conversion.  ``bias`` (bf16 bits, [N]) is the bias
+    of nn.Linear, which BlockSparseLinear replaces as a drop-in (Hugging Face
+    pytorch_block_sparse release note, "Block-Sparse Implementation and
+    Usage"): one added term per output column.  Returns (Y, Yabs), shape
+    [len(rows), N].
     """
     Xd = widen(X) if Xd is None else Xd
     Wt = dense_weight(W, mask, b) if Wt is None else Wt
@@ -117,6 +123,43 @@ def forward(X, W, mask, b, rows=None, *, Xd=None, Wt=None):
     A = np.empty((rows.size, N))
     _load().bsl_oracle_forward_rows(M, N, K, _ptr(Xd), _ptr(Wt), _ptr(rows), rows.size,
                                     _ptr(Y), _ptr(A))
+    if bias is not None:
+        bd = widen(bias).reshape(-1)
+        if bd.size != N:
+            raise ValueError("bias must have N entries")
+        Y += bd[None, :]
+        A += np.abs(bd)[None, :]
+    return Y, A
+
+
+def bias_grad(dY, *, dYd=None):
+    """Gradient of the bias: dbias[n] = sum_m dY[m][n] in fp64 (a column sum,
+    rows added in increasing m), and sum_m |dY[m][n]|.  Returns (dbias, abs)."""
+    dYd = widen(dY) if dYd is None else dYd
+    M, N = dYd.shape
+    s = np.zeros(N)
+    a = np.zeros(N)
+    for m in range(M):
+        s += dYd[m]
+        a += np.abs(dYd[m])
+    return s, a
+
+
+def forward_blockskip(X, W, mask, b, rows=None, *, Xd=None, Wt=None):
+    """The forward of :func:`forward` visiting only the kept blocks (the
+    stored blocks' work only; bit-identical results).  Returns (Y, Yabs)."""
+    Xd = widen(X) if Xd is None else Xd
+    Wt = dense_weight(W, mask, b) if Wt is None else Wt
+    mask = np.ascontiguousarray(mask, dtype=np.uint8)
+    M, K = Xd.shape
+    N = Wt.shape[0]
+    if mask.shape != (N // b, K // b):
+        raise ValueError("mask shape does not match W and b")
+    rows = _rows(rows, M)
+    Y = np.empty((rows.size, N))
+    A = np.empty((rows.size, N))
+    _load().bsl_oracle_forward_rows_blockskip(M, N, K, b, _ptr(Xd), _ptr(Wt), _ptr(mask), _ptr(rows),
+                                              rows.size, _ptr(Y), _ptr(A))
     return Y, A
 
 
@@ -208,57 +251,3 @@ def schedule_order(ptr) -> np.ndarray:
     ptr = [int(v) for v in ptr]
     counts = [ptr[i + 1] - ptr[i] for i in range(len(ptr) - 1)]
     return np.asarray(sorted(range(len(counts)), key=lambda i: (-counts[i], i)), dtype=np.int32)
-
-
-def group_plan(ptr, idx, order, G: int, blk=None):
-    """Work plan of the tensor-core forward (segments = block rows) or input
-    gradient (segments = block columns).
-
-    Segments are taken G at a time in ``order`` (longest first).  For each
-    group, the block coordinates of its members are merged into one
-    ascending list of distinct values ("entries"); each entry records which
-    members hold a block there (bit i = i-th member of the group).  The
-    blocks of the present members are listed entry by entry, members in
-    group order.  ``ptr``/``idx`` are the segment pointer and per-entry
-    coordinate arrays (BSR row_ptr/col_idx, or CSC col_ptr/row_idx); ``blk``
-    maps a segment entry to its BSR block (None: the entry position itself).
-
-    Returns (grp_ptr, grp_bptr, ent, blk_list) with ent = coordinate |
-    (mask << 24).
-    """
-    ptr = [int(v) for v in ptr]
-    idx = [int(v) for v in idx]
-    order = [int(v) for v in order]
-    nseg = len(ptr) - 1
-    ngroups = (nseg + G - 1) // G
-    grp_ptr, grp_bptr, ent, blk_list = [0], [0], [], []
-    for g in range(ngroups):
-        members = order[g * G:(g + 1) * G]
-        coords = {}
-        for i, sgm in enumerate(members):
-            for j in range(ptr[sgm], ptr[sgm + 1]):
-                coords.setdefault(idx[j], {})[i] = j
-        for c in sorted(coords):
-            present = coords[c]
-            mask = 0
-            for i in sorted(present):
-                mask |= 1 << i
-                j = present[i]
-                blk_list.append(j if blk is None else int(blk[j]))
-            ent.append(c | (mask << 24))
-        grp_ptr.append(len(ent))
-        grp_bptr.append(len(blk_list))
-    i32 = lambda v: np.asarray(v, dtype=np.int64).astype(np.int32)
-    return i32(grp_ptr), i32(grp_bptr), i32(ent), i32(blk_list)
-
-
-def dw_group_ptr(col_ptr, group: int) -> np.ndarray:
-    """Exclusive prefix over block columns of ceil(blocks_in_column / group):
-    the weight-gradient kernel processes the blocks of one column in groups
-    of ``group`` (= 128 / b) sharing the column's X strip."""
-    col_ptr = [int(v) for v in col_ptr]
-    out = [0]
-    for c in range(len(col_ptr) - 1):
-        n = col_ptr[c + 1] - col_ptr[c]
-        out.append(out[-1] + (n + group - 1) // group)
-    return np.asarray(out, dtype=np.int32)

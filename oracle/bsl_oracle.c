@@ -87,6 +87,42 @@ void bsl_oracle_forward_rows(int64_t M, int64_t N, int64_t K,
     }
 }
 
+/* The same forward with the masked-out blocks skipped instead of multiplied
+ * as zeros: for output n, only the k inside kept blocks of block row n / b
+ * are visited, still in increasing k.  A skipped term is +-0, which never
+ * changes a double sum that starts at +0, so the result is bit-identical to
+ * bsl_oracle_forward_rows; it is timed beside it as the CPU baseline that
+ * does only the stored blocks' work (the layer computes only the nonzero
+ * blocks: Hugging Face pytorch_block_sparse release note, "Block-Sparse
+ * Implementation and Usage"). */
+void bsl_oracle_forward_rows_blockskip(int64_t M, int64_t N, int64_t K, int64_t b,
+                                       const double *X, const double *Wt, const uint8_t *mask,
+                                       const int64_t *rows, int64_t nrows,
+                                       double *Y, double *Yabs)
+{
+    (void)M;
+    const int64_t C = K / b;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        const double *x = X + rows[i] * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const double *w = Wt + n * K;
+            const uint8_t *mrow = mask + (n / b) * C;
+            double s = 0.0, a = 0.0;
+            for (int64_t c = 0; c < C; ++c) {
+                if (!mrow[c]) continue;
+                for (int64_t k = c * b; k < (c + 1) * b; ++k) {
+                    double t = x[k] * w[k];
+                    s += t;
+                    a += fabs(t);
+                }
+            }
+            Y[i * N + n] = s;
+            Yabs[i * N + n] = a;
+        }
+    }
+}
+
 /* Input gradient on the listed token rows: dX[i][k] = sum_n dY[rows[i]][n] * Wt[n][k].
  * For each output element the terms are added in increasing n. */
 void bsl_oracle_backward_input_rows(int64_t M, int64_t N, int64_t K,

@@ -10,12 +10,15 @@
 // bsl_forward_stream_noalloc runs the same kernels with the scratch taken
 // from a fixed array in this library's own device memory.
 //
-// The array is a file-scope __device__ variable: every GPU that loads the
-// library keeps BSL_NOALLOC_SCRATCH_BYTES of device memory for it until the
-// process exits.  Host code must not use the array's name as a device
-// address (on the host it only names a host-side stand-in), so the device
-// address is looked up once per device with cudaGetSymbolAddress, with that
-// device current, and passed to the kernel.
+// The array is a file-scope __device__ variable.  The runtime loads it on a
+// device the first time this file's module is used there (this entry
+// point's first call on that device), which takes BSL_NOALLOC_SCRATCH_BYTES
+// of device memory and can fail if the device is full; the device then keeps
+// it until the process exits.  Host code must not use the array's name as a
+// device address (on the host it only names a host-side stand-in), so the
+// device address is looked up once per device with cudaGetSymbolAddress,
+// with that device current, cached, and passed to the kernel.  The cache
+// assumes the device's primary context lives as long as the process.
 #include <mutex>
 
 #include "common.cuh"

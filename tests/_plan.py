@@ -1,0 +1,63 @@
+"""Reference builders for the tensor-core kernels' work plans (test helper).
+
+These are layouts of this library's CUDA engine, not definitions from the
+pages, so they live with the tests rather than in the oracle: the GPU tests
+compare the plans that ``bsl_pack`` builds on the device with the ones
+built here by plain loops, and ``test_plan_layout.py`` checks these builders
+against independent properties (every stored block covered exactly once,
+group counts found by walking the columns).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def group_plan(ptr, idx, order, G: int, blk=None):
+    """Plan of the forward (segments = block rows) or input gradient
+    (segments = block columns) engine.
+
+    Segments are taken G at a time in ``order`` (longest first).  For each
+    group the members' block coordinates are merged into one ascending list
+    of distinct values ("entries"); an entry records which members hold a
+    block there (bit i = i-th member).  The blocks of the present members are
+    listed entry by entry, members in group order.  ``blk`` maps a segment
+    position to its BSR block (None: the position itself).
+
+    Returns (grp_ptr, grp_bptr, ent, blk_list) with ent = coordinate | (mask << 24).
+    """
+    ptr = [int(v) for v in ptr]
+    idx = [int(v) for v in idx]
+    order = [int(v) for v in order]
+    nseg = len(ptr) - 1
+    ngroups = (nseg + G - 1) // G
+    grp_ptr, grp_bptr, ent, blk_list = [0], [0], [], []
+    for g in range(ngroups):
+        members = order[g * G:(g + 1) * G]
+        coords = {}
+        for i, sgm in enumerate(members):
+            for j in range(ptr[sgm], ptr[sgm + 1]):
+                coords.setdefault(idx[j], {})[i] = j
+        for c in sorted(coords):
+            present = coords[c]
+            mask = 0
+            for i in sorted(present):
+                mask |= 1 << i
+                j = present[i]
+                blk_list.append(j if blk is None else int(blk[j]))
+            ent.append(c | (mask << 24))
+        grp_ptr.append(len(ent))
+        grp_bptr.append(len(blk_list))
+    i32 = lambda v: np.asarray(v, dtype=np.int64).astype(np.int32)
+    return i32(grp_ptr), i32(grp_bptr), i32(ent), i32(blk_list)
+
+
+def dw_group_ptr(col_ptr, group: int) -> np.ndarray:
+    """Start of each block column's weight-gradient groups: the column's
+    blocks are cut into consecutive runs of ``group`` (the last run may be
+    shorter) and the runs are numbered column after column."""
+    col_ptr = [int(v) for v in col_ptr]
+    out = [0]
+    for c in range(len(col_ptr) - 1):
+        n = col_ptr[c + 1] - col_ptr[c]
+        out.append(out[-1] + (n + group - 1) // group)
+    return np.asarray(out, dtype=np.int32)

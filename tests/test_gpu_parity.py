@@ -13,6 +13,7 @@ import torch
 
 import oracle
 import synth
+from tests import _plan
 from tests._gpu import bits, mask_dev, to_dev, to_f64
 from tests._parity import assert_parity
 
@@ -46,10 +47,10 @@ def check_pack(Wp, case, b):
     assert np.array_equal(bits(Wp.block_values()), want["values"].reshape(nnz, b, b))
     assert np.array_equal(Wp.row_order.cpu().numpy(), oracle.schedule_order(want["row_ptr"]))
     assert np.array_equal(Wp.col_order.cpu().numpy(), oracle.schedule_order(want["col_ptr"]))
-    assert np.array_equal(Wp.dw_gptr.cpu().numpy(), oracle.dw_group_ptr(want["col_ptr"], 128 // b))
+    assert np.array_equal(Wp.dw_gptr.cpu().numpy(), _plan.dw_group_ptr(want["col_ptr"], 128 // b))
     G = 128 // b
-    rplan = oracle.group_plan(want["row_ptr"], want["col_idx"], oracle.schedule_order(want["row_ptr"]), G)
-    cplan = oracle.group_plan(want["col_ptr"], want["row_idx"], oracle.schedule_order(want["col_ptr"]), G,
+    rplan = _plan.group_plan(want["row_ptr"], want["col_idx"], oracle.schedule_order(want["row_ptr"]), G)
+    cplan = _plan.group_plan(want["col_ptr"], want["row_idx"], oracle.schedule_order(want["col_ptr"]), G,
                               blk=want["csc_to_bsr"])
     for pre, plan in (("rgrp", rplan), ("cgrp", cplan)):
         gp, gb, ent, blk = plan
@@ -313,10 +314,35 @@ def test_autograd_function_matches_oracle():
 
 # ----------------------------------------------------- full-size workloads (sampled)
 
-def _sample_rows(M, n, seed):
+def _sample_rows(M, n, seed, tile=128):
+    """Rows checked at full size: the first and last row of every `tile`-row
+    tile of M (every work unit of the tensor-core kernels starts and ends on
+    such a boundary, so a unit that is skipped, duplicated or shifted shows
+    up at its edges), plus `n` random rows."""
     rng = np.random.default_rng(seed)
     rows = {0, M - 1} | set(rng.choice(M, size=min(n, M), replace=False).tolist())
+    for t0 in range(0, M, tile):
+        rows |= {t0, min(M, t0 + tile) - 1}
     return np.array(sorted(rows))
+
+
+def _dw_check_blocks(mask, seed, G):
+    """Blocks checked at full size for the weight gradient: every block of
+    the heaviest block column, every block of a column whose block count is
+    not a multiple of G (the weight-gradient kernel works on G blocks of a
+    column at a time, so this covers a short last group), the first and last
+    block, and a random sample.  Returned as BSR positions."""
+    rr, cc = np.nonzero(mask)                    # BSR order (row-major scan)
+    counts = mask.sum(0)
+    cols = {int(np.argmax(counts))}
+    ragged = [c for c in range(mask.shape[1]) if counts[c] % G]
+    if ragged:
+        cols.add(int(ragged[0]))
+    pick = set(np.nonzero(np.isin(cc, list(cols)))[0].tolist())
+    pick |= {0, len(rr) - 1}
+    rng = np.random.default_rng(seed)
+    pick |= set(rng.choice(len(rr), size=min(24, len(rr)), replace=False).tolist())
+    return np.array(sorted(pick)), rr, cc
 
 
 @pytest.mark.parametrize("name", ["tiny_fwd", "enc_fwd", "large_fwd", "decode_fwd"])
@@ -328,7 +354,7 @@ def test_workload_forward(name):
     Y = sg.forward(X, Wp)          # the entry point bench.py times
     torch.cuda.synchronize()
     assert sg.device_status(Wp) == 0
-    rows = np.arange(w.M) if w.M <= 64 else _sample_rows(w.M, 24, w.seed)
+    rows = np.arange(w.M) if w.M <= 64 else _sample_rows(w.M, 16, w.seed)
     ref, S = oracle.forward(inp["X"], inp["W"], inp["mask"], w.b, rows=rows)
     assert_parity(to_f64(Y[torch.from_numpy(rows).cuda()]), ref, S, name)
 
@@ -350,9 +376,7 @@ def test_workload_training_step(d):
     assert_parity(to_f64(Y[torch.from_numpy(rows).cuda()]), ref, S, "Y")
     ref, S = oracle.backward_input(inp["dY"], inp["W"], inp["mask"], w.b, rows=rows, Wt=Wt)
     assert_parity(to_f64(dX[torch.from_numpy(rows).cuda()]), ref, S, "dX")
-    rr, cc = np.nonzero(inp["mask"])
-    pick = np.random.default_rng(w.seed).choice(len(rr), size=min(24, len(rr)), replace=False)
-    pick = np.unique(np.concatenate([pick, [0, len(rr) - 1]]))
+    pick, rr, cc = _dw_check_blocks(inp["mask"], w.seed, 128 // w.b)
     ref, S = oracle.backward_weight(inp["dY"], inp["X"], inp["mask"], w.b,
                                     blocks=[(int(rr[i]), int(cc[i])) for i in pick])
     got = to_f64(dW[torch.from_numpy(pick).cuda()])

@@ -184,13 +184,6 @@ def test_schedule_order_matches_lexsort(oracle_lib):
     assert np.array_equal(oracle.schedule_order(ptr), want)
 
 
-def test_dw_group_ptr_closed_form(oracle_lib):
-    col_ptr = np.array([0, 0, 1, 5, 9, 10, 17])
-    got = oracle.dw_group_ptr(col_ptr, 4)
-    counts = np.diff(col_ptr)
-    assert np.array_equal(got, np.concatenate([[0], np.cumsum(-(-counts // 4))]))
-
-
 # --------------------------------------------------------------- invariants
 
 def _permute_block_cols(a, perm, b):
@@ -266,6 +259,50 @@ def test_row_subset_equals_full(oracle_lib):
     assert np.array_equal(dXs, dXf[[5, 38]])
 
 
+def test_blockskip_forward_is_bit_identical_and_matches_brute_force(oracle_lib):
+    """The block-skipping forward (the CPU baseline that does only the stored
+    blocks' work) must give the dense-with-zeros result bit for bit, and the
+    exact integer result on integer inputs."""
+    b = 4
+    case = int_case(6, 16, 20, b, 9, 28)
+    got, A = oracle.forward_blockskip(case["X"], case["W"], case["mask"], b)
+    assert np.array_equal(got, brute_forward(case["X"], case["W"], case["mask"].tolist(), b))
+    case = synth.random_case(9, 256, 320, 32, 23, 29, empty_rows=(2,))
+    want, wa = oracle.forward(case["X"], case["W"], case["mask"], 32)
+    got, ga = oracle.forward_blockskip(case["X"], case["W"], case["mask"], 32)
+    assert np.array_equal(got, want) and np.array_equal(ga, wa)
+
+
+def test_bias_matches_integer_brute_force(oracle_lib):
+    """Y = X Wt^T + bias and dbias = column sums of dY, against Python ints."""
+    b = 4
+    case = int_case(6, 16, 12, b, 5, 30)
+    bias = synth.bf16_bits(np.random.default_rng(30).integers(-3, 4, size=16).astype(np.float32))
+    Y, A = oracle.forward(case["X"], case["W"], case["mask"], b, bias=bias)
+    want = brute_forward(case["X"], case["W"], case["mask"].tolist(), b) + as_int(bias)[None, :]
+    assert np.array_equal(Y, want)
+    Y0, A0 = oracle.forward(case["X"], case["W"], case["mask"], b)
+    assert np.array_equal(A, A0 + np.abs(as_int(bias))[None, :])
+    dYi = as_int(case["dY"])[:, :16]
+    db, dba = oracle.bias_grad(case["dY"][:, :16].copy())
+    assert db.tolist() == [sum(int(dYi[m][n]) for m in range(6)) for n in range(16)]
+    assert dba.tolist() == [sum(abs(int(dYi[m][n])) for m in range(6)) for n in range(16)]
+
+
+def test_bias_adjoint_identity(oracle_lib):
+    """<dY, Y(bias)> = <dY, Y(0)> + <dbias, bias>: pins the bias term and its
+    gradient against each other (exact on integers)."""
+    b = 4
+    case = int_case(7, 12, 8, b, 4, 31)
+    bias = synth.bf16_bits(np.random.default_rng(31).integers(-3, 4, size=12).astype(np.float32))
+    dY = case["dY"][:, :12].copy()
+    Yb, _ = oracle.forward(case["X"], case["W"], case["mask"], b, bias=bias)
+    Y0, _ = oracle.forward(case["X"], case["W"], case["mask"], b)
+    db, _ = oracle.bias_grad(dY)
+    dyd = oracle.widen(dY)
+    assert float((dyd * Yb).sum()) == float((dyd * Y0).sum()) + float((db * oracle.widen(bias)).sum())
+
+
 # ----------------------------------------------------------- planted mistakes
 
 def _mutants():
@@ -293,6 +330,31 @@ def _mutants():
     return [transposed_mask, mask_ignored, last_block_dropped, sign_flipped, operand_shifted]
 
 
+def _bias_mutants():
+    """Copies of the oracle's biased forward with one plausible mistake each."""
+    def bias_ignored(X, W, mask, b, bias):
+        return oracle.forward(X, W, mask, b)[0]
+
+    def bias_reversed(X, W, mask, b, bias):
+        return oracle.forward(X, W, mask, b, bias=bias[::-1].copy())[0]
+
+    def bias_twice(X, W, mask, b, bias):
+        Y, _ = oracle.forward(X, W, mask, b, bias=bias)
+        return Y + oracle.widen(bias)[None, :]
+
+    return [bias_ignored, bias_reversed, bias_twice]
+
+
+@pytest.mark.parametrize("mutant", _bias_mutants(), ids=lambda f: f.__name__)
+def test_bias_pin_catches_planted_mistakes(oracle_lib, mutant):
+    b = 4
+    case = int_case(5, 16, 16, b, 7, 32)
+    bias = synth.bf16_bits(np.arange(-8, 8).astype(np.float32))
+    want = brute_forward(case["X"], case["W"], case["mask"].tolist(), b) + as_int(bias)[None, :]
+    assert np.array_equal(oracle.forward(case["X"], case["W"], case["mask"], b, bias=bias)[0], want)
+    assert not np.array_equal(mutant(case["X"], case["W"], case["mask"], b, bias), want)
+
+
 @pytest.mark.parametrize("mutant", _mutants(), ids=lambda f: f.__name__)
 def test_pins_catch_planted_mistakes(oracle_lib, mutant):
     b = 4
@@ -300,37 +362,3 @@ def test_pins_catch_planted_mistakes(oracle_lib, mutant):
     want = brute_forward(case["X"], case["W"], case["mask"].tolist(), b)
     assert np.array_equal(oracle.forward(case["X"], case["W"], case["mask"], b)[0], want)
     assert not np.array_equal(mutant(case["X"], case["W"], case["mask"], b), want)
-
-
-def test_group_plan_covers_every_block_once(oracle_lib):
-    """Each stored block appears exactly once, under its own coordinate and
-    member, and entries are strictly ascending inside a group."""
-    b, R, C, G = 4, 11, 9, 4
-    mask = synth.mask_uniform(R, C, 37, np.random.default_rng(31))
-    mask[5, :] = 0
-    W = synth.bf16_bits(np.random.default_rng(31).standard_normal((R * b, C * b), dtype=np.float32))
-    pk = oracle.pack(W, mask, b)
-    order = oracle.schedule_order(pk["row_ptr"])
-    gp, gb, ent, blk = oracle.group_plan(pk["row_ptr"], pk["col_idx"], order, G)
-    assert sorted(blk.tolist()) == list(range(pk["nnz"]))
-    seen = set()
-    for g in range(len(gp) - 1):
-        members = order[g * G:(g + 1) * G]
-        cols = [int(e) & 0xFFFFFF for e in ent[gp[g]:gp[g + 1]]]
-        assert cols == sorted(set(cols))
-        q = gb[g]
-        for e in ent[gp[g]:gp[g + 1]]:
-            c, m = int(e) & 0xFFFFFF, int(e) >> 24
-            for i in range(G):
-                if m >> i & 1:
-                    p = blk[q]
-                    q += 1
-                    r = members[i]
-                    assert pk["row_ptr"][r] <= p < pk["row_ptr"][r + 1] and pk["col_idx"][p] == c
-                    seen.add((r, c))
-        assert q == gb[g + 1]
-    assert seen == set(zip(*np.nonzero(mask)))
-    # transposed plan over the CSC index maps to the same blocks
-    corder = oracle.schedule_order(pk["col_ptr"])
-    gp, gb, ent, blk = oracle.group_plan(pk["col_ptr"], pk["row_idx"], corder, G, blk=pk["csc_to_bsr"])
-    assert sorted(blk.tolist()) == list(range(pk["nnz"]))

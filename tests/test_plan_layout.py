@@ -1,0 +1,66 @@
+"""CPU checks of the plan builders in tests/_plan.py (the reference the GPU
+tests hold the device-built plans to).  Each is checked against a property
+found independently: a walk over the stored blocks, not the same formula."""
+import numpy as np
+
+import oracle
+import synth
+from tests import _plan
+
+
+def test_group_plan_covers_every_block_once(oracle_lib):
+    """Each stored block appears exactly once, under its own coordinate and
+    member, and entries are strictly ascending inside a group."""
+    b, R, C, G = 4, 11, 9, 4
+    mask = synth.mask_uniform(R, C, 37, np.random.default_rng(31))
+    mask[5, :] = 0
+    W = synth.bf16_bits(np.random.default_rng(31).standard_normal((R * b, C * b), dtype=np.float32))
+    pk = oracle.pack(W, mask, b)
+    order = oracle.schedule_order(pk["row_ptr"])
+    gp, gb, ent, blk = _plan.group_plan(pk["row_ptr"], pk["col_idx"], order, G)
+    assert sorted(blk.tolist()) == list(range(pk["nnz"]))
+    seen = set()
+    for g in range(len(gp) - 1):
+        members = order[g * G:(g + 1) * G]
+        cols = [int(e) & 0xFFFFFF for e in ent[gp[g]:gp[g + 1]]]
+        assert cols == sorted(set(cols))
+        q = gb[g]
+        for e in ent[gp[g]:gp[g + 1]]:
+            c, m = int(e) & 0xFFFFFF, int(e) >> 24
+            for i in range(G):
+                if m >> i & 1:
+                    p = blk[q]
+                    q += 1
+                    r = members[i]
+                    assert pk["row_ptr"][r] <= p < pk["row_ptr"][r + 1] and pk["col_idx"][p] == c
+                    seen.add((r, c))
+        assert q == gb[g + 1]
+    assert seen == set(zip(*np.nonzero(mask)))
+    # transposed plan over the CSC index maps to the same blocks
+    corder = oracle.schedule_order(pk["col_ptr"])
+    gp, gb, ent, blk = _plan.group_plan(pk["col_ptr"], pk["row_idx"], corder, G, blk=pk["csc_to_bsr"])
+    assert sorted(blk.tolist()) == list(range(pk["nnz"]))
+
+
+def test_dw_group_ptr_by_walking_the_columns():
+    """Walk the mask column by column, opening a new group at the first
+    block of a column and after every `group` blocks; the group index at
+    which each column starts must be what dw_group_ptr gives."""
+    rng = np.random.default_rng(17)
+    for group in (1, 2, 4):
+        mask = (rng.random((23, 9)) < 0.45).astype(np.uint8)
+        mask[:, 3] = 0            # an empty column
+        mask[:, 5] = 1            # a full column (23 blocks: not a multiple of 2 or 4)
+        starts, ngroups = [], 0
+        for c in range(mask.shape[1]):
+            starts.append(ngroups)
+            in_group = group      # forces a new group at the column's first block
+            for r in range(mask.shape[0]):
+                if mask[r, c]:
+                    if in_group == group:
+                        ngroups += 1
+                        in_group = 0
+                    in_group += 1
+        starts.append(ngroups)
+        col_ptr = np.concatenate([[0], np.cumsum(mask.sum(0))])
+        assert np.array_equal(_plan.dw_group_ptr(col_ptr, group), np.array(starts)), group
