@@ -103,18 +103,11 @@ typedef struct {
     int32_t *cgrp_bptr;   /* [ceil(C/G)+1] */
     int32_t *cgrp_ent;    /* [nnz] */
     int32_t *cgrp_blk;    /* [nnz] */
-    /* Copies of the block values in the order the tensor-core kernels read
-     * them (rgrp_blk / cgrp_blk order), each block stored as the image the
-     * tensor core expects in shared memory: row-major b x b bf16 with the
-     * 16-byte chunks of row i permuted to chunk j ^ (i % 8) for b = 64 or
-     * j ^ ((i / 2) % 4) for b = 32.  One entry's blocks are then a single
-     * contiguous copy.  Written by bsl_pack. */
-    void *values_rg;      /* bf16 [nnz][b][b] */
-    void *values_cg;      /* bf16 [nnz][b][b] */
     int32_t *status;      /* [1] device status word; must be zeroed once at allocation */
-    int32_t *sched;       /* [8] work counters of the persistent tensor-core kernels; zeroed by
-                           * bsl_pack and left at zero by every kernel that uses them, so the
-                           * kernels of one weight must run in stream order (not concurrently) */
+    int32_t *sched;       /* [8] work counters of the persistent tensor-core kernels, zeroed on
+                           * the call's stream before each launch (contents on entry do not
+                           * matter).  Two calls of the same contraction on one weight must not
+                           * run at the same time: they would share a counter. */
 } bsl_bsr;
 
 /* Human-readable name of a status code (static string). */
@@ -140,12 +133,15 @@ BSL_API bsl_status bsl_pack_count(const uint8_t *mask, int32_t R, int32_t C, int
  * past its size.  A masked-in block is stored even if all its values are 0. */
 BSL_API bsl_status bsl_pack(const void *W, const uint8_t *mask, const bsl_bsr *out, void *stream);
 
-/* Y [M][N] = X [M][K] . W~^T.  Picks the weight-streaming kernel for
- * M <= bsl_small_m_max() and the tensor-core kernel otherwise.  workspace:
- * device scratch of bsl_forward_workspace_bytes(M, W) bytes (may be NULL
- * when that size is 0). */
-BSL_API bsl_status bsl_forward(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *workspace,
-                       size_t workspace_bytes, void *stream);
+/* Y [M][N] = X [M][K] . W~^T (+ bias).  BlockSparseLinear is a drop-in for
+ * nn.Linear (release note, "Block-Sparse Implementation and Usage"), so the
+ * forward takes nn.Linear's bias: bias is bf16 [N] added to every row of Y
+ * in fp32 before the one rounding to bf16, or NULL for none.  Picks the
+ * weight-streaming kernel for M <= bsl_small_m_max() and the tensor-core
+ * kernel otherwise.  workspace: device scratch of
+ * bsl_forward_workspace_bytes(M, W) bytes (may be NULL when that size is 0). */
+BSL_API bsl_status bsl_forward(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y,
+                       void *workspace, size_t workspace_bytes, void *stream);
 
 /* Largest M routed to the weight-streaming kernel by bsl_forward. */
 BSL_API int32_t bsl_small_m_max(void);
@@ -154,15 +150,18 @@ BSL_API int32_t bsl_small_m_max(void);
 BSL_API size_t bsl_forward_workspace_bytes(int32_t M, const bsl_bsr *W);
 
 /* Tensor-core forward for any M >= 1 (persistent tcgen05 kernel; TMA
- * loads of X tiles and weight blocks, fp32 accumulators in TMEM). */
-BSL_API bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *stream);
+ * loads of X tiles and weight blocks, fp32 accumulators in TMEM).  bias:
+ * bf16 [N] or NULL, as for bsl_forward. */
+BSL_API bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y,
+                          void *stream);
 
 /* Weight-streaming forward ("load and sparse expand", lecture summary at
  * 48:12) for 1 <= M <= bsl_small_m_max(): each warp streams a contiguous,
  * equal share of the packed blocks once; block rows split between warps
  * are summed in a fixed order.  workspace: bsl_forward_workspace_bytes(M, W)
- * bytes; contents on entry do not matter. */
-BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, void *Y,
+ * bytes; contents on entry do not matter.  bias: bf16 [N] or NULL, as for
+ * bsl_forward. */
+BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y,
                               void *workspace, size_t workspace_bytes, void *stream);
 
 /* Same computation and kernels as bsl_forward_stream, for callers that cannot
@@ -205,6 +204,14 @@ BSL_API bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *
  * order (sampled dense-dense product over M; tensor-core kernel). */
 BSL_API bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const bsl_bsr *W,
                                void *dW_values, void *stream);
+
+/* dbias [N] = sum over the M rows of dY [M][N]: the gradient of the forward's
+ * bias (nn.Linear's bias, which BlockSparseLinear keeps as a drop-in;
+ * release note, "Block-Sparse Implementation and Usage").  fp32 sums in a
+ * fixed order (identical results run to run), rounded once to bf16.  N must
+ * be a multiple of 32; dbias is bf16 [N], 16-byte aligned.  Needs no
+ * scratch. */
+BSL_API bsl_status bsl_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, void *stream);
 
 /* SYNCHRONOUS: waits for the stream, copies the device status word of W to
  * *status_host (a bsl_status value) and resets it to BSL_OK. */

@@ -23,8 +23,8 @@ __all__ = [
     "BslError", "BsrWeight", "library", "count_blocks", "pack", "forward", "forward_tc",
     "forward_stream", "forward_workspace_bytes", "backward_input", "backward_weight",
     "device_status", "set_wait_timeout_us", "debug_wait_timeout", "small_m_max",
-    "forward_stream_noalloc",
-    "BlockSparseLinearFunction",
+    "forward_stream_noalloc", "bias_grad",
+    "BlockSparseLinearFunction", "BlockSparseLinear",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -49,7 +49,7 @@ class _BSR(ctypes.Structure):
         (name, ctypes.c_void_p) for name in
         ("row_ptr", "col_idx", "values", "col_ptr", "row_idx", "csc_to_bsr", "row_order",
          "col_order", "dw_gptr", "rgrp_ptr", "rgrp_bptr", "rgrp_ent", "rgrp_blk", "cgrp_ptr",
-         "cgrp_bptr", "cgrp_ent", "cgrp_blk", "values_rg", "values_cg", "status", "sched")]
+         "cgrp_bptr", "cgrp_ent", "cgrp_blk", "status", "sched")]
 
 
 _lib = None
@@ -69,11 +69,12 @@ def library() -> ctypes.CDLL:
             "bsl_last_cuda_error": (ctypes.c_char_p, []),
             "bsl_pack_count": (ctypes.c_int, [P, I32, I32, P, ctypes.POINTER(I32), P]),
             "bsl_pack": (ctypes.c_int, [P, P, BP, P]),
-            "bsl_forward": (ctypes.c_int, [P, I32, BP, P, P, SZ, P]),
+            "bsl_forward": (ctypes.c_int, [P, I32, BP, P, P, P, SZ, P]),
             "bsl_small_m_max": (I32, []),
             "bsl_forward_workspace_bytes": (SZ, [I32, BP]),
-            "bsl_forward_tc": (ctypes.c_int, [P, I32, BP, P, P]),
-            "bsl_forward_stream": (ctypes.c_int, [P, I32, BP, P, P, SZ, P]),
+            "bsl_forward_tc": (ctypes.c_int, [P, I32, BP, P, P, P]),
+            "bsl_forward_stream": (ctypes.c_int, [P, I32, BP, P, P, P, SZ, P]),
+            "bsl_bias_grad": (ctypes.c_int, [P, I32, I32, P, P]),
             "bsl_backward_input": (ctypes.c_int, [P, I32, BP, P, P]),
             "bsl_backward_weight": (ctypes.c_int, [P, P, I32, BP, P, P]),
             "bsl_get_device_status": (ctypes.c_int, [BP, ctypes.POINTER(I32), P]),
@@ -136,8 +137,6 @@ class BsrWeight:
         self.cgrp_bptr = torch.empty(ncg + 1, **i32)
         self.cgrp_ent = torch.empty(max(nnz, 1), **i32)
         self.cgrp_blk = torch.empty(max(nnz, 1), **i32)
-        self.values_rg = torch.empty((max(nnz, 1), b, b), dtype=torch.bfloat16, device=device)
-        self.values_cg = torch.empty((max(nnz, 1), b, b), dtype=torch.bfloat16, device=device)
         self.status = torch.zeros(1, **i32)
         self.sched = torch.zeros(8, **i32)
         self._c = _BSR(self.N, self.K, self.b, self.nnz,
@@ -146,8 +145,7 @@ class BsrWeight:
                                                 self.col_order, self.dw_gptr, self.rgrp_ptr,
                                                 self.rgrp_bptr, self.rgrp_ent, self.rgrp_blk,
                                                 self.cgrp_ptr, self.cgrp_bptr, self.cgrp_ent,
-                                                self.cgrp_blk, self.values_rg, self.values_cg,
-                                                self.status, self.sched)])
+                                                self.cgrp_blk, self.status, self.sched)])
 
     @property
     def R(self):
@@ -164,6 +162,25 @@ class BsrWeight:
     def block_values(self) -> torch.Tensor:
         """Packed values [nnz, b, b] (empty view when nnz == 0)."""
         return self.values[: self.nnz]
+
+    def repack(self, W: torch.Tensor, mask: torch.Tensor) -> "BsrWeight":
+        """Re-pack a new dense weight and block mask with the same number of
+        kept blocks into this weight's existing device arrays (no
+        allocation, the tensors keep their addresses): the pattern can move
+        during training (release note, "Future Development Roadmap"; torchao
+        README, "Pruning Criteria", out-of-place mask updates) while every
+        buffer, CUDA graph and optimizer state that refers to it stays
+        valid.  Raises if the mask keeps a different number of blocks."""
+        _cuda_bf16_2d(W, "W", self.K)
+        if W.shape[0] != self.N:
+            raise ValueError(f"W has {W.shape[0]} rows, expected {self.N}")
+        m = _mask_u8(mask, self.R, self.C)
+        n = count_blocks(m)
+        if n != self.nnz:
+            raise ValueError(f"mask keeps {n} blocks; this weight holds {self.nnz}")
+        _check(library().bsl_pack(W.data_ptr(), m.data_ptr(), self.cref(), _stream(W)), "bsl_pack")
+        self._mask = m
+        return self
 
     def cref(self):
         return ctypes.byref(self._c)
@@ -211,10 +228,22 @@ def _out(M, cols, like):
     return torch.empty((M, cols), dtype=torch.bfloat16, device=like.device)
 
 
+def _bias_ptr(bias, N: int, like: torch.Tensor):
+    if bias is None:
+        return None
+    if not (isinstance(bias, torch.Tensor) and bias.is_cuda and bias.dtype == torch.bfloat16
+            and bias.dim() == 1 and bias.shape[0] == N and bias.is_contiguous()):
+        raise TypeError(f"bias must be a contiguous 1-D bfloat16 CUDA tensor of {N} entries")
+    if bias.device != like.device:
+        raise ValueError("bias must be on the same device as X")
+    return bias.data_ptr()
+
+
 def forward(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None,
-            workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """Y = X W^T, kernel chosen by M (weight streaming for M <= small_m_max())."""
+            workspace: torch.Tensor | None = None, bias: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T (+ bias), kernel chosen by M (weight streaming for M <= small_m_max())."""
     _cuda_bf16_2d(X, "X", Wp.K)
+    bptr = _bias_ptr(bias, Wp.N, X)
     M = X.shape[0]
     Y = _out(M, Wp.N, X) if out is None else out
     nbytes = forward_workspace_bytes(M, Wp)
@@ -222,30 +251,34 @@ def forward(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None,
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
     wptr = workspace.data_ptr() if workspace is not None else None
     wlen = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(library().bsl_forward(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), wptr, wlen, _stream(X)),
+    _check(library().bsl_forward(X.data_ptr(), M, Wp.cref(), bptr, Y.data_ptr(), wptr, wlen, _stream(X)),
            "bsl_forward")
     return Y
 
 
-def forward_tc(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None) -> torch.Tensor:
-    """Y = X W^T on the tensor-core kernel (any M)."""
+def forward_tc(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None,
+               bias: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T (+ bias) on the tensor-core kernel (any M)."""
     _cuda_bf16_2d(X, "X", Wp.K)
+    bptr = _bias_ptr(bias, Wp.N, X)
     M = X.shape[0]
     Y = _out(M, Wp.N, X) if out is None else out
-    _check(library().bsl_forward_tc(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), _stream(X)), "bsl_forward_tc")
+    _check(library().bsl_forward_tc(X.data_ptr(), M, Wp.cref(), bptr, Y.data_ptr(), _stream(X)),
+           "bsl_forward_tc")
     return Y
 
 
 def forward_stream(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None,
-                   workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """Y = X W^T on the weight-streaming kernel (M <= small_m_max())."""
+                   workspace: torch.Tensor | None = None, bias: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T (+ bias) on the weight-streaming kernel (M <= small_m_max())."""
     _cuda_bf16_2d(X, "X", Wp.K)
+    bptr = _bias_ptr(bias, Wp.N, X)
     M = X.shape[0]
     Y = _out(M, Wp.N, X) if out is None else out
     nbytes = forward_workspace_bytes(M, Wp)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=X.device)
-    _check(library().bsl_forward_stream(X.data_ptr(), M, Wp.cref(), Y.data_ptr(), workspace.data_ptr(),
+    _check(library().bsl_forward_stream(X.data_ptr(), M, Wp.cref(), bptr, Y.data_ptr(), workspace.data_ptr(),
                                         workspace.numel() * workspace.element_size(), _stream(X)),
            "bsl_forward_stream")
     return Y
@@ -287,6 +320,15 @@ def backward_weight(dY: torch.Tensor, X: torch.Tensor, Wp: BsrWeight,
     return dW[: Wp.nnz]
 
 
+def bias_grad(dY: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """dbias = column sums of dY [M, N] (the gradient of the forward's bias), bf16 [N]."""
+    _cuda_bf16_2d(dY, "dY")
+    M, N = dY.shape
+    db = torch.empty(N, dtype=torch.bfloat16, device=dY.device) if out is None else out
+    _check(library().bsl_bias_grad(dY.data_ptr(), M, N, db.data_ptr(), _stream(dY)), "bsl_bias_grad")
+    return db
+
+
 def device_status(Wp: BsrWeight) -> int:
     """Read and clear the device status word (synchronises the stream)."""
     out = ctypes.c_int32(0)
@@ -308,17 +350,24 @@ def debug_wait_timeout(status: torch.Tensor, us: int) -> None:
 
 
 class BlockSparseLinearFunction(torch.autograd.Function):
-    """Autograd wrapper: forward Y = X W^T; backward dX and dW at kept blocks.
+    """Autograd wrapper: forward Y = X W^T (+ bias); backward dX, dW at the
+    kept blocks and dbias.
 
-    ``values`` is the packed weight's value tensor (the parameter being
-    trained); its gradient is returned in the same [nnz, b, b] layout.
+    ``values`` must be the packed weight's own value tensor
+    (``Wp.block_values()``, the parameter being trained: the kernels read
+    the weight from it, so an in-place update is seen by the next call); its
+    gradient comes back in the same [nnz, b, b] layout.  ``bias`` is a bf16
+    [N] tensor or None.
     """
 
     @staticmethod
-    def forward(ctx, X, values, Wp):
+    def forward(ctx, X, values, Wp, bias=None):
+        if values.data_ptr() != Wp.values.data_ptr():
+            raise ValueError("values must be the packed weight's block_values()")
         ctx.save_for_backward(X)
         ctx.Wp = Wp
-        return forward(X.contiguous(), Wp)
+        ctx.has_bias = bias is not None
+        return forward(X.contiguous(), Wp, bias=bias)
 
     @staticmethod
     def backward(ctx, dY):
@@ -327,4 +376,46 @@ class BlockSparseLinearFunction(torch.autograd.Function):
         dY = dY.contiguous()
         dX = backward_input(dY, Wp) if ctx.needs_input_grad[0] else None
         dW = backward_weight(dY, X.contiguous(), Wp) if ctx.needs_input_grad[1] else None
-        return dX, dW, None
+        db = bias_grad(dY) if ctx.has_bias and ctx.needs_input_grad[3] else None
+        return dX, dW, None, db
+
+
+class BlockSparseLinear(torch.nn.Module):
+    """Drop-in for ``torch.nn.Linear`` with a block-sparse weight (Hugging
+    Face pytorch_block_sparse release note, "Block-Sparse Implementation and
+    Usage"): ``in_features`` -> ``out_features``, weight kept as its b x b
+    blocks under a block mask, optional bias, bf16 on an sm_100 GPU.
+
+    Build it from a dense weight (zeros in place or not) and a block mask
+    with :meth:`from_dense`.  The trainable parameters are ``values`` (the
+    packed blocks, [nnz, b, b], BSR order) and ``bias`` ([out_features]).
+    Inputs may have any leading dimensions; the last one is in_features.
+    """
+
+    def __init__(self, packed: BsrWeight, bias: torch.Tensor | None = None):
+        super().__init__()
+        self.packed = packed
+        self.in_features, self.out_features = packed.K, packed.N
+        self.values = torch.nn.Parameter(packed.block_values(), requires_grad=True)
+        if bias is not None:
+            if bias.shape != (packed.N,):
+                raise ValueError("bias must have out_features entries")
+            bias = torch.nn.Parameter(bias.detach().to(device=packed.device, dtype=torch.bfloat16).contiguous())
+        self.bias = bias
+
+    @classmethod
+    def from_dense(cls, weight: torch.Tensor, mask: torch.Tensor, block: int,
+                   bias: torch.Tensor | None = None) -> "BlockSparseLinear":
+        return cls(pack(weight.detach().to(torch.bfloat16).contiguous(), mask, block), bias)
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        x2 = x.reshape(-1, self.in_features)
+        if x2.dtype != torch.bfloat16:
+            x2 = x2.to(torch.bfloat16)
+        y = BlockSparseLinearFunction.apply(x2, self.values, self.packed, self.bias)
+        return y.reshape(*lead, self.out_features)
+
+    def extra_repr(self) -> str:
+        return (f"in_features={self.in_features}, out_features={self.out_features}, "
+                f"block={self.packed.b}, nnz_blocks={self.packed.nnz}, bias={self.bias is not None}")

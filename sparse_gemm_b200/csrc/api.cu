@@ -100,8 +100,6 @@ bsl_status check_bsr(const bsl_bsr *W)
         for (const void *p : nz)
             if (!p || !aligned(p, 4)) return BSL_ERR_INVALID_ARG;
         if (!W->values || !aligned(W->values, 16)) return BSL_ERR_INVALID_ARG;
-        if (!W->values_rg || !aligned(W->values_rg, 16) || !W->values_cg || !aligned(W->values_cg, 16))
-            return BSL_ERR_INVALID_ARG;
     }
     return BSL_OK;
 }
@@ -165,6 +163,26 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) note_driver_error(static_cast<int>(r));
+    return r == CUDA_SUCCESS;
+}
+
+bool make_block_map(CUtensorMap *map, const void *values, int32_t b, int32_t nblocks, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        note_driver_error(999);
+        return false;
+    }
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(b), static_cast<cuuint64_t>(b),
+                                static_cast<cuuint64_t>(nblocks > 0 ? nblocks : 1)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(b) * 2, static_cast<cuuint64_t>(b) * b * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(b), box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(values), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          b == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) note_driver_error(static_cast<int>(r));
     return r == CUDA_SUCCESS;
 }
@@ -249,33 +267,36 @@ size_t bsl_forward_workspace_bytes(int32_t M, const bsl_bsr *W)
     return stream_workspace_bytes(M, W);
 }
 
-bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *stream)
+bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, void *stream)
 {
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 16)) return BSL_ERR_INVALID_ARG;
     BSL_TRY(bind_device(X));
     BSL_TRY(check_device());
-    return launch_spmm_tc(X, M, W->K, W, false, Y, W->N, static_cast<cudaStream_t>(stream));
+    return launch_spmm_tc(X, M, W->K, W, false, bias, Y, W->N, static_cast<cudaStream_t>(stream));
 }
 
-bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *workspace,
-                              size_t workspace_bytes, void *stream)
+bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y,
+                              void *workspace, size_t workspace_bytes, void *stream)
 {
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 16)) return BSL_ERR_INVALID_ARG;
     if (M > kSmallMMax) return BSL_ERR_UNSUPPORTED;
     BSL_TRY(bind_device(X));
     BSL_TRY(check_device());
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < stream_workspace_bytes(M, W))
         return BSL_ERR_INVALID_ARG;
-    return launch_stream_fwd(X, M, W, Y, workspace, static_cast<cudaStream_t>(stream));
+    return launch_stream_fwd(X, M, W, bias, Y, workspace, static_cast<cudaStream_t>(stream));
 }
 
-bsl_status bsl_forward(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *workspace,
+bsl_status bsl_forward(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, void *workspace,
                        size_t workspace_bytes, void *stream)
 {
-    if (M > 0 && M <= kSmallMMax) return bsl_forward_stream(X, M, W, Y, workspace, workspace_bytes, stream);
-    return bsl_forward_tc(X, M, W, Y, stream);
+    if (M > 0 && M <= kSmallMMax)
+        return bsl_forward_stream(X, M, W, bias, Y, workspace, workspace_bytes, stream);
+    return bsl_forward_tc(X, M, W, bias, Y, stream);
 }
 
 bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *W, void *dX, void *stream)
@@ -284,7 +305,16 @@ bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *W, void 
     if (M <= 0 || check_matrix(dY, M) != BSL_OK || check_matrix(dX, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
     BSL_TRY(bind_device(dY));
     BSL_TRY(check_device());
-    return launch_spmm_tc(dY, M, W->N, W, true, dX, W->K, static_cast<cudaStream_t>(stream));
+    return launch_spmm_tc(dY, M, W->N, W, true, nullptr, dX, W->K, static_cast<cudaStream_t>(stream));
+}
+
+bsl_status bsl_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, void *stream)
+{
+    if (M <= 0 || N <= 0 || N % 32 || check_matrix(dY, M) != BSL_OK || !dbias || !aligned(dbias, 16))
+        return BSL_ERR_INVALID_ARG;
+    BSL_TRY(bind_device(dY));
+    BSL_TRY(check_device());
+    return launch_bias_grad(dY, M, N, dbias, static_cast<cudaStream_t>(stream));
 }
 
 bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const bsl_bsr *W, void *dW_values,

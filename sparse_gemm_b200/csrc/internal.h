@@ -16,6 +16,12 @@ namespace bsl {
 bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                  uint32_t box_inner, uint32_t box_outer, int swizzle_bytes);
 
+// Encode the packed weight values bf16 [nblocks][b][b] as a 3-D tensor map
+// (x = column inside a block, y = row inside a block, z = block) with a
+// box of b columns x box_rows rows x 1 block, swizzled like the kernels'
+// shared-memory operands (128-byte rows for b = 64, 64-byte rows for b = 32).
+bool make_block_map(CUtensorMap *map, const void *values, int32_t b, int32_t nblocks, uint32_t box_rows);
+
 int num_sms();
 // Argument and device checks shared by the entry points (api.cu).
 bsl_status bind_device(const void *p);  // make the device owning p current
@@ -31,14 +37,17 @@ bsl_status launch_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t 
 
 // Forward (A = X, segments = block rows) and input gradient (A = dY,
 // segments = block columns through the CSC index) share one engine.
+// bias: bf16 [out_cols] added to every output row (forward only; may be null).
 bsl_status launch_spmm_tc(const void *A, int32_t M, int32_t a_cols, const bsl_bsr *W, bool transposed,
-                          void *out, int32_t out_cols, cudaStream_t s);
+                          const void *bias, void *out, int32_t out_cols, cudaStream_t s);
 
 bsl_status launch_sddmm_tc(const void *dY, const void *X, int32_t M, const bsl_bsr *W, void *dW,
                            cudaStream_t s);
 
 size_t stream_workspace_bytes(int32_t M, const bsl_bsr *W);
-bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *ws, cudaStream_t s);
+bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, void *ws,
+                             cudaStream_t s);
+bsl_status launch_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, cudaStream_t s);
 
 bsl_status launch_debug_wait(int32_t *status, uint64_t timeout_ns, cudaStream_t s);
 

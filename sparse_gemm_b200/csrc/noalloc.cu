@@ -68,5 +68,5 @@ extern "C" bsl_status bsl_forward_stream_noalloc(const void *X, int32_t M, const
     if (stream_workspace_bytes(M, W) > BSL_NOALLOC_SCRATCH_BYTES) return BSL_ERR_SCRATCH_TOO_SMALL;
     void *scratch = nullptr;
     if ((b = scratch_address(&scratch)) != BSL_OK) return b;
-    return bsl_forward_stream(X, M, W, Y, scratch, BSL_NOALLOC_SCRATCH_BYTES, stream);
+    return bsl_forward_stream(X, M, W, nullptr, Y, scratch, BSL_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -18,9 +18,8 @@
 //   k_group_plan one warp per group of G = 128/b rows (columns) in that order:
 //                merges the members' sorted block coordinates into the
 //                entry list of the tensor-core kernels (count pass, scan,
-//                fill pass)
-//   k_gather_mma the values again, in plan order and in the tensor core's
-//                swizzled shared-memory image (one copy per plan)
+//                fill pass); the kernels read the values themselves from
+//                `values` (stored once) through this list
 #include "common.cuh"
 #include "internal.h"
 
@@ -276,27 +275,6 @@ __global__ void __launch_bounds__(1024) k_scan_groups(int32_t *a, int32_t na, in
     scan_counts(d, nd, nullptr, 1, sm);
 }
 
-// dst[i] = block map[i] of `values`, with the 16-byte chunks of each row
-// permuted as the 128-byte (b = 64) / 64-byte (b = 32) swizzle places them.
-__global__ void k_gather_mma(const uint4 *__restrict__ values, const int32_t *__restrict__ map,
-                             uint4 *__restrict__ dst, int32_t b, int32_t nnz)
-{
-    const int vpr = b / 8;
-    const int64_t per_block = static_cast<int64_t>(b) * vpr;
-    const int64_t total = per_block * nnz;
-    for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
-         t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int i = static_cast<int>(t / per_block);
-        const int rem = static_cast<int>(t - static_cast<int64_t>(i) * per_block);
-        const int row = rem / vpr, ch = rem - row * vpr;
-        int src = map[i];
-        src = src < 0 ? 0 : (src >= nnz ? nnz - 1 : src);
-        const int pch = b == 64 ? (ch ^ (row & 7)) : (ch ^ ((row >> 1) & 3));
-        dst[(static_cast<int64_t>(i) * b + row) * vpr + pch] =
-            values[(static_cast<int64_t>(src) * b + row) * vpr + ch];
-    }
-}
-
 template <int G>
 void launch_group_plans(const bsl_bsr *o, cudaStream_t s)
 {
@@ -358,15 +336,6 @@ bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cud
     if (o->b == 64) launch_group_plans<2>(o, s);
     else launch_group_plans<4>(o, s);
     cudaMemsetAsync(o->sched, 0, 8 * sizeof(int32_t), s);
-    if (nnz > 0) {
-        const int64_t total = static_cast<int64_t>(nnz) * o->b * (o->b / 8);
-        const int64_t want = (total + 255) / 256;
-        const int grid = static_cast<int>(want < 8L * num_sms() ? want : 8L * num_sms());
-        k_gather_mma<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(o->values), o->rgrp_blk,
-                                          static_cast<uint4 *>(o->values_rg), o->b, nnz);
-        k_gather_mma<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(o->values), o->cgrp_blk,
-                                          static_cast<uint4 *>(o->values_cg), o->b, nnz);
-    }
     return cuda_status(cudaGetLastError());
 }
 

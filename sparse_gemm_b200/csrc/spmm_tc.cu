@@ -47,9 +47,10 @@
 // stay balanced under skewed block rows.  The first producer warp takes a
 // unit only when it starts issuing it (a CTA never sits on work another SM
 // could do) and publishes it to the other roles through a small ring in
-// shared memory.  The last CTA to stop taking units puts the counter back to
-// zero for the next launch, so launches on one weight must be ordered (one
-// stream, or events).
+// shared memory.  The launcher zeroes the counter in stream order before
+// every launch, so a launch that never finished leaves nothing behind; two
+// launches of the same contraction on one weight must not run at the same
+// time (they would share the counter).
 //
 // Roles per CTA (persistent grid, one CTA per SM):
 //   warps 0..P-1   producers: TMA tile copy of the activation tile, bulk
@@ -94,8 +95,9 @@ struct SpmmCfg {
     static constexpr int NUM_BARS = 2 * S + 2 * ACC + 2 * UR + 1;
     static constexpr int HDR_V4 = (G + 1) / 2;          // 16-byte header words per slot (two runs each)
     static constexpr int HDR_BYTES = S * HDR_V4 * 16;
+    static constexpr int BLK_IDS = 32 * G;              // block ids of one 32-entry chunk, per producer warp
     static constexpr int SMEM_BYTES =
-        S * SLOT_BYTES + OUT_BYTES + NUM_BARS * 8 + HDR_BYTES + UR * 4 + 64 + 1024;
+        S * SLOT_BYTES + OUT_BYTES + NUM_BARS * 8 + HDR_BYTES + UR * 4 + P * BLK_IDS * 4 + 64 + 1024;
     static_assert((1 << S_LOG) == S && S % P == 0 && (P & (P - 1)) == 0, "slot ownership");
     static_assert(ACC_COLS == 256 && TMEM_COLS == 512, "TMEM layout");
     static_assert(G <= 8, "member mask is 8 bits");
@@ -109,8 +111,9 @@ struct SpmmArgs {
     const int32_t *grp_ptr;    // [ngroups+1] entry range per group
     const int32_t *grp_bptr;   // [ngroups+1] block range per group
     const int32_t *grp_ent;    // entries: coordinate | (mask << 24)
-    const uint8_t *grp_vals;   // weight blocks in plan order, swizzled smem image
-    int32_t *sched;            // [2] next unit, CTAs finished taking units (zero between launches)
+    const int32_t *grp_blk;    // BSR block of every present member, entry by entry
+    int32_t *sched;            // [1] next unit (zeroed in stream order before every launch)
+    const __nv_bfloat16 *bias; // [nseg * b] added to every output row (forward only; null: none)
     int32_t *status;
     uint64_t timeout_ns;
 };
@@ -172,7 +175,8 @@ __device__ __forceinline__ bool unit_take(uint64_t *ufull, uint64_t *uempty, con
 
 template <int B, bool TRANS>
 __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
-    k_spmm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmO, const SpmmArgs args)
+    k_spmm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmO,
+              const __grid_constant__ CUtensorMap tmW, const SpmmArgs args)
 {
     using Cfg = SpmmCfg<B>;
     extern __shared__ uint8_t smem_raw[];
@@ -195,6 +199,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
     volatile int *uring = reinterpret_cast<volatile int *>(hdr + Cfg::S * Cfg::HDR_V4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(const_cast<int *>(uring + Cfg::UR));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int32_t *blk_ids = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [P][BLK_IDS]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
@@ -217,6 +222,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         fence_barrier_init();
         tma_prefetch_map(&tmA);
         tma_prefetch_map(&tmO);
+        tma_prefetch_map(&tmW);
     }
     if (warp == Cfg::W_MMA) {
         tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -294,6 +300,11 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                 seen_ex = (lane == 0 ? 0u : seen_ex) | seen_carry;
                 const int total = __shfl_sync(0xffffffffu, incl, 31);
                 const uint32_t all_or = __shfl_sync(0xffffffffu, orl, 31);
+                // the BSR blocks of the chunk's entries (total <= 32 * G), for the copies
+                int32_t *ids = blk_ids + p * Cfg::BLK_IDS;
+                __syncwarp();  // lane 0 has finished reading the previous chunk's ids
+                for (int i = lane; i < total; i += 32) ids[i] = args.grp_blk[bcur + i];
+                __syncwarp();
                 for (int t = (p - e) & (Cfg::P - 1); t < n; t += Cfg::P) {
                     const uint32_t ent = static_cast<uint32_t>(__shfl_sync(0xffffffffu, el, t));
                     const int off = __shfl_sync(0xffffffffu, excl, t);
@@ -338,9 +349,11 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                             uint8_t *sp = slots + slot * Cfg::SLOT_BYTES;
                             mbar_arrive_expect_tx(&full[slot], Cfg::X_BYTES + k * Cfg::W_BYTES);
                             tma_load_2d(sp, &tmA, &full[slot], static_cast<int>(ent & 0xFFFFFFu) * B, m0);
-                            bulk_load(sp + Cfg::X_BYTES,
-                                      args.grp_vals + static_cast<int64_t>(bcur + off) * Cfg::W_BYTES,
-                                      k * Cfg::W_BYTES, &full[slot]);
+                            // the present members' blocks, one swizzled tile each, straight
+                            // from the packed values (stored once, in BSR order)
+                            for (uint32_t qq = 0; qq < k; ++qq)
+                                tma_load_3d(sp + Cfg::X_BYTES + qq * Cfg::W_BYTES, &tmW, &full[slot], 0, 0,
+                                            ids[off + qq]);
                             if (tn < n) tma_prefetch_2d(&tmA, static_cast<int>(entn & 0xFFFFFFu) * B, m0);
 #pragma unroll
                             for (int i = 0; i < Cfg::S / Cfg::P; ++i)
@@ -361,14 +374,6 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
             if (!ok) {
                 *abort_flag = 1;
                 set_status(args.status, BSL_ERR_TIMEOUT);
-            }
-            if (p == 0) {
-                // the last CTA to stop taking units resets the counter for the next launch
-                __threadfence();
-                if (atomicAdd(args.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
-                    atomicExch(args.sched, 0);
-                    atomicExch(args.sched + 1, 0);
-                }
             }
             // every copy this warp issued lands before the CTA's smem is released
             // (the last fill of a slot is the newest phase of its barrier)
@@ -517,6 +522,21 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                     const int nz = __shfl_sync(0xffffffffu, mnz, mbr);
                     if (seg < 0) break;
                     uint32_t v[B];
+                    // the bias of the member's b output columns (the same for every row)
+                    float bv[B];
+                    if (args.bias) {
+                        const uint4 *bp = reinterpret_cast<const uint4 *>(args.bias + static_cast<int64_t>(seg) * B);
+#pragma unroll
+                        for (int c = 0; c < B / 8; ++c) {
+                            const uint4 u = __ldg(bp + c);
+                            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                bv[8 * c + 2 * h] = __uint_as_float(w4[h] << 16);
+                                bv[8 * c + 2 * h + 1] = __uint_as_float(w4[h] & 0xFFFF0000u);
+                            }
+                        }
+                    }
                     if (nz) {
                         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                                ar.slot * Cfg::ACC_COLS + s * Cfg::HALF_COLS + mbr * B;
@@ -527,6 +547,10 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                     } else {
 #pragma unroll
                         for (int c = 0; c < B; ++c) v[c] = 0u;
+                    }
+                    if (args.bias) {
+#pragma unroll
+                        for (int c = 0; c < B; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) + bv[c]);
                     }
                     if (lane == 0) bulk_wait_group_read<1>();  // staging chunk `ob` was read out
                     __syncwarp();
@@ -573,29 +597,36 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
 }
 
 template <int B, bool TRANS>
-bsl_status run(const CUtensorMap &a, const CUtensorMap &o, const SpmmArgs &args, cudaStream_t s)
+bsl_status run(const CUtensorMap &a, const CUtensorMap &o, const CUtensorMap &w, const SpmmArgs &args,
+               cudaStream_t s)
 {
     using Cfg = SpmmCfg<B>;
     auto kern = k_spmm_tc<B, TRANS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_status(e);
+    // the work counters start at zero on every launch, in stream order, so a
+    // launch that did not finish cannot make a later one skip units
+    e = cudaMemsetAsync(args.sched, 0, 2 * sizeof(int32_t), s);
+    if (e != cudaSuccess) return cuda_status(e);
     const int grid = args.units < num_sms() ? args.units : num_sms();
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(a, o, args);
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(a, o, w, args);
     return cuda_status(cudaGetLastError());
 }
 
 }  // namespace
 
 bsl_status launch_spmm_tc(const void *A, int32_t M, int32_t a_cols, const bsl_bsr *W, bool transposed,
-                          void *out, int32_t out_cols, cudaStream_t s)
+                          const void *bias, void *out, int32_t out_cols, cudaStream_t s)
 {
     const int B = W->b;
-    if (W->nnz == 0)
+    if (W->nnz == 0 && (transposed || !bias))
         return cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(M) * out_cols * 2, s));
-    CUtensorMap ma, mo;
+    CUtensorMap ma, mo, mw;
     if (!make_map_2d(&ma, A, a_cols, M, static_cast<uint64_t>(a_cols) * 2, B, 256, 2 * B) ||
-        !make_map_2d(&mo, out, out_cols, M, static_cast<uint64_t>(out_cols) * 2, B, 32, 2 * B))
+        !make_map_2d(&mo, out, out_cols, M, static_cast<uint64_t>(out_cols) * 2, B, 32, 2 * B) ||
+        (W->nnz > 0 && !make_block_map(&mw, W->values, B, W->nnz, B)))
         return BSL_ERR_CUDA;
+    if (W->nnz == 0) mw = ma;  // no weight block is ever loaded
     const int G = 128 / B;
     SpmmArgs args;
     args.M = M;
@@ -608,12 +639,13 @@ bsl_status launch_spmm_tc(const void *A, int32_t M, int32_t a_cols, const bsl_bs
     args.grp_ptr = transposed ? W->cgrp_ptr : W->rgrp_ptr;
     args.grp_bptr = transposed ? W->cgrp_bptr : W->rgrp_bptr;
     args.grp_ent = transposed ? W->cgrp_ent : W->rgrp_ent;
-    args.grp_vals = static_cast<const uint8_t *>(transposed ? W->values_cg : W->values_rg);
+    args.grp_blk = transposed ? W->cgrp_blk : W->rgrp_blk;
     args.sched = W->sched + (transposed ? 2 : 0);
+    args.bias = transposed ? nullptr : static_cast<const __nv_bfloat16 *>(bias);
     args.status = W->status;
     args.timeout_ns = wait_timeout_ns();
-    if (B == 64) return transposed ? run<64, true>(ma, mo, args, s) : run<64, false>(ma, mo, args, s);
-    return transposed ? run<32, true>(ma, mo, args, s) : run<32, false>(ma, mo, args, s);
+    if (B == 64) return transposed ? run<64, true>(ma, mo, mw, args, s) : run<64, false>(ma, mo, mw, args, s);
+    return transposed ? run<32, true>(ma, mo, mw, args, s) : run<32, false>(ma, mo, mw, args, s);
 }
 
 }  // namespace bsl

@@ -55,6 +55,7 @@ struct StreamArgs {
     __nv_bfloat16 *Y;
     float *ws;
     const int32_t *row_ptr, *col_idx;
+    const __nv_bfloat16 *bias;  // [N] added to every output row (null: none)
     int32_t M, N, K, R, C, nnz;
     int32_t *status;
     uint64_t timeout_ns;
@@ -127,9 +128,10 @@ __device__ __forceinline__ void flush_row(const RowAcc<B, MP> &acc, const Stream
                 const int m = j * 8 + c2;           // token
                 const float v0 = acc.d[i][j][2 * h], v1 = acc.d[i][j][2 * h + 1];
                 if (direct) {
+                    const float bb = a.bias ? __bfloat162float(a.bias[static_cast<int64_t>(r) * B + n]) : 0.f;
                     __nv_bfloat16 *y = a.Y + static_cast<int64_t>(m) * a.N + static_cast<int64_t>(r) * B + n;
-                    if (m < a.M) y[0] = __float2bfloat16_rn(v0);
-                    if (m + 1 < a.M) y[a.N] = __float2bfloat16_rn(v1);
+                    if (m < a.M) y[0] = __float2bfloat16_rn(a.bias ? v0 + bb : v0);
+                    if (m + 1 < a.M) y[a.N] = __float2bfloat16_rn(a.bias ? v1 + bb : v1);
                 } else {
                     *reinterpret_cast<float2 *>(slot + n * MP + m) = make_float2(v0, v1);
                 }
@@ -312,8 +314,9 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     }
 }
 
-// One warp per block row: zeros for rows without blocks; for rows cut between
-// warp shares, the sum of the shares' partials in warp order.
+// One warp per block row: zeros (or the bias) for rows without blocks; for
+// rows cut between warp shares, the sum of the shares' partials in warp order
+// (plus the bias).
 template <int B, int MP>
 __global__ void k_stream_fixup(const StreamArgs a, int GW)
 {
@@ -353,8 +356,9 @@ __global__ void k_stream_fixup(const StreamArgs a, int GW)
     for (int e = 0; e < PER; ++e) {
         const int idx = e * 32 + lane;  // = n * MP + m
         const int n = idx / MP, m = idx % MP;
+        const float v = a.bias ? sum[e] + __bfloat162float(a.bias[static_cast<int64_t>(r) * B + n]) : sum[e];
         if (m < a.M)
-            a.Y[static_cast<int64_t>(m) * a.N + static_cast<int64_t>(r) * B + n] = __float2bfloat16_rn(sum[e]);
+            a.Y[static_cast<int64_t>(m) * a.N + static_cast<int64_t>(r) * B + n] = __float2bfloat16_rn(v);
     }
 }
 
@@ -398,7 +402,8 @@ size_t stream_workspace_bytes(int32_t M, const bsl_bsr *W)
     return static_cast<size_t>(num_sms()) * kStreamWarps * 2 * W->b * MP * sizeof(float);
 }
 
-bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, void *Y, void *ws, cudaStream_t s)
+bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, void *ws,
+                             cudaStream_t s)
 {
     const int B = W->b;
     StreamArgs a;
@@ -407,6 +412,7 @@ bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, void *Y
     a.ws = static_cast<float *>(ws);
     a.row_ptr = W->row_ptr;
     a.col_idx = W->col_idx;
+    a.bias = static_cast<const __nv_bfloat16 *>(bias);
     a.M = M;
     a.N = W->N;
     a.K = W->K;

@@ -51,17 +51,20 @@ def _bsr(**kw):
 ])
 def test_bad_weight_descriptor_is_rejected_on_host(lib, bad, code):
     s = _bsr(**bad)
-    assert lib.bsl_forward_tc(4096, 64, ctypes.byref(s), 4096, None) == code
+    assert lib.bsl_forward_tc(4096, 64, ctypes.byref(s), None, 4096, None) == code
     assert lib.bsl_backward_input(4096, 64, ctypes.byref(s), 4096, None) == code
 
 
 def test_bad_matrices_are_rejected_on_host(lib):
     s = _bsr()
-    assert lib.bsl_forward_tc(0, 64, ctypes.byref(s), 4096, None) == 1       # null X
-    assert lib.bsl_forward_tc(4096, 0, ctypes.byref(s), 4096, None) == 1     # M = 0
-    assert lib.bsl_forward_tc(4104, 64, ctypes.byref(s), 4096, None) == 1    # misaligned X
+    assert lib.bsl_forward_tc(0, 64, ctypes.byref(s), None, 4096, None) == 1       # null X
+    assert lib.bsl_forward_tc(4096, 0, ctypes.byref(s), None, 4096, None) == 1     # M = 0
+    assert lib.bsl_forward_tc(4104, 64, ctypes.byref(s), None, 4096, None) == 1    # misaligned X
+    assert lib.bsl_forward_tc(4096, 64, ctypes.byref(s), 4104, 4096, None) == 1    # misaligned bias
     assert lib.bsl_backward_weight(4096, 0, 8, ctypes.byref(s), 4096, None) == 1
-    assert lib.bsl_forward_stream(4096, 64, ctypes.byref(s), 4096, 4096, 1 << 20, None) == 2  # M too big
+    assert lib.bsl_forward_stream(4096, 64, ctypes.byref(s), None, 4096, 4096, 1 << 20, None) == 2  # M too big
+    assert lib.bsl_bias_grad(4096, 64, 100, 4096, None) == 1                        # N not a multiple of 32
+    assert lib.bsl_bias_grad(4096, 64, 256, 0, None) == 1                           # null output
     assert lib.bsl_pack_count(0, 4, 4, 4096, ctypes.byref(ctypes.c_int32()), None) == 1
 
 
