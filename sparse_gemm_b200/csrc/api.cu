@@ -130,6 +130,26 @@ int num_sms()
     return n;
 }
 
+bsl_status set_smem_once(const void *func, int bytes)
+{
+    struct Entry {
+        const void *func;
+        int dev;
+    };
+    static Entry done[64];
+    static int ndone = 0;
+    static std::mutex mu;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < ndone; ++i)
+        if (done[i].func == func && done[i].dev == dev) return BSL_OK;
+    const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (ndone < 64) done[ndone++] = Entry{func, dev};
+    return BSL_OK;
+}
+
 uint64_t wait_timeout_ns()
 {
     std::call_once(g_timeout_once, [] {
@@ -242,7 +262,8 @@ bsl_status bsl_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *ro
                           void *stream)
 {
     if (!mask || !row_ptr || !nnz_host || R <= 0 || C <= 0) return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(row_ptr));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(row_ptr));
     BSL_TRY(check_device());
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     BSL_TRY(launch_pack_count(mask, R, C, row_ptr, s));
@@ -254,7 +275,8 @@ bsl_status bsl_pack(const void *W, const uint8_t *mask, const bsl_bsr *out, void
 {
     BSL_TRY(check_bsr(out));
     if (!mask || check_matrix(W, out->N) != BSL_OK) return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(W));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(W));
     BSL_TRY(check_device());
     return launch_pack(W, mask, out, static_cast<cudaStream_t>(stream));
 }
@@ -272,9 +294,10 @@ bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, const void
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
     if (bias && !aligned(bias, 16)) return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(X));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(X));
     BSL_TRY(check_device());
-    return launch_spmm_tc(X, M, W->K, W, false, bias, Y, W->N, static_cast<cudaStream_t>(stream));
+    return launch_spmm_pair(X, M, W, bias, Y, static_cast<cudaStream_t>(stream));
 }
 
 bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y,
@@ -284,7 +307,8 @@ bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, const 
     if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
     if (bias && !aligned(bias, 16)) return BSL_ERR_INVALID_ARG;
     if (M > kSmallMMax) return BSL_ERR_UNSUPPORTED;
-    BSL_TRY(bind_device(X));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(X));
     BSL_TRY(check_device());
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < stream_workspace_bytes(M, W))
         return BSL_ERR_INVALID_ARG;
@@ -303,16 +327,18 @@ bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *W, void 
 {
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(dY, M) != BSL_OK || check_matrix(dX, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(dY));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(dY));
     BSL_TRY(check_device());
-    return launch_spmm_tc(dY, M, W->N, W, true, nullptr, dX, W->K, static_cast<cudaStream_t>(stream));
+    return launch_spmm_dx(dY, M, W, dX, static_cast<cudaStream_t>(stream));
 }
 
 bsl_status bsl_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, void *stream)
 {
     if (M <= 0 || N <= 0 || N % 32 || check_matrix(dY, M) != BSL_OK || !dbias || !aligned(dbias, 16))
         return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(dY));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(dY));
     BSL_TRY(check_device());
     return launch_bias_grad(dY, M, N, dbias, static_cast<cudaStream_t>(stream));
 }
@@ -323,7 +349,8 @@ bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const b
     BSL_TRY(check_bsr(W));
     if (M <= 0 || check_matrix(dY, M) != BSL_OK || check_matrix(X, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
     if (W->nnz > 0 && (!dW_values || !aligned(dW_values, 16))) return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(dY));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(dY));
     BSL_TRY(check_device());
     return launch_sddmm_tc(dY, X, M, W, dW_values, static_cast<cudaStream_t>(stream));
 }
@@ -331,7 +358,8 @@ bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const b
 bsl_status bsl_get_device_status(const bsl_bsr *W, int32_t *status_host, void *stream)
 {
     if (!W || !W->status || !status_host) return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(W->status));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(W->status));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     BSL_TRY(cuda_status(cudaMemcpyAsync(status_host, W->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s)));
     BSL_TRY(cuda_status(cudaMemsetAsync(W->status, 0, sizeof(int32_t), s)));
@@ -347,7 +375,8 @@ void bsl_set_wait_timeout_us(uint64_t timeout_us)
 bsl_status bsl_debug_wait_timeout(int32_t *status, uint64_t timeout_us, void *stream)
 {
     if (!status || !aligned(status, 4)) return BSL_ERR_INVALID_ARG;
-    BSL_TRY(bind_device(status));
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(status));
     BSL_TRY(check_device());
     return launch_debug_wait(status, timeout_us * 1000ull, static_cast<cudaStream_t>(stream));
 }

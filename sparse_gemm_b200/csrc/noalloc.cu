@@ -62,7 +62,8 @@ extern "C" bsl_status bsl_forward_stream_noalloc(const void *X, int32_t M, const
     if (!X || !Y || M <= 0) return BSL_ERR_INVALID_ARG;
     if (M > bsl_small_m_max()) return BSL_ERR_UNSUPPORTED;
     // the scratch lives on the device that owns X: make it current first
-    bsl_status b = bind_device(X);
+    DeviceGuard guard;
+    bsl_status b = guard.bind(X);
     if (b != BSL_OK) return b;
     if ((b = check_device()) != BSL_OK) return b;
     if (stream_workspace_bytes(M, W) > BSL_NOALLOC_SCRATCH_BYTES) return BSL_ERR_SCRATCH_TOO_SMALL;

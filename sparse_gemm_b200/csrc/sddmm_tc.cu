@@ -283,8 +283,8 @@ bsl_status run(const CUtensorMap &dy, const CUtensorMap &x, const SddmmArgs &arg
 {
     using Cfg = SddmmCfg<B>;
     auto kern = k_sddmm_tc<B>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_status(e);
+    const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(kern), Cfg::SMEM_BYTES);
+    if (sa != BSL_OK) return sa;
     const int grid = ngroups_max < num_sms() ? ngroups_max : num_sms();
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(dy, x, args);
     return cuda_status(cudaGetLastError());

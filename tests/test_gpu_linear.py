@@ -134,8 +134,8 @@ def test_repack_in_place_with_a_new_mask():
     for key in ("col_idx", "row_idx", "csc_to_bsr"):
         assert np.array_equal(getattr(Wp, key)[:nnz].cpu().numpy(), want[key]), key
     assert np.array_equal(bits(Wp.block_values()), want["values"].reshape(nnz, b, b))
-    G = 128 // b
-    gp, gb, ent, blk = _plan.group_plan(want["row_ptr"], want["col_idx"], oracle.schedule_order(want["row_ptr"]), G)
+    gp, gb, ent, blk = _plan.group_plan(want["row_ptr"], want["col_idx"], oracle.schedule_order(want["row_ptr"]),
+                                        256 // b)
     assert np.array_equal(Wp.rgrp_ptr.cpu().numpy(), gp)
     assert np.array_equal(Wp.rgrp_ent[:len(ent)].cpu().numpy(), ent)
     ref, S = oracle.forward(second["X"], second["W"], second["mask"], b)
