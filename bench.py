@@ -49,16 +49,10 @@ L2_BYTES_DEFAULT = 126 * 2 ** 20
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload.  The
 # entry is only used while the kernel source still hashes to `src_sha`.
 TRAFFIC = {
-    ("large_fwd", "fwd"): {"bytes": 292852736, "files": ["spmm_tc.cu", "common.cuh"],
-                           "src_sha": "7041d64ad13d53e9", "profile": "profiles/k_spmm_tc_fwd_large_fwd.md"},
-    ("enc_train_d1.0", "dx"): {"bytes": 29933824, "files": ["spmm_tc.cu", "common.cuh"],
-                               "src_sha": "7041d64ad13d53e9", "profile": "profiles/k_spmm_tc_dx_enc_train_d1.md"},
-    ("enc_train_d1.0", "dw"): {"bytes": 31499008, "files": ["sddmm_tc.cu", "common.cuh"],
-                               "src_sha": "b597a71c38505806", "profile": "profiles/k_sddmm_tc_dw_enc_train_d1.md"},
-    # k_stream_fwd alone (the fix-up kernel reads and writes well under 1 MB)
-    ("decode_fwd", "fwd"): {"bytes": 22754560, "files": ["stream_fwd.cu", "common.cuh"],
-                            "src_sha": "fa4f48f3f5bf4d99", "profile": "profiles/k_stream_fwd_decode_fwd.md"},
 }
+# the kernel source files each contraction's traffic figure depends on
+TRAFFIC_FILES = {"fwd": ["spmm_pair.cu", "common.cuh"], "fwd_small": ["stream_fwd.cu", "common.cuh"],
+                 "dx": ["spmm_tc.cu", "common.cuh"], "dw": ["sddmm_tc.cu", "common.cuh"]}
 
 
 def log(*a):
@@ -347,7 +341,7 @@ def run_gpu(args):
     small = w.M <= sg.small_m_max()
 
     kinds = ["fwd", "dx", "dw"] if train else ["fwd"]
-    launches_per_step = (2 if small else 1) + (2 if train else 0)
+    launches_per_step = 1 + (2 if train else 0)  # kernels per step (each also has a small memset)
 
     def step(i):
         j = i % ncopy
@@ -459,11 +453,12 @@ def run_gpu(args):
     # dominant kernel + its roofline
     dom = max(per_kernel, key=per_kernel.get)
     roof = roofline_entry(dom, alg[dom], per_kernel[dom], pk)
-    roof["kernel"] = {"fwd": "k_stream_fwd+k_stream_fixup" if small else "k_spmm_tc (forward)",
+    roof["kernel"] = {"fwd": "k_stream_fwd" if small else "k_spmm_pair (forward)",
                       "dx": "k_spmm_tc (input gradient)", "dw": "k_sddmm_tc"}[dom]
     roof["peak_source"] = pk["source"] + (" burst bf16" if roof["unit"] == "TFLOP/s" else " HBM copy")
     tr = TRAFFIC.get((w.name, dom))
-    roof["traffic"] = tr["bytes"] if tr and tr.get("src_sha") == src_sha(*tr["files"]) else None
+    files = TRAFFIC_FILES["fwd_small" if (dom == "fwd" and small) else dom]
+    roof["traffic"] = tr["bytes"] if tr and tr.get("src_sha") == src_sha(*files) else None
     roof["algorithmic_bytes"] = alg[dom]["bytes"]
     roof["algorithmic_flops"] = alg[dom]["flops"]
     roof["tensor_frac_of_sustained"] = round(alg[dom]["flops"] / (per_kernel[dom] * 1e-3) / 1e12

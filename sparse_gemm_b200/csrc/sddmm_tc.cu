@@ -8,53 +8,56 @@
 // written as bf16 into dW_values[p] (BSR order), reduction over all M rows in
 // fp32.
 //
-// MMA shape: the blocks of one block column c share the X strip X[:, c-block],
-// so a work unit ("group") stacks G = 128/b blocks of the same column along
-// MMA M: A = [dY[:, r_1-block] | ... | dY[:, r_G-block]]^T (128 x 128 rows of
-// M per stage, MN-major in smem: the dY tiles are loaded untransposed),
-// B = X[:, c-block]^T (b x 128, MN-major), D = 128 x b fp32 in TMEM.  Groups
-// are listed per column by the pack's dw_gptr prefix (ceil(count/G) per
-// column); a column's last group may hold fewer than G blocks, and its
-// unused accumulator lanes are never stored.
+// Tiles.  The block grid is cut into tiles of GR x GC blocks (GR*b = 128 rows
+// of dW, GC*b = 128 columns).  For a tile, every stage brings in 128 rows of
+// M of the dY strips dY[:, r-block] of the tile's block rows and of the X
+// strips X[:, c-block] of its block columns, and one tcgen05.mma of
+// M = 128, N = 128 per 16 rows computes the whole 128 x 128 tile of
+// dY^T . X (fp32 in TMEM).  Only strips of block rows / columns that hold a
+// stored block in the tile are copied (a skipped strip leaves old data in
+// shared memory, which only reaches accumulator entries that are never
+// stored), only stored blocks are written out, and tiles without a stored
+// block are skipped.  Each strip is read once per tile instead of once per
+// stored block, and every MMA is full width.
 //
-// Roles: warps 0..P-1 TMA producers (one thread cannot start copies fast
-// enough, so k-step i is issued by warp i % P; the stage ring is partitioned
-// so that slot i % STAGES is only ever filled by that warp), warp P TMEM
-// owner + MMA issuer, warps P+1..P+4 epilogue (TMEM -> bf16 -> 16-byte
-// global stores).
+// Roles: warps 0..P-1 TMA producers (stage i of this CTA is filled by warp
+// i % P, which owns that stage slot alone), warp P TMEM owner + MMA issuer,
+// warps P+1..P+4 epilogue (TMEM -> bf16 -> 16-byte global stores of the
+// stored blocks).  Tiles go round-robin over the CTAs, consecutive tiles
+// sharing their block rows (their dY strips stay in L2).  Results do not
+// depend on the schedule: every output is one fixed-order fp32 reduction.
 #include "common.cuh"
 #include "internal.h"
 
 namespace bsl {
 namespace {
 
-// Rows of M per stage: copies are the bottleneck of this kernel (one thread
-// starts only about four per microsecond), so each copy moves a tall strip.
-constexpr int kSddmmRows = 128;
-
 template <int B>
 struct SddmmCfg {
-    static constexpr int G = 128 / B;                    // blocks stacked along MMA M
-    static constexpr int MK = kSddmmRows;                // rows of M reduced per stage
+    static constexpr int GR = 128 / B;                   // block rows per tile (MMA M = 128)
+    static constexpr int GC = 128 / B;                   // block columns per tile (MMA N = 128)
+    static constexpr int MK = 128;                       // rows of M reduced per stage
     static constexpr int ROW_BYTES = B * 2;
     static constexpr int T_BYTES = MK * ROW_BYTES;       // one strip tile (MK x b)
-    static constexpr int STAGE_BYTES = (G + 1) * T_BYTES;
-    static constexpr int STAGES = 4;
-    static constexpr int P = 4;                          // producer warps (STAGES % P == 0)
+    static constexpr int STAGE_BYTES = (GR + GC) * T_BYTES;
+    static constexpr int STAGES = 3;
+    static constexpr int P = STAGES;                     // producer warps: one per stage slot
     static constexpr int THREADS = (P + 5) * 32;
-    static_assert(STAGES % P == 0, "each stage slot belongs to one producer warp");
     static constexpr int ACC = 2;
-    static constexpr int TMEM_COLS = ACC * B;            // 64 or 128
+    static constexpr int ACC_COLS = GC * B;              // 128
+    static constexpr int TMEM_COLS = ACC * ACC_COLS;     // 256
     static constexpr uint32_t LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t SBO = 8 * ROW_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NUM_BARS * 8 + 16 + 1024;
+    static_assert(STAGES % P == 0, "each stage slot belongs to one producer warp");
+    static_assert(GR * GC <= 32, "one lane per block of a tile");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct SddmmArgs {
-    int32_t M, C, ksteps;
-    const int32_t *col_ptr, *row_idx, *csc_to_bsr, *dw_gptr;
+    int32_t M, R, C, ksteps, nrg, ncg, ntiles;
+    const int32_t *row_ptr, *col_idx;
     __nv_bfloat16 *dW;
     int32_t *status;
     uint64_t timeout_ns;
@@ -65,16 +68,43 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// column c of group g: last c with dw_gptr[c] <= g
-__device__ __forceinline__ int group_column(const int32_t *gptr, int C, int g)
+// Stored blocks of tile t, found by the whole warp (lane l < GR*GC looks up
+// block (i, j) = (l / GC, l % GC) in its block row's ascending columns):
+// returns the lane's BSR position (-1: not stored) and the tile's block-row /
+// block-column masks.
+template <int B>
+__device__ __forceinline__ int tile_blocks(const SddmmArgs &a, int t, int lane, uint32_t *rmask, uint32_t *cmask,
+                                           int *rg_out, int *cg_out)
 {
-    int lo = 0, hi = C;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (gptr[mid] <= g) lo = mid;
-        else hi = mid;
+    using Cfg = SddmmCfg<B>;
+    const int rg = t / a.ncg, cg = t - (t / a.ncg) * a.ncg;
+    *rg_out = rg;
+    *cg_out = cg;
+    int pos = -1;
+    if (lane < Cfg::GR * Cfg::GC) {
+        const int i = lane / Cfg::GC, j = lane % Cfg::GC;
+        const int r = rg * Cfg::GR + i, c = cg * Cfg::GC + j;
+        if (r < a.R && c < a.C) {
+            int lo = a.row_ptr[r], hi = a.row_ptr[r + 1];
+            while (lo < hi) {  // first position with column >= c
+                const int mid = (lo + hi) >> 1;
+                if (a.col_idx[mid] < c) lo = mid + 1;
+                else hi = mid;
+            }
+            if (lo < a.row_ptr[r + 1] && a.col_idx[lo] == c) pos = lo;
+        }
     }
-    return lo;
+    const uint32_t present = __ballot_sync(0xffffffffu, pos >= 0);
+    uint32_t rm = 0, cm = 0;
+#pragma unroll
+    for (int l = 0; l < Cfg::GR * Cfg::GC; ++l)
+        if ((present >> l) & 1u) {
+            rm |= 1u << (l / Cfg::GC);
+            cm |= 1u << (l % Cfg::GC);
+        }
+    *rmask = rm;
+    *cmask = cm;
+    return pos;
 }
 
 template <int B>
@@ -93,7 +123,6 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
     uint64_t *drain = tempty + Cfg::ACC;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_go = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
@@ -105,11 +134,10 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
         }
         for (int a = 0; a < Cfg::ACC; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        *epi_go = 0;
         fence_barrier_init();
         tma_prefetch_map(&tmDY);
         tma_prefetch_map(&tmX);
@@ -122,42 +150,53 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int ngroups = args.dw_gptr[args.C];
 
     if (warp < Cfg::P) {
-        // k-step i (counted over all groups of this CTA) uses slot i % STAGES and
-        // is issued by warp i % P; the slot's previous fill, step i - STAGES,
-        // was issued by the same warp, so every wait is on the warp's own fills
-        if (lane == 0) {
-            uint32_t issued = 0, issued_par = 0;
-            bool ok = true;
-            int i = 0;
-            for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x) {
-                const int c = group_column(args.dw_gptr, args.C, g);
-                const int j0 = args.col_ptr[c] + (g - args.dw_gptr[c]) * Cfg::G;
-                const int cnt = min(Cfg::G, args.col_ptr[c + 1] - j0);
-                int rows[Cfg::G];
-#pragma unroll
-                for (int q = 0; q < Cfg::G; ++q) rows[q] = q < cnt ? args.row_idx[j0 + q] : 0;
-                for (int ks = 0; ks < args.ksteps; ++ks, ++i) {
-                    if (i % Cfg::P != warp) continue;
-                    const int stage = i % Cfg::STAGES;
-                    const uint32_t phase = (i / Cfg::STAGES) & 1;
+        // ------------------------------------------------------------ producers
+        // stage i (counted over this CTA's non-empty tiles) uses slot i % STAGES
+        // and is filled by warp i % P; the slot's previous fill, stage
+        // i - STAGES, came from the same warp, so every wait is on its own fills
+        uint32_t issued = 0, issued_par = 0;
+        bool ok = true;
+        int i = 0;
+        for (int t = blockIdx.x; t < args.ntiles && ok; t += gridDim.x) {
+            uint32_t rm, cm;
+            int rg, cg;
+            tile_blocks<B>(args, t, lane, &rm, &cm, &rg, &cg);
+            if (!rm) continue;
+            const uint32_t nstrips = __popc(rm) + __popc(cm);
+            for (int ks = 0; ks < args.ksteps; ++ks, ++i) {
+                if (i % Cfg::P != warp) continue;
+                const int stage = i % Cfg::STAGES;
+                const uint32_t phase = (i / Cfg::STAGES) & 1;
+                int good = 1;
+                if (lane == 0) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, tmo, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *sa = stages + stage * Cfg::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], (cnt + 1) * Cfg::T_BYTES);
+                        good = 0;
+                    } else {
+                        uint8_t *sa = stages + stage * Cfg::STAGE_BYTES;
+                        mbar_arrive_expect_tx(&full[stage], nstrips * Cfg::T_BYTES);
 #pragma unroll
-                    for (int q = 0; q < Cfg::G; ++q)
-                        if (q < cnt)
-                            tma_load_2d(sa + q * Cfg::T_BYTES, &tmDY, &full[stage], rows[q] * B, ks * Cfg::MK);
-                    tma_load_2d(sa + Cfg::G * Cfg::T_BYTES, &tmX, &full[stage], c * B, ks * Cfg::MK);
-                    issued |= 1u << stage;
-                    issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                        for (int q = 0; q < Cfg::GR; ++q)
+                            if ((rm >> q) & 1u)
+                                tma_load_2d(sa + q * Cfg::T_BYTES, &tmDY, &full[stage], (rg * Cfg::GR + q) * B,
+                                            ks * Cfg::MK);
+#pragma unroll
+                        for (int q = 0; q < Cfg::GC; ++q)
+                            if ((cm >> q) & 1u)
+                                tma_load_2d(sa + (Cfg::GR + q) * Cfg::T_BYTES, &tmX, &full[stage],
+                                            (cg * Cfg::GC + q) * B, ks * Cfg::MK);
+                        issued |= 1u << stage;
+                        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, good, 0)) {
+                    ok = false;
+                    break;
                 }
             }
+        }
+        if (lane == 0) {
             if (!ok) {
                 *abort_flag = 1;
                 set_status(args.status, BSL_ERR_TIMEOUT);
@@ -168,88 +207,97 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
         }
         __syncwarp();
     } else if (warp == Cfg::P) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc_bf16(128, B, true, true);
-            uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-            bool ok = true, any = false;
-            for (int g = blockIdx.x; g < ngroups && ok; g += gridDim.x) {
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, tmo, abort_flag)) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = make_idesc_bf16(128, Cfg::GC * B, true, true);
+        uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+        bool ok = true, any = false;
+        const uint32_t lead = lane == 0 ? 1u : 0u;
+        for (int t = blockIdx.x; t < args.ntiles && ok; t += gridDim.x) {
+            uint32_t rm, cm;
+            int rg, cg;
+            tile_blocks<B>(args, t, lane, &rm, &cm, &rg, &cg);
+            if (!rm) continue;
+            if (__any_sync(0xffffffffu, !mbar_wait(&tempty[acc], acc_phase ^ 1, tmo, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + acc * Cfg::ACC_COLS;
+            for (int ks = 0; ks < args.ksteps; ++ks) {
+                if (__any_sync(0xffffffffu, !mbar_wait(&full[stage], phase, tmo, abort_flag))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d = tmem_base + acc * B;
-                for (int ks = 0; ks < args.ksteps; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, tmo, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(stages + stage * Cfg::STAGE_BYTES);
-                    const uint32_t x0 = a0 + Cfg::G * Cfg::T_BYTES;
+                const uint32_t a0 = smem_u32(stages + stage * Cfg::STAGE_BYTES);
+                const uint32_t x0 = a0 + Cfg::GR * Cfg::T_BYTES;
+                // A: the GR dY strips side by side along M (MN-major, T_BYTES apart);
+                // B: the GC X strips along N; K = 16 rows of M per instruction
+                const uint64_t ad0 = make_sdesc(a0, Cfg::T_BYTES, Cfg::SBO, Cfg::LAYOUT);
+                const uint64_t xd0 = make_sdesc(x0, Cfg::T_BYTES, Cfg::SBO, Cfg::LAYOUT);
+                const uint32_t alo = static_cast<uint32_t>(ad0), ahi = static_cast<uint32_t>(ad0 >> 32);
+                const uint32_t xlo = static_cast<uint32_t>(xd0), xhi = static_cast<uint32_t>(xd0 >> 32);
+                constexpr uint32_t KSTEP = (16 * Cfg::ROW_BYTES) >> 4;
 #pragma unroll
-                    for (int k = 0; k < Cfg::MK / 16; ++k) {
-                        const uint64_t ad =
-                            make_sdesc(a0 + k * 16 * Cfg::ROW_BYTES, Cfg::T_BYTES, Cfg::SBO, Cfg::LAYOUT);
-                        const uint64_t xd =
-                            make_sdesc(x0 + k * 16 * Cfg::ROW_BYTES, Cfg::T_BYTES, Cfg::SBO, Cfg::LAYOUT);
-                        umma_bf16(d, ad, xd, idesc, (ks > 0 || k > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&empty[stage]);
-                    any = true;
-                    if (++stage == Cfg::STAGES) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
-                }
-                if (!ok) break;
-                umma_commit(&tfull[acc]);
-                if (++acc == Cfg::ACC) {
-                    acc = 0;
-                    acc_phase ^= 1;
+                for (int k = 0; k < Cfg::MK / 16; ++k)
+                    umma_bf16_lo_lead(lead, d, alo + k * KSTEP, ahi, xlo + k * KSTEP, xhi, idesc,
+                                      (ks > 0 || k > 0) ? 1u : 0u);
+                umma_commit_lead(lead, &empty[stage]);
+                any = true;
+                if (++stage == Cfg::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
                 }
             }
-            if (!ok) {
-                *abort_flag = 1;
-                set_status(args.status, BSL_ERR_TIMEOUT);
+            if (!ok) break;
+            umma_commit_lead(lead, &tfull[acc]);
+            __syncwarp();
+            if (++acc == Cfg::ACC) {
+                acc = 0;
+                acc_phase ^= 1;
             }
-            if (any) {
-                umma_commit(drain);
-                if (!mbar_wait(drain, 0, tmo, nullptr)) set_status(args.status, BSL_ERR_TIMEOUT);
-            }
+        }
+        if (lane == 0 && !ok) {
+            *abort_flag = 1;
+            set_status(args.status, BSL_ERR_TIMEOUT);
+        }
+        if (any) {
+            umma_commit_lead(lead, drain);
+            if (lane == 0 && !mbar_wait(drain, 0, tmo, nullptr)) set_status(args.status, BSL_ERR_TIMEOUT);
         }
         __syncwarp();
     } else {
-        const int et = threadIdx.x - (Cfg::P + 1) * 32;
+        // ------------------------------------------------------------ epilogue
+        // warp q reads TMEM lanes 32q..32q+31 = dW rows u of block row i of
+        // the tile (i = 32q / b, u = 32q % b + lane) and writes the stored
+        // blocks of that row: one 2b-byte row of each per thread.
         const int q = warp & 3;
-        const int l = q * 32 + lane;      // accumulator row = TMEM lane
-        const int blk_in_group = l / B, u = l % B;
+        const int i = (32 * q) / B;
+        const int u = (32 * q) % B + lane;
         uint32_t acc = 0, acc_phase = 0;
-        for (int g = blockIdx.x; g < ngroups; g += gridDim.x) {
-            const int c = group_column(args.dw_gptr, args.C, g);
-            const int j0 = args.col_ptr[c] + (g - args.dw_gptr[c]) * Cfg::G;
-            const int cnt = min(Cfg::G, args.col_ptr[c + 1] - j0);
-            if (et == 0) {
-                const bool go = mbar_wait(&tfull[acc], acc_phase, tmo, abort_flag);
-                if (!go) {
-                    *abort_flag = 1;
-                    set_status(args.status, BSL_ERR_TIMEOUT);
-                }
-                *epi_go = go ? 1 : 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < args.ntiles; t += gridDim.x) {
+            uint32_t rm, cm;
+            int rg, cg;
+            const int pos = tile_blocks<B>(args, t, lane, &rm, &cm, &rg, &cg);
+            if (!rm) continue;
+            int go = 1;
+            if (lane == 0) go = mbar_wait(&tfull[acc], acc_phase, tmo, abort_flag);
+            if (!__shfl_sync(0xffffffffu, go, 0)) {
+                ok = false;
+                break;
             }
-            named_bar_sync(1, 128);
-            if (!*epi_go) break;
             tc_fence_after();
-            uint32_t v[B];
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * B;
+#pragma unroll 1
+            for (int j = 0; j < Cfg::GC; ++j) {
+                const int p = __shfl_sync(0xffffffffu, pos, i * Cfg::GC + j);
+                if (p < 0) continue;
+                uint32_t v[B];
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS + j * B;
 #pragma unroll
-            for (int k = 0; k < B / 16; ++k)
-                tmem_ld16(taddr + k * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[k * 16]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
-            if (blk_in_group < cnt) {
-                const int p = args.csc_to_bsr[j0 + blk_in_group];
+                for (int k = 0; k < B / 16; ++k)
+                    tmem_ld16(taddr + k * 16, *reinterpret_cast<uint32_t(*)[16]>(&v[k * 16]));
+                tmem_wait_ld();
                 uint4 *dst = reinterpret_cast<uint4 *>(args.dW + (static_cast<int64_t>(p) * B + u) * B);
 #pragma unroll
                 for (int k = 0; k < B / 8; ++k) {
@@ -261,12 +309,20 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
                     dst[k] = pk;
                 }
             }
-            named_bar_sync(1, 128);  // everyone has read epi_go before it is rewritten
+            // every TMEM read of this accumulator is complete (each was waited)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
             if (++acc == Cfg::ACC) {
                 acc = 0;
                 acc_phase ^= 1;
             }
         }
+        if (lane == 0 && !ok) {
+            *abort_flag = 1;
+            set_status(args.status, BSL_ERR_TIMEOUT);
+        }
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -278,14 +334,13 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
 }
 
 template <int B>
-bsl_status run(const CUtensorMap &dy, const CUtensorMap &x, const SddmmArgs &args, int ngroups_max,
-               cudaStream_t s)
+bsl_status run(const CUtensorMap &dy, const CUtensorMap &x, const SddmmArgs &args, cudaStream_t s)
 {
     using Cfg = SddmmCfg<B>;
     auto kern = k_sddmm_tc<B>;
     const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(kern), Cfg::SMEM_BYTES);
     if (sa != BSL_OK) return sa;
-    const int grid = ngroups_max < num_sms() ? ngroups_max : num_sms();
+    const int grid = args.ntiles < num_sms() ? args.ntiles : num_sms();
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(dy, x, args);
     return cuda_status(cudaGetLastError());
 }
@@ -297,24 +352,24 @@ bsl_status launch_sddmm_tc(const void *dY, const void *X, int32_t M, const bsl_b
     const int B = W->b;
     if (W->nnz == 0) return BSL_OK;
     CUtensorMap mdy, mx;
-    if (!make_map_2d(&mdy, dY, W->N, M, static_cast<uint64_t>(W->N) * 2, B, kSddmmRows, 2 * B) ||
-        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, B, kSddmmRows, 2 * B))
+    if (!make_map_2d(&mdy, dY, W->N, M, static_cast<uint64_t>(W->N) * 2, B, 128, 2 * B) ||
+        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, B, 128, 2 * B))
         return BSL_ERR_CUDA;
+    const int G = 128 / B;
     SddmmArgs args;
     args.M = M;
+    args.R = W->N / B;
     args.C = W->K / B;
-    args.ksteps = (M + kSddmmRows - 1) / kSddmmRows;
-    args.col_ptr = W->col_ptr;
-    args.row_idx = W->row_idx;
-    args.csc_to_bsr = W->csc_to_bsr;
-    args.dw_gptr = W->dw_gptr;
+    args.ksteps = (M + 127) / 128;
+    args.nrg = (args.R + G - 1) / G;
+    args.ncg = (args.C + G - 1) / G;
+    args.ntiles = args.nrg * args.ncg;
+    args.row_ptr = W->row_ptr;
+    args.col_idx = W->col_idx;
     args.dW = static_cast<__nv_bfloat16 *>(dW);
     args.status = W->status;
     args.timeout_ns = wait_timeout_ns();
-    // groups <= nnz; the kernel reads the exact count from dw_gptr[C]
-    const int G = 128 / B;
-    const int gmax = W->nnz < args.C * ((W->N / B + G - 1) / G) ? W->nnz : args.C * ((W->N / B + G - 1) / G);
-    return B == 64 ? run<64>(mdy, mx, args, gmax, s) : run<32>(mdy, mx, args, gmax, s);
+    return B == 64 ? run<64>(mdy, mx, args, s) : run<32>(mdy, mx, args, s);
 }
 
 }  // namespace bsl

@@ -560,22 +560,26 @@ __global__ void __launch_bounds__(PairCfg<B>::THREADS, 1)
                 const uint4 h0 = hs[0];
                 const uint32_t xlo = rlo0 + h0.x * U_LO;
                 const int nr = static_cast<int>(h0.y);
-                auto issue_run = [&](uint32_t x, uint32_t y) {
-                    const uint32_t dcol = d0 + (x & 0xFFu);
-                    const uint32_t blo = rlo0 + ((x >> 8) & 0xFFu) * U_LO;
-                    const uint32_t st = (x >> 28) & 1u;
-#pragma unroll
-                    for (int kk = 0; kk < B / 16; ++kk)
-                        umma2_lead(lead, dcol, xlo + kk * 2, rhi, blo + kk * 2, rhi, y, kk ? 1u : st);
-                };
+                // K-step major over the runs: the runs accumulate into different TMEM
+                // columns, so consecutive MMAs are independent and the tensor pipe
+                // does not wait for one MMA's result before the next
+                uint32_t rx[Cfg::G], ry[Cfg::G];
 #pragma unroll
                 for (int wv = 1; wv < Cfg::HDR_V4; ++wv) {
-                    if (nr > 2 * (wv - 1)) {
-                        const uint4 h1 = hs[wv];
-                        issue_run(h1.x, h1.y);
-                        if (nr > 2 * (wv - 1) + 1) issue_run(h1.z, h1.w);
-                    }
+                    const uint4 h1 = nr > 2 * (wv - 1) ? hs[wv] : make_uint4(0, 0, 0, 0);
+                    rx[2 * (wv - 1)] = h1.x;
+                    ry[2 * (wv - 1)] = h1.y;
+                    rx[2 * (wv - 1) + 1] = h1.z;
+                    ry[2 * (wv - 1) + 1] = h1.w;
                 }
+#pragma unroll
+                for (int kk = 0; kk < B / 16; ++kk)
+#pragma unroll
+                    for (int r = 0; r < Cfg::G; ++r)
+                        if (r < nr)
+                            umma2_lead(lead, d0 + (rx[r] & 0xFFu), xlo + kk * 2, rhi,
+                                       rlo0 + ((rx[r] >> 8) & 0xFFu) * U_LO + kk * 2, rhi, ry[r],
+                                       kk ? 1u : ((rx[r] >> 28) & 1u));
                 umma2_commit_both(lead, &empty[slot]);  // the entry's slots are free in both CTAs
                 any = true;
             }

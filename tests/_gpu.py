@@ -13,7 +13,7 @@ def mask_dev(mask: np.ndarray) -> torch.Tensor:
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:
-    return t.float().cpu().numpy().astype(np.float64)
+    return t.detach().float().cpu().numpy().astype(np.float64)
 
 
 def bits(t: torch.Tensor) -> np.ndarray:

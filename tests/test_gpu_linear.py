@@ -106,7 +106,8 @@ def test_module_matches_oracle_and_sees_in_place_updates():
     with torch.no_grad():
         layer.values.mul_(2.0)
         layer.bias.zero_()
-    Y2 = layer(X.detach())
+    with torch.no_grad():
+        Y2 = layer(X.detach())
     W2 = synth.bf16_bits((synth.bits_to_f32(case["W"]) * 2.0).astype(np.float32))
     ref, S = oracle.forward(case["X"], W2, case["mask"], b)
     assert_parity(to_f64(Y2.reshape(M, N)), ref, S, "module Y after update")
@@ -115,7 +116,18 @@ def test_module_matches_oracle_and_sees_in_place_updates():
 def test_repack_in_place_with_a_new_mask():
     M, N, K, b, nnz = 300, 640, 448, 64, 30
     first = synth.random_case(M, N, K, b, nnz, 66)
-    second = synth.random_case(M, N, K, b, nnz, 67, empty_rows=(0, 9))
+    second = synth.random_case(M, N, K, b, nnz, 67)
+    # same block count, different pattern: block rows 0 and 9 emptied, their
+    # blocks moved to the free positions of other rows
+    m = second["mask"].copy()
+    moved = int(m[0].sum() + m[9].sum())
+    m[0] = 0
+    m[9] = 0
+    free = np.argwhere(m == 0)
+    free = free[(free[:, 0] != 0) & (free[:, 0] != 9)][:moved]
+    m[free[:, 0], free[:, 1]] = 1
+    second["mask"] = m
+    assert int(m.sum()) == nnz
     assert not np.array_equal(first["mask"], second["mask"])
     Wp = sg.pack(to_dev(first["W"]), mask_dev(first["mask"]), b)
     sg.forward_tc(to_dev(first["X"]), Wp)

@@ -296,7 +296,7 @@ def test_autograd_function_matches_oracle():
     case = synth.random_case(M, N, K, b, 40, 44)
     Wp = pack_dev(case, b)
     X = to_dev(case["X"]).requires_grad_(True)
-    vals = Wp.block_values().clone().requires_grad_(True)
+    vals = torch.nn.Parameter(Wp.block_values())  # the packed values themselves (the kernels read them)
     Y = sg.BlockSparseLinearFunction.apply(X, vals, Wp)
     Y.backward(to_dev(case["dY"]))
     ref, S = oracle.forward(case["X"], case["W"], case["mask"], b)
