@@ -178,12 +178,12 @@ BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W
  * with BSL_ERR_CUDA if the device has no room left, so make one call at
  * start-up, before the memory budget is spent.  From then on the device keeps
  * the array until the process exits.  The entry point allocates nothing
- * itself and calls no cudaMalloc / cudaFree.  It returns BSL_ERR_SCRATCH_TOO_SMALL, launching
- * nothing, when the call would need more scratch than that (the need is
- * bsl_forward_workspace_bytes(M, W) = SMs x 8 warps x 2 x b x M' x 4 bytes,
- * M' = 16 for M <= 16, else 32; on a 148-SM B200 that is 4.8 MB for b = 32,
- * M <= 16, and 9.7 MB for b = 32, M <= 32 or b = 64, M <= 16, which fit;
- * b = 64 with M > 16 needs 19.4 MB and is rejected).
+ * itself and calls no cudaMalloc / cudaFree.  It returns
+ * BSL_ERR_SCRATCH_TOO_SMALL, launching nothing, when the call would need more
+ * scratch than that.  The need is bsl_forward_workspace_bytes(M, W) =
+ * SMs x (2 x b x M' x 4 + 4) bytes, M' = 16 for M <= 16, else 32: at most
+ * 2.4 MB on a 148-SM B200 (b = 64, M <= 32), so every supported call fits
+ * there; only a device with more than about 1000 SMs would be turned away.
  *
  * The first call on each device also looks up the array's device address
  * (cudaGetSymbolAddress) and keeps it for the life of the process, so make

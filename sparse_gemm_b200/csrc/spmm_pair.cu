@@ -197,6 +197,7 @@ struct PairCfg {
     static constexpr int RU = B == 64 ? 46 : 192;       // ring units (184 KB or 192 KB)
     static constexpr int UPL = (RU + 31) / 32;          // ring units tracked per lane
     static constexpr int SE = 16;                       // entries in flight at most (barriers, headers)
+    static constexpr int W = 16 / G;                    // entries the MMA issuer interleaves
     static constexpr int P = 4;                         // producer warps
     static constexpr int UR = 16;                       // unit-id ring
     static constexpr int W_MMA = P;
@@ -550,38 +551,53 @@ __global__ void __launch_bounds__(PairCfg<B>::THREADS, 1)
             }
             tc_fence_after();
             const uint32_t d0 = tmem_base + acc * Cfg::ACC_COLS;
-            for (int t = z; t < zend; ++t, ++e) {
-                const int slot = e % Cfg::SE;
-                if (__any_sync(0xffffffffu, !mbar_wait(&full[slot], (e / Cfg::SE) & 1, tmo, abort_flag))) {
+            // Entries are issued a window of W at a time, K-step major over all
+            // the window's runs: consecutive MMAs then accumulate into different
+            // TMEM columns (other members, other runs), so the tensor pipe does not
+            // wait for one MMA's result before starting the next.  MMAs that do
+            // share a member keep their order within each K step, so the first
+            // (overwriting) MMA of a member still comes first.
+            for (int t = z; t < zend;) {
+                const int nw = min(Cfg::W, zend - t);
+                bool bad = false;
+                for (int i = 0; i < nw; ++i)
+                    bad |= !mbar_wait(&full[(e + i) % Cfg::SE], ((e + i) / Cfg::SE) & 1, tmo, abort_flag);
+                if (__any_sync(0xffffffffu, bad)) {
                     ok = false;
                     break;
                 }
-                const uint4 *hs = hdr + slot * Cfg::HDR_V4;
-                const uint4 h0 = hs[0];
-                const uint32_t xlo = rlo0 + h0.x * U_LO;
-                const int nr = static_cast<int>(h0.y);
-                // K-step major over the runs: the runs accumulate into different TMEM
-                // columns, so consecutive MMAs are independent and the tensor pipe
-                // does not wait for one MMA's result before the next
-                uint32_t rx[Cfg::G], ry[Cfg::G];
+                // runs of the window: x = TMEM column | ring unit of the run's first
+                // half-block << 8 | ring unit of its activation half-tile << 16 |
+                // overwrite-free flag << 28; y = instruction descriptor (0: no run)
+                uint32_t rx[Cfg::W * Cfg::G], ry[Cfg::W * Cfg::G];
 #pragma unroll
-                for (int wv = 1; wv < Cfg::HDR_V4; ++wv) {
-                    const uint4 h1 = nr > 2 * (wv - 1) ? hs[wv] : make_uint4(0, 0, 0, 0);
-                    rx[2 * (wv - 1)] = h1.x;
-                    ry[2 * (wv - 1)] = h1.y;
-                    rx[2 * (wv - 1) + 1] = h1.z;
-                    ry[2 * (wv - 1) + 1] = h1.w;
+                for (int i = 0; i < Cfg::W; ++i) {
+                    const uint4 *hs = hdr + ((e + i) % Cfg::SE) * Cfg::HDR_V4;
+                    const uint4 h0 = i < nw ? hs[0] : make_uint4(0, 0, 0, 0);
+                    const int nr = static_cast<int>(h0.y);
+#pragma unroll
+                    for (int wv = 1; wv < Cfg::HDR_V4; ++wv) {
+                        const uint4 h1 = nr > 2 * (wv - 1) ? hs[wv] : make_uint4(0, 0, 0, 0);
+                        const int r0 = i * Cfg::G + 2 * (wv - 1);
+                        rx[r0] = h1.x | (h0.x << 16);
+                        ry[r0] = nr > 2 * (wv - 1) ? h1.y : 0u;
+                        rx[r0 + 1] = h1.z | (h0.x << 16);
+                        ry[r0 + 1] = nr > 2 * (wv - 1) + 1 ? h1.w : 0u;
+                    }
                 }
 #pragma unroll
                 for (int kk = 0; kk < B / 16; ++kk)
 #pragma unroll
-                    for (int r = 0; r < Cfg::G; ++r)
-                        if (r < nr)
-                            umma2_lead(lead, d0 + (rx[r] & 0xFFu), xlo + kk * 2, rhi,
-                                       rlo0 + ((rx[r] >> 8) & 0xFFu) * U_LO + kk * 2, rhi, ry[r],
+                    for (int r = 0; r < Cfg::W * Cfg::G; ++r)
+                        if (ry[r])
+                            umma2_lead(lead, d0 + (rx[r] & 0xFFu), rlo0 + ((rx[r] >> 16) & 0xFFu) * U_LO + kk * 2,
+                                       rhi, rlo0 + ((rx[r] >> 8) & 0xFFu) * U_LO + kk * 2, rhi, ry[r],
                                        kk ? 1u : ((rx[r] >> 28) & 1u));
-                umma2_commit_both(lead, &empty[slot]);  // the entry's slots are free in both CTAs
+                for (int i = 0; i < nw; ++i)
+                    umma2_commit_both(lead, &empty[(e + i) % Cfg::SE]);  // the entry's slots are free in both CTAs
                 any = true;
+                e += nw;
+                t += nw;
             }
             if (!ok) break;
             if (zend > z) {

@@ -9,27 +9,30 @@
 //
 // Decomposition: the BSR block list [0, nnz) is cut into equal contiguous
 // shares, one per warp of a one-CTA-per-SM grid (block counts, not block
-// rows, are balanced).  Each warp streams its share through its own ring of
-// slots; a slot holds one weight block and the activation slice
-// X[0:MP, c*b:(c+1)*b] it multiplies, both brought in by TMA (swizzled rows,
-// rows past M read as zeros).  Every warp issues its own copies (one thread
-// starts only a few copies per microsecond), and a ring usually holds the
-// warp's whole share, so all its loads are in flight from the start.  The
-// operands go to registers with ldmatrix; mma.sync m16n8k16 (bf16 in, fp32
-// accumulate) forms Y^T[n][m] = W_blk[n][:] . X[m][:], and the partial sum
-// of the current block row stays in registers:
+// rows, are balanced; the 8 warps of a CTA hold consecutive shares).  Each
+// warp streams its share through its own ring of slots; a slot holds one
+// weight block and the activation slice X[0:MP, c*b:(c+1)*b] it multiplies,
+// both brought in by TMA (swizzled rows, rows past M read as zeros).  The
+// weight copies, which depend on nothing, leave first; a ring usually holds
+// the warp's whole share.  The operands go to registers with ldmatrix;
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate) forms
+// Y^T[n][m] = W_blk[n][:] . X[m][:], and the sum of the current block row
+// stays in registers:
 //   - a block row entirely inside the warp's share is finished there: bias
-//     added, rounded to bf16, staged in shared memory and written to Y with
+//     added, rounded to bf16, staged in shared memory, written to Y with
 //     16-byte stores;
-//   - a block row cut by share boundaries leaves an fp32 partial in the
-//     workspace (slot 0 if it is the share's first row, else slot 1); each
-//     contributor then counts itself in on the row's counter, and the last to
-//     arrive sums the partials of all contributors in warp order and writes
-//     the row.  The sum order does not depend on who arrives last, so
-//     results are identical run to run.
-// Block rows without blocks are written (bias or zeros) by warp r % warps.
-// The counters are zeroed on the stream before every launch, so nothing in
-// the workspace has to survive from one call to the next.
+//   - a block row cut by share boundaries leaves an fp32 partial.  After all
+//     warps of the CTA are done, the partials sit in their rings and the
+//     CTA's first contributor to each cut row adds them in warp order.  A row
+//     that lies inside the CTA's share is then written; a row that reaches
+//     into other CTAs' shares leaves the CTA's sum in the workspace, and the
+//     last CTA to count itself in on the row's counter adds the CTAs' sums in
+//     CTA order and writes the row.
+// Every sum has a fixed order (the same whoever arrives last), so results
+// are identical run to run.  Block rows without blocks are written (bias or
+// zeros) at the end.  The counters are zeroed on the stream before every
+// launch, so nothing in the workspace has to survive from one call to the
+// next.
 #include "common.cuh"
 #include "internal.h"
 
@@ -53,13 +56,14 @@ struct StreamCfg {
         kStreamWarps * (WARP_BYTES + OUT_BYTES) + kStreamWarps * NSLOT * 8 + 1024;
     static_assert(NSLOT >= 2, "ring too small");
     static_assert(SLOT % 1024 == 0 && W_BLK % 1024 == 0, "slot alignment for the swizzled copies");
+    static_assert(2 * PART * 4 <= WARP_BYTES, "a warp's two partials fit in its ring");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct StreamArgs {
     __nv_bfloat16 *Y;
-    float *ws;                  // [GW][2][b*MP] partials
-    int32_t *cnt;               // [GW] arrival counters (zero at launch)
+    float *ws;                  // [CTAs][2][b*MP] partial sums of rows cut between CTAs
+    int32_t *cnt;               // [CTAs] arrival counters (zero at launch)
     const int32_t *row_ptr, *col_idx;
     const __nv_bfloat16 *bias;  // [N] added to every output row (null: none)
     int32_t M, N, K, R, C, nnz;
@@ -72,22 +76,21 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// first block of warp share gw when nnz blocks are split over GW warps
-__device__ __forceinline__ int share_begin(int gw, int GW, int nnz)
+// first block of share u when nnz blocks are split over U shares
+__device__ __forceinline__ int share_begin(int u, int U, int nnz)
 {
-    return static_cast<int>((static_cast<int64_t>(gw) * nnz) / GW);
+    return static_cast<int>((static_cast<int64_t>(u) * nnz) / U);
 }
 
-// the warp whose share holds block p (the last gw with share_begin(gw) <= p);
-// share_begin(gw) = floor(gw * nnz / GW), so gw is within one of
-// floor(p * GW / nnz)
-__device__ __forceinline__ int warp_of(int p, int GW, int nnz)
+// the share that holds block p (the last u with share_begin(u) <= p);
+// share_begin(u) = floor(u * nnz / U), so u is within one of floor(p * U / nnz)
+__device__ __forceinline__ int share_of(int p, int U, int nnz)
 {
-    int w = static_cast<int>((static_cast<int64_t>(p) * GW) / nnz);
-    w = w < 0 ? 0 : (w > GW - 1 ? GW - 1 : w);
-    while (w > 0 && share_begin(w, GW, nnz) > p) --w;
-    while (w + 1 < GW && share_begin(w + 1, GW, nnz) <= p) ++w;
-    return w;
+    int u = static_cast<int>((static_cast<int64_t>(p) * U) / nnz);
+    u = u < 0 ? 0 : (u > U - 1 ? U - 1 : u);
+    while (u > 0 && share_begin(u, U, nnz) > p) --u;
+    while (u + 1 < U && share_begin(u + 1, U, nnz) <= p) ++u;
+    return u;
 }
 
 template <int B>
@@ -128,7 +131,25 @@ struct RowAcc {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) d[i][j][e] = 0.f;
     }
+    // store as floats, element (feature n, token m) at n * MP + m
+    __device__ __forceinline__ void store(float *dst, int lane) const
+    {
+        const int g = lane >> 2, c2 = (lane & 3) * 2;
+#pragma unroll
+        for (int i = 0; i < MT; ++i)
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    *reinterpret_cast<float2 *>(dst + (i * 16 + g + h * 8) * MP + j * 8 + c2) =
+                        make_float2(d[i][j][2 * h], d[i][j][2 * h + 1]);
+    }
 };
+
+__device__ __forceinline__ float bias_of(const StreamArgs &a, int64_t col)
+{
+    return a.bias ? __bfloat162float(a.bias[col]) : 0.f;
+}
 
 // Write M rows of block row r from the warp's bf16 staging ([MP][b]) with
 // 16-byte stores.
@@ -145,77 +166,39 @@ __device__ __forceinline__ void store_staged(const StreamArgs &a, const uint8_t 
     __syncwarp();
 }
 
-__device__ __forceinline__ float bias_of(const StreamArgs &a, int64_t col)
-{
-    return a.bias ? __bfloat162float(a.bias[col]) : 0.f;
-}
-
-// A finished block row: either the whole row (written to Y) or this warp's
-// part of a row shared with other warps (fp32 partial, then the last of the
-// row's contributors writes the row).
+// A whole block row held in registers: bias, bf16, staged, stored.
 template <int B, int MP>
-__device__ void finish_row(const RowAcc<B, MP> &acc, const StreamArgs &a, int r, int gw, int GW, int q0,
-                           uint8_t *stage, int lane)
+__device__ __forceinline__ void write_row(const RowAcc<B, MP> &acc, const StreamArgs &a, int r, uint8_t *stage,
+                                          int lane)
 {
     const int g = lane >> 2, c2 = (lane & 3) * 2;
-    const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
-    const int q1 = share_begin(gw + 1, GW, a.nnz);
-    if (beg >= q0 && end <= q1) {  // whole row in this share
-#pragma unroll
-        for (int i = 0; i < RowAcc<B, MP>::MT; ++i)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int n = i * 16 + g + h * 8;
-                const float bb = bias_of(a, static_cast<int64_t>(r) * B + n);
-#pragma unroll
-                for (int j = 0; j < RowAcc<B, MP>::NT; ++j) {
-                    const int m = j * 8 + c2;
-                    __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(stage);
-                    s[m * B + n] = __float2bfloat16_rn(acc.d[i][j][2 * h] + bb);
-                    s[(m + 1) * B + n] = __float2bfloat16_rn(acc.d[i][j][2 * h + 1] + bb);
-                }
-            }
-        store_staged<B, MP>(a, stage, r, lane);
-        return;
-    }
-    // partial: slot 0 if the row is this share's first row, else slot 1
-    constexpr int PART = StreamCfg<B, MP>::PART;
-    float *mine = a.ws + (static_cast<int64_t>(gw) * 2 + (q0 >= beg ? 0 : 1)) * PART;
+    __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(stage);
 #pragma unroll
     for (int i = 0; i < RowAcc<B, MP>::MT; ++i)
 #pragma unroll
-        for (int j = 0; j < RowAcc<B, MP>::NT; ++j)
+        for (int h = 0; h < 2; ++h) {
+            const int n = i * 16 + g + h * 8;
+            const float bb = bias_of(a, static_cast<int64_t>(r) * B + n);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int n = i * 16 + g + h * 8, m = j * 8 + c2;
-                __stcg(reinterpret_cast<float2 *>(mine + n * MP + m),
-                       make_float2(acc.d[i][j][2 * h], acc.d[i][j][2 * h + 1]));
+            for (int j = 0; j < RowAcc<B, MP>::NT; ++j) {
+                const int m = j * 8 + c2;
+                s[m * B + n] = __float2bfloat16_rn(acc.d[i][j][2 * h] + bb);
+                s[(m + 1) * B + n] = __float2bfloat16_rn(acc.d[i][j][2 * h + 1] + bb);
             }
-    const int w0 = warp_of(beg, GW, a.nnz), w1 = warp_of(end - 1, GW, a.nnz);
-    int contributors = 0;
-    for (int w = w0; w <= w1; ++w) contributors += share_begin(w + 1, GW, a.nnz) > share_begin(w, GW, a.nnz);
-    __threadfence();  // every lane's part of the partial is visible before the count says so
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(a.cnt + w0, 1) == contributors - 1;
-    if (!__shfl_sync(0xffffffffu, last, 0)) return;
-    __threadfence();  // the other contributors' partials are read after their counts
-    // last contributor: sum every contributor's partial in warp order
-    constexpr int PER = PART / 32;
-    float sum[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) sum[e] = 0.f;
-    for (int w = w0; w <= w1; ++w) {
-        const int sb = share_begin(w, GW, a.nnz);
-        if (share_begin(w + 1, GW, a.nnz) == sb) continue;  // empty share wrote nothing
-        const float *src = a.ws + (static_cast<int64_t>(w) * 2 + (sb >= beg ? 0 : 1)) * PART;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) sum[e] += __ldcg(src + e * 32 + lane);
-    }
+        }
+    store_staged<B, MP>(a, stage, r, lane);
+}
+
+// A block row held as floats (n * MP + m, PER = b*MP/32 per lane): bias,
+// bf16, staged, stored.
+template <int B, int MP>
+__device__ __forceinline__ void write_row_flat(const float (&sum)[B * MP / 32], const StreamArgs &a, int r,
+                                               uint8_t *stage, int lane)
+{
     __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(stage);
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-        const int idx = e * 32 + lane;  // = n * MP + m
+    for (int e = 0; e < B * MP / 32; ++e) {
+        const int idx = e * 32 + lane;
         const int n = idx / MP, m = idx % MP;
         s[m * B + n] = __float2bfloat16_rn(sum[e] + bias_of(a, static_cast<int64_t>(r) * B + n));
     }
@@ -228,6 +211,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                  const StreamArgs a)
 {
     using Cfg = StreamCfg<B, MP>;
+    constexpr int PER = Cfg::PART / 32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -238,127 +222,139 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
 
     const int GW = gridDim.x * kStreamWarps;
     const int gw = blockIdx.x * kStreamWarps + warp;
-
-    // block rows without blocks: bias (or zeros), rows r = gw, gw + GW, ...
-    for (int r = gw; r < a.R; r += GW) {
-        if (a.row_ptr[r + 1] != a.row_ptr[r]) continue;
-        __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(stage);
-        for (int idx = lane; idx < MP * B; idx += 32)
-            s[idx] = __float2bfloat16_rn(bias_of(a, static_cast<int64_t>(r) * B + (idx % B)));
-        store_staged<B, MP>(a, stage, r, lane);
-    }
-
     const int q0 = share_begin(gw, GW, a.nnz), q1 = share_begin(gw + 1, GW, a.nnz);
-    if (q0 >= q1) return;  // no block for this warp (no block-wide sync follows)
-    const int nblk = q1 - q0;
+    const int cq0 = share_begin(blockIdx.x * kStreamWarps, GW, a.nnz);          // this CTA's blocks
+    const int cq1 = share_begin((blockIdx.x + 1) * kStreamWarps, GW, a.nnz);
+    const int nblk = q1 > q0 ? q1 - q0 : 0;
+    const int nfirst = nblk < Cfg::NSLOT ? nblk : Cfg::NSLOT;
 
-    // block columns of 32 consecutive blocks of the share, one per lane
-    int cbase = q0;
-    int cidx = q0 + lane < q1 ? a.col_idx[q0 + lane] : 0;
-    auto col_of = [&](int p) {  // warp-uniform p; refreshes the lane cache when p leaves it
-        if (p >= cbase + 32) {
-            cbase = p;
-            cidx = p + lane < q1 ? a.col_idx[p + lane] : 0;
-        }
-        const int c = __shfl_sync(0xffffffffu, cidx, p - cbase);
-        return c >= 0 && c < a.C ? c : 0;  // a column outside the weight (bad index) reads column 0
-    };
-    auto issue = [&](int t, int c) {  // lane 0: block q0 + t and its activation slice into slot t % NSLOT
-        const int s = t % Cfg::NSLOT;
-        uint8_t *dst = ring + s * Cfg::SLOT;
-        mbar_arrive_expect_tx(&bars[s], Cfg::SLOT);
-        tma_load_2d(dst, &tmW, &bars[s], 0, (q0 + t) * B);
-        tma_load_2d(dst + Cfg::W_BLK, &tmX, &bars[s], c * B, 0);
-    };
-    if (lane == 0) {
+    // the weight blocks depend on nothing: their copies go out first, each
+    // slot armed for its block and activation slice together
+    if (lane == 0 && nblk > 0) {
         for (int s = 0; s < Cfg::NSLOT; ++s) mbar_init(&bars[s], 1);
         fence_barrier_init();
+        for (int t = 0; t < nfirst; ++t) {
+            mbar_arrive_expect_tx(&bars[t], Cfg::SLOT);
+            tma_load_2d(ring + t * Cfg::SLOT, &tmW, &bars[t], 0, (q0 + t) * B);
+        }
     }
     __syncwarp();
-    const int nfirst = nblk < Cfg::NSLOT ? nblk : Cfg::NSLOT;
-    for (int t = 0; t < nfirst; ++t) {
-        const int c = col_of(q0 + t);
-        if (lane == 0) issue(t, c);
-    }
 
-    // first block row of the share: last r with row_ptr[r] <= q0, by a
-    // warp-parallel search (two or three rounds of one load per lane)
-    int lo = 0, hi = a.R;  // row_ptr[lo] <= q0 < row_ptr[hi]
-    while (hi - lo > 1) {
-        const int step = (hi - lo + 31) / 32;
-        const int probe = lo + lane * step;
-        const bool le = probe < hi && a.row_ptr[probe] <= q0;
-        const int last = 31 - __clz(__ballot_sync(0xffffffffu, le));  // lane 0 always qualifies
-        lo = lo + last * step;
-        hi = min(hi, lo + step);
-    }
-    int r = lo;
-    int rbase = r;
-    int rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
-    int row_end = __shfl_sync(0xffffffffu, rp, 0);
-
-    RowAcc<B, MP> acc;
+    RowAcc<B, MP> acc, part0;  // the current row; the share's first row when it is cut
     acc.zero();
-    bool have = false, ok = true;
+    part0.zero();
+    int first_row = 0, last_row = -1;  // rows of blocks q0 and q1 - 1
+    bool cut_first = false, cut_last = false, ok = true;
     int issued = nfirst;
-    constexpr int KK = B / 16;
 
-    for (int t = 0; t < nblk; ++t) {
-        const int p = q0 + t;
-        while (p >= row_end) {  // leaving block row r
-            if (have) {
-                finish_row<B, MP>(acc, a, r, gw, GW, q0, stage, lane);
-                acc.zero();
-                have = false;
+    if (nblk > 0) {
+        // block columns of 32 consecutive blocks of the share, one per lane
+        int cbase = q0;
+        int cidx = q0 + lane < q1 ? a.col_idx[q0 + lane] : 0;
+        auto col_of = [&](int p) {  // warp-uniform p; refreshes the lane cache when p leaves it
+            if (p >= cbase + 32) {
+                cbase = p;
+                cidx = p + lane < q1 ? a.col_idx[p + lane] : 0;
             }
-            ++r;
-            if (r - rbase >= 32) {  // refresh the lane cache of row ends
-                rbase = r;
-                rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
-            }
-            row_end = __shfl_sync(0xffffffffu, rp, r - rbase);
+            const int c = __shfl_sync(0xffffffffu, cidx, p - cbase);
+            return c >= 0 && c < a.C ? c : 0;  // a column outside the weight (bad index) reads column 0
+        };
+        // the activation slices of the first blocks, once their columns are known
+        for (int t = 0; t < nfirst; ++t) {
+            const int c = col_of(q0 + t);
+            if (lane == 0) tma_load_2d(ring + t * Cfg::SLOT + Cfg::W_BLK, &tmX, &bars[t], c * B, 0);
         }
-        const int s = t % Cfg::NSLOT;
-        const bool landed = mbar_wait(&bars[s], (t / Cfg::NSLOT) & 1, a.timeout_ns, nullptr);
-        if (!__all_sync(0xffffffffu, landed)) {  // uniform decision across the warp
-            ok = false;
-            break;
+
+        // first block row of the share: last r with row_ptr[r] <= q0, by a
+        // warp-parallel search (two or three rounds of one load per lane)
+        int lo = 0, hi = a.R;  // row_ptr[lo] <= q0 < row_ptr[hi]
+        while (hi - lo > 1) {
+            const int step = (hi - lo + 31) / 32;
+            const int probe = lo + lane * step;
+            const bool le = probe < hi && a.row_ptr[probe] <= q0;
+            const int last = 31 - __clz(__ballot_sync(0xffffffffu, le));  // lane 0 always qualifies
+            lo = lo + last * step;
+            hi = min(hi, lo + step);
         }
-        have = true;
-        const uint32_t wbase = smem_u32(ring + s * Cfg::SLOT);
-        const uint32_t xbase = wbase + Cfg::W_BLK;
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) {
-            // activation fragments of this k step: two 8-token tiles per ldmatrix.x4
-            uint32_t xb[RowAcc<B, MP>::NT][2];
-#pragma unroll
-            for (int j = 0; j < RowAcc<B, MP>::NT; j += 2) {
-                const int tok = (j + (lane >> 4)) * 8 + (lane & 7);
-                const int chunk = kk * 2 + ((lane >> 3) & 1);
-                ldmatrix_x4(xbase + tok * Cfg::ROW_BYTES + swz_chunk<B>(chunk, tok) * 16, xb[j][0], xb[j][1],
-                            xb[j + 1][0], xb[j + 1][1]);
+        first_row = lo;
+        int r = lo;
+        int rbase = r;
+        int rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
+        int row_end = __shfl_sync(0xffffffffu, rp, 0);
+        cut_first = a.row_ptr[first_row] < q0;
+        bool have = false;
+        constexpr int KK = B / 16;
+
+        for (int t = 0; t < nblk; ++t) {
+            const int p = q0 + t;
+            while (p >= row_end) {  // leaving block row r (which ended inside the share)
+                if (have) {
+                    if (r == first_row && cut_first) part0 = acc;
+                    else write_row<B, MP>(acc, a, r, stage, lane);
+                    acc.zero();
+                    have = false;
+                }
+                ++r;
+                if (r - rbase >= 32) {  // refresh the lane cache of row ends
+                    rbase = r;
+                    rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
+                }
+                row_end = __shfl_sync(0xffffffffu, rp, r - rbase);
             }
+            const int s = t % Cfg::NSLOT;
+            const bool landed = mbar_wait(&bars[s], (t / Cfg::NSLOT) & 1, a.timeout_ns, nullptr);
+            if (!__all_sync(0xffffffffu, landed)) {  // uniform decision across the warp
+                ok = false;
+                break;
+            }
+            have = true;
+            const uint32_t wbase = smem_u32(ring + s * Cfg::SLOT);
+            const uint32_t xbase = wbase + Cfg::W_BLK;
 #pragma unroll
-            for (int i = 0; i < RowAcc<B, MP>::MT; ++i) {
-                const int row = i * 16 + (lane & 15);  // weight row inside the block
-                const int chunk = kk * 2 + (lane >> 4);
-                uint32_t a0, a1, a2, a3;
-                ldmatrix_x4(wbase + row * Cfg::ROW_BYTES + swz_chunk<B>(chunk, row) * 16, a0, a1, a2, a3);
+            for (int kk = 0; kk < KK; ++kk) {
+                // activation fragments of this k step: two 8-token tiles per ldmatrix.x4
+                uint32_t xb[RowAcc<B, MP>::NT][2];
 #pragma unroll
-                for (int j = 0; j < RowAcc<B, MP>::NT; ++j)
-                    mma_bf16_16816(acc.d[i][j], a0, a1, a2, a3, xb[j][0], xb[j][1]);
+                for (int j = 0; j < RowAcc<B, MP>::NT; j += 2) {
+                    const int tok = (j + (lane >> 4)) * 8 + (lane & 7);
+                    const int chunk = kk * 2 + ((lane >> 3) & 1);
+                    ldmatrix_x4(xbase + tok * Cfg::ROW_BYTES + swz_chunk<B>(chunk, tok) * 16, xb[j][0], xb[j][1],
+                                xb[j + 1][0], xb[j + 1][1]);
+                }
+#pragma unroll
+                for (int i = 0; i < RowAcc<B, MP>::MT; ++i) {
+                    const int row = i * 16 + (lane & 15);  // weight row inside the block
+                    const int chunk = kk * 2 + (lane >> 4);
+                    uint32_t a0, a1, a2, a3;
+                    ldmatrix_x4(wbase + row * Cfg::ROW_BYTES + swz_chunk<B>(chunk, row) * 16, a0, a1, a2, a3);
+#pragma unroll
+                    for (int j = 0; j < RowAcc<B, MP>::NT; ++j)
+                        mma_bf16_16816(acc.d[i][j], a0, a1, a2, a3, xb[j][0], xb[j][1]);
+                }
+            }
+            // the slot is read: refill it with the block NSLOT ahead
+            const int tn = t + Cfg::NSLOT;
+            if (tn < nblk) {
+                const int c = col_of(q0 + tn);
+                __syncwarp();
+                if (lane == 0) {
+                    fence_async_smem();  // ldmatrix reads of this slot precede the next TMA write
+                    mbar_arrive_expect_tx(&bars[s], Cfg::SLOT);
+                    tma_load_2d(ring + s * Cfg::SLOT, &tmW, &bars[s], 0, (q0 + tn) * B);
+                    tma_load_2d(ring + s * Cfg::SLOT + Cfg::W_BLK, &tmX, &bars[s], c * B, 0);
+                }
+                issued = tn + 1;
             }
         }
-        // the slot is read: refill it with the block NSLOT ahead
-        const int tn = t + Cfg::NSLOT;
-        if (tn < nblk) {
-            const int c = col_of(q0 + tn);
-            __syncwarp();
-            if (lane == 0) {
-                fence_async_smem();  // ldmatrix reads of this slot precede the next TMA write
-                issue(tn, c);
+        if (ok) {
+            last_row = r;
+            cut_last = row_end > q1;
+            if (last_row == first_row && cut_first) {
+                part0 = acc;  // the share lies inside one row cut at its start: one partial
+                cut_last = false;
+            } else if (!cut_last) {
+                write_row<B, MP>(acc, a, last_row, stage, lane);
             }
-            issued = tn + 1;
         }
     }
     if (!ok) {
@@ -370,10 +366,81 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                 mbar_wait(&bars[s], (lastt / Cfg::NSLOT) & 1, a.timeout_ns, nullptr);
             }
         }
-        __syncwarp();
-        return;
+        cut_first = cut_last = false;  // nothing of this warp is combined
     }
-    if (have) finish_row<B, MP>(acc, a, r, gw, GW, q0, stage, lane);
+    // the ring is read out: it now holds the warp's partials, [0] = first row
+    // cut at the share's start, [1] = last row cut at its end
+    float *myparts = reinterpret_cast<float *>(ring);
+    __syncwarp();
+    if (cut_first) part0.store(myparts, lane);
+    if (cut_last) acc.store(myparts + Cfg::PART, lane);
+    __syncthreads();
+
+    // Cut rows.  The CTA's first contributor to a row (the warp whose share
+    // holds the row's first block inside this CTA) adds the CTA's partials of
+    // that row in warp order.
+    const int w_lo = blockIdx.x * kStreamWarps;
+    for (int which = 0; which < 2; ++which) {
+        const bool mine = which == 0 ? cut_first : cut_last;
+        if (!mine) continue;
+        const int r = which == 0 ? first_row : last_row;
+        const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
+        const int lead = share_of(beg > cq0 ? beg : cq0, GW, a.nnz);
+        if (lead != gw) continue;
+        float sum[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) sum[e] = 0.f;
+        const int wl = share_of(end - 1 < cq1 - 1 ? end - 1 : cq1 - 1, GW, a.nnz);
+        for (int w = gw; w <= wl; ++w) {
+            const int sb = share_begin(w, GW, a.nnz);
+            if (share_begin(w + 1, GW, a.nnz) == sb) continue;  // empty share: no partial
+            // slot 0 holds a row that began before the warp's share, slot 1 the rest
+            const float *src = reinterpret_cast<const float *>(smem + (w - w_lo) * Cfg::WARP_BYTES) +
+                               (sb > beg ? 0 : Cfg::PART);
+#pragma unroll
+            for (int e = 0; e < PER; ++e) sum[e] += src[e * 32 + lane];
+        }
+        if (beg >= cq0 && end <= cq1) {  // the whole row lies in this CTA's share
+            write_row_flat<B, MP>(sum, a, r, stage, lane);
+            continue;
+        }
+        // the row reaches into other CTAs: this CTA's sum goes to the workspace;
+        // the last CTA to arrive adds all of them in CTA order
+        float *mine_ws = a.ws + (static_cast<int64_t>(blockIdx.x) * 2 + (cq0 >= beg ? 0 : 1)) * Cfg::PART;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) __stcg(mine_ws + e * 32 + lane, sum[e]);
+        // CTAs holding the row's first and last block (CTA c owns warps 8c .. 8c+7)
+        const int c0 = share_of(beg, GW, a.nnz) / kStreamWarps;
+        const int c1 = share_of(end - 1, GW, a.nnz) / kStreamWarps;
+        int contributors = 0;
+        for (int c = c0; c <= c1; ++c)
+            contributors += share_begin((c + 1) * kStreamWarps, GW, a.nnz) > share_begin(c * kStreamWarps, GW, a.nnz);
+        __threadfence();  // every lane's part of the sum is visible before the count says so
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(a.cnt + c0, 1) == contributors - 1;
+        if (!__shfl_sync(0xffffffffu, last, 0)) continue;
+        __threadfence();  // the other CTAs' sums are read after their counts
+#pragma unroll
+        for (int e = 0; e < PER; ++e) sum[e] = 0.f;
+        for (int c = c0; c <= c1; ++c) {
+            const int cb = share_begin(c * kStreamWarps, GW, a.nnz);
+            if (share_begin((c + 1) * kStreamWarps, GW, a.nnz) == cb) continue;  // empty CTA share
+            const float *src = a.ws + (static_cast<int64_t>(c) * 2 + (cb >= beg ? 0 : 1)) * Cfg::PART;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) sum[e] += __ldcg(src + e * 32 + lane);
+        }
+        write_row_flat<B, MP>(sum, a, r, stage, lane);
+    }
+
+    // block rows without blocks: bias (or zeros), rows r = gw, gw + GW, ...
+    for (int r = gw; r < a.R; r += GW) {
+        if (a.row_ptr[r + 1] != a.row_ptr[r]) continue;
+        __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(stage);
+        for (int idx = lane; idx < MP * B; idx += 32)
+            s[idx] = __float2bfloat16_rn(bias_of(a, static_cast<int64_t>(r) * B + (idx % B)));
+        store_staged<B, MP>(a, stage, r, lane);
+    }
 }
 
 template <int B, int MP>
@@ -381,9 +448,8 @@ bsl_status run(const void *X, const void *values, StreamArgs a, cudaStream_t s)
 {
     using Cfg = StreamCfg<B, MP>;
     const int grid = num_sms();
-    const int GW = grid * kStreamWarps;
     // counters start at zero on every launch (stream order)
-    cudaError_t e = cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(GW) * sizeof(int32_t), s);
+    cudaError_t e = cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(grid) * sizeof(int32_t), s);
     if (e != cudaSuccess) return cuda_status(e);
     CUtensorMap mw, mx;
     if (!make_map_2d(&mw, a.nnz > 0 ? values : X, B, static_cast<uint64_t>(a.nnz > 0 ? a.nnz : 1) * B, 2 * B, B, B,
@@ -400,14 +466,14 @@ bsl_status run(const void *X, const void *values, StreamArgs a, cudaStream_t s)
 size_t partials_bytes(int32_t M, int32_t b)
 {
     const int MP = M <= 16 ? 16 : 32;
-    return static_cast<size_t>(num_sms()) * kStreamWarps * 2 * b * MP * sizeof(float);
+    return static_cast<size_t>(num_sms()) * 2 * b * MP * sizeof(float);
 }
 
 }  // namespace
 
 size_t stream_workspace_bytes(int32_t M, const bsl_bsr *W)
 {
-    return partials_bytes(M, W->b) + static_cast<size_t>(num_sms()) * kStreamWarps * sizeof(int32_t);
+    return partials_bytes(M, W->b) + static_cast<size_t>(num_sms()) * sizeof(int32_t);
 }
 
 bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, void *ws,

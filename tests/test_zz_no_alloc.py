@@ -75,16 +75,37 @@ def test_noalloc_matches_caller_scratch_entry_point(sg, name, M):
     assert torch.equal(Y2.view(torch.int16), want.view(torch.int16))
 
 
-def test_noalloc_rejects_calls_needing_more_scratch(sg):
-    # b = 64 with 32 tokens needs SMs x 128 KiB of partial-sum scratch, more
-    # than the fixed array on any part with over 128 SMs (a B200 has 148)
+def test_noalloc_takes_the_largest_supported_call(sg):
+    """b = 64 with 32 tokens is the largest scratch need of the small-M
+    forward (SMs x 16 KiB); it fits the fixed array, runs, and matches the
+    caller-scratch entry point bit for bit and the oracle element by element."""
     b, M = 64, 32
-    inp = synth.random_case(M, 1024, 512, b, 40, 52)
+    inp = synth.random_case(M, 1024, 512, b, 40, 52, empty_rows=(5,))
     Wp = sg.pack(to_dev(inp["W"]), mask_dev(inp["mask"]), b)
-    assert torch.cuda.get_device_properties(0).multi_processor_count > 128
-    assert sg.forward_workspace_bytes(M, Wp) > SCRATCH_BYTES
-    Y = torch.zeros((M, 1024), dtype=torch.bfloat16, device="cuda")
-    st = _noalloc(sg, to_dev(inp["X"]), Wp, Y)
-    assert st == 7  # BSL_ERR_SCRATCH_TOO_SMALL, nothing launched
+    assert sg.forward_workspace_bytes(M, Wp) <= SCRATCH_BYTES
+    X = to_dev(inp["X"])
+    want = sg.forward_stream(X, Wp)
+    Y = torch.full((M, 1024), 3.0, dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(sg, X, Wp, Y) == 0
+    torch.cuda.synchronize()
+    assert sg.device_status(Wp) == 0
+    assert torch.equal(Y.view(torch.int16), want.view(torch.int16))
+    ref, S = oracle.forward(inp["X"], inp["W"], inp["mask"], b)
+    assert_parity(to_f64(Y), ref, S, "no-alloc, b = 64, M = 32")
+
+
+def test_noalloc_rejects_bad_arguments_before_any_launch(sg):
+    """Arguments the entry point cannot serve come back as a status, with
+    nothing launched and the output untouched: too many tokens for the
+    small-M kernel, a null output."""
+    b = 32
+    inp = synth.random_case(40, 256, 256, b, 16, 53)
+    Wp = sg.pack(to_dev(inp["W"]), mask_dev(inp["mask"]), b)
+    Y = torch.zeros((40, 256), dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(sg, to_dev(inp["X"]), Wp, Y) == 2   # BSL_ERR_UNSUPPORTED: M > small_m_max
+    lib = sg.library()
+    fn = lib.bsl_forward_stream_noalloc
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert fn(to_dev(inp["X"][:8]).data_ptr(), 8, Wp.cref(), None, stream) == 1   # null Y
     torch.cuda.synchronize()
     assert torch.count_nonzero(Y) == 0
