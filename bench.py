@@ -51,7 +51,7 @@ L2_BYTES_DEFAULT = 126 * 2 ** 20
 TRAFFIC = {
 }
 # the kernel source files each contraction's traffic figure depends on
-TRAFFIC_FILES = {"fwd": ["spmm_pair.cu", "common.cuh"], "fwd_small": ["stream_fwd.cu", "common.cuh"],
+TRAFFIC_FILES = {"fwd": ["spmm_tc.cu", "common.cuh"], "fwd_small": ["stream_fwd.cu", "common.cuh"],
                  "dx": ["spmm_tc.cu", "common.cuh"], "dw": ["sddmm_tc.cu", "common.cuh"]}
 
 
@@ -453,7 +453,7 @@ def run_gpu(args):
     # dominant kernel + its roofline
     dom = max(per_kernel, key=per_kernel.get)
     roof = roofline_entry(dom, alg[dom], per_kernel[dom], pk)
-    roof["kernel"] = {"fwd": "k_stream_fwd" if small else "k_spmm_pair (forward)",
+    roof["kernel"] = {"fwd": "k_stream_fwd" if small else "k_spmm_tc (forward)",
                       "dx": "k_spmm_tc (input gradient)", "dw": "k_sddmm_tc"}[dom]
     roof["peak_source"] = pk["source"] + (" burst bf16" if roof["unit"] == "TFLOP/s" else " HBM copy")
     tr = TRAFFIC.get((w.name, dom))

@@ -87,7 +87,7 @@ typedef struct {
     int32_t *row_order;   /* [R] block rows by block count, largest first, ties lower id first */
     int32_t *col_order;   /* [C] block columns, same order rule */
     int32_t *dw_gptr;     /* [C+1] prefix over columns of ceil(col_count / (128/b)) (weight-gradient groups) */
-    /* Work plan of the tensor-core forward: block rows taken G = 256/b at a
+    /* Work plan of the tensor-core forward: block rows taken G = 128/b at a
      * time in row_order ("row groups", ceil(R/G) of them).  For each group
      * the members' block columns are merged into one ascending list of
      * entries; entry = block column | (member mask << 24), bit i set when the
@@ -98,9 +98,9 @@ typedef struct {
     int32_t *rgrp_ent;    /* [nnz] entries (at most nnz) */
     int32_t *rgrp_blk;    /* [nnz] BSR block of each present member */
     /* The same plan for the input gradient over block columns (col_order, CSC
-     * index), G' = 128/b columns per group; entry = block row | (member mask << 24). */
-    int32_t *cgrp_ptr;    /* [ceil(C/G')+1] */
-    int32_t *cgrp_bptr;   /* [ceil(C/G')+1] */
+     * index), G = 128/b columns per group; entry = block row | (member mask << 24). */
+    int32_t *cgrp_ptr;    /* [ceil(C/G)+1] */
+    int32_t *cgrp_bptr;   /* [ceil(C/G)+1] */
     int32_t *cgrp_ent;    /* [nnz] */
     int32_t *cgrp_blk;    /* [nnz] */
     int32_t *status;      /* [1] device status word; must be zeroed once at allocation */

@@ -127,8 +127,8 @@ class BsrWeight:
         self.row_order = torch.empty(R, **i32)
         self.col_order = torch.empty(C, **i32)
         self.dw_gptr = torch.empty(C + 1, **i32)
-        GR, GC = 256 // b, 128 // b   # row groups (forward), column groups (input gradient)
-        nrg, ncg = (R + GR - 1) // GR, (C + GC - 1) // GC
+        G = 128 // b   # block rows (forward) / block columns (input gradient) per group
+        nrg, ncg = (R + G - 1) // G, (C + G - 1) // G
         self.rgrp_ptr = torch.empty(nrg + 1, **i32)
         self.rgrp_bptr = torch.empty(nrg + 1, **i32)
         self.rgrp_ent = torch.empty(max(nnz, 1), **i32)

@@ -297,7 +297,7 @@ bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, const void
     DeviceGuard guard;
     BSL_TRY(guard.bind(X));
     BSL_TRY(check_device());
-    return launch_spmm_pair(X, M, W, bias, Y, static_cast<cudaStream_t>(stream));
+    return launch_spmm_tc(X, M, W->K, W, false, bias, Y, W->N, static_cast<cudaStream_t>(stream));
 }
 
 bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y,
@@ -330,7 +330,7 @@ bsl_status bsl_backward_input(const void *dY, int32_t M, const bsl_bsr *W, void 
     DeviceGuard guard;
     BSL_TRY(guard.bind(dY));
     BSL_TRY(check_device());
-    return launch_spmm_dx(dY, M, W, dX, static_cast<cudaStream_t>(stream));
+    return launch_spmm_tc(dY, M, W->N, W, true, nullptr, dX, W->K, static_cast<cudaStream_t>(stream));
 }
 
 bsl_status bsl_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, void *stream)

@@ -56,12 +56,11 @@ void note_driver_error(int code);
 bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *out, cudaStream_t s);
 bsl_status launch_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *row_ptr, cudaStream_t s);
 
-// Input gradient dX = dY . W~ on the single-SM tensor-core engine (segments =
-// block columns through the CSC index).
-bsl_status launch_spmm_dx(const void *dY, int32_t M, const bsl_bsr *W, void *dX, cudaStream_t s);
-
-// Forward on pairs of SMs (tcgen05 cta_group::2, M = 256 per instruction).
-bsl_status launch_spmm_pair(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, cudaStream_t s);
+// Forward (A = X, segments = block rows) and input gradient (A = dY,
+// segments = block columns through the CSC index) share one engine.
+// bias: bf16 [out_cols] added to every output row (forward only; may be null).
+bsl_status launch_spmm_tc(const void *A, int32_t M, int32_t a_cols, const bsl_bsr *W, bool transposed,
+                          const void *bias, void *out, int32_t out_cols, cudaStream_t s);
 
 bsl_status launch_sddmm_tc(const void *dY, const void *X, int32_t M, const bsl_bsr *W, void *dW,
                            cudaStream_t s);

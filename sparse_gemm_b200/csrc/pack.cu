@@ -15,7 +15,7 @@
 //   k_fill_cols  one warp per block column: row_idx, csc_to_bsr
 //   k_gather     16-byte vector copy of every kept block into `values`
 //   k_order      rank of each row / column in the longest-first order
-//   k_group_plan one warp per group of 256/b rows (128/b columns) in that order:
+//   k_group_plan one warp per group of G = 128/b rows (columns) in that order:
 //                merges the members' sorted block coordinates into the
 //                entry list of the tensor-core kernels (count pass, scan,
 //                fill pass); the kernels read the values themselves from
@@ -275,21 +275,19 @@ __global__ void __launch_bounds__(1024) k_scan_groups(int32_t *a, int32_t na, in
     scan_counts(d, nd, nullptr, 1, sm);
 }
 
-// Row groups of GR = 256/b block rows (the pair forward engine), column groups
-// of GC = 128/b block columns (the input-gradient engine).
-template <int GR, int GC>
+template <int G>
 void launch_group_plans(const bsl_bsr *o, cudaStream_t s)
 {
     const int32_t R = o->N / o->b, C = o->K / o->b, nnz = o->nnz;
-    const int nrg = (R + GR - 1) / GR, ncg = (C + GC - 1) / GC;
+    const int nrg = (R + G - 1) / G, ncg = (C + G - 1) / G;
     const int rb = (nrg + kWarps - 1) / kWarps, cbk = (ncg + kWarps - 1) / kWarps;
     for (int fill = 0; fill < 2; ++fill) {
-        k_group_plan<GR><<<rb, kWarps * 32, 0, s>>>(o->row_ptr, o->col_idx, nullptr, o->row_order, R, nrg,
-                                                    o->rgrp_ptr, o->rgrp_bptr, o->rgrp_ent, o->rgrp_blk, nnz,
+        k_group_plan<G><<<rb, kWarps * 32, 0, s>>>(o->row_ptr, o->col_idx, nullptr, o->row_order, R, nrg,
+                                                   o->rgrp_ptr, o->rgrp_bptr, o->rgrp_ent, o->rgrp_blk, nnz,
+                                                   fill);
+        k_group_plan<G><<<cbk, kWarps * 32, 0, s>>>(o->col_ptr, o->row_idx, o->csc_to_bsr, o->col_order, C, ncg,
+                                                    o->cgrp_ptr, o->cgrp_bptr, o->cgrp_ent, o->cgrp_blk, nnz,
                                                     fill);
-        k_group_plan<GC><<<cbk, kWarps * 32, 0, s>>>(o->col_ptr, o->row_idx, o->csc_to_bsr, o->col_order, C, ncg,
-                                                     o->cgrp_ptr, o->cgrp_bptr, o->cgrp_ent, o->cgrp_blk, nnz,
-                                                     fill);
         if (!fill)
             k_scan_groups<<<1, 1024, 0, s>>>(o->rgrp_ptr, nrg, o->rgrp_bptr, nrg, o->cgrp_ptr, ncg, o->cgrp_bptr,
                                              ncg);
@@ -335,8 +333,8 @@ bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cud
         cudaMemsetAsync(o->cgrp_ent, 0, sizeof(int32_t) * nnz, s);
         cudaMemsetAsync(o->cgrp_blk, 0, sizeof(int32_t) * nnz, s);
     }
-    if (o->b == 64) launch_group_plans<4, 2>(o, s);
-    else launch_group_plans<8, 4>(o, s);
+    if (o->b == 64) launch_group_plans<2>(o, s);
+    else launch_group_plans<4>(o, s);
     cudaMemsetAsync(o->sched, 0, 8 * sizeof(int32_t), s);
     return cuda_status(cudaGetLastError());
 }

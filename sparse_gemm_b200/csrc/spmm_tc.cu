@@ -1,11 +1,12 @@
-// spmm_tc.cu -- input gradient of the block-sparse layer on one SM's tensor core.
+// spmm_tc.cu -- block-sparse x dense products on the sm_100a tensor cores.
 //
+// One engine computes both contractions of the layer that have a dense
+// activation operand and a sparse weight operand:
+//
+//   forward         Y [M,N]  = X  [M,K] . W~^T   segments = block rows,
+//                   activation tile = X[:, c-block] for block column c
 //   input gradient  dX[M,K]  = dY [M,N] . W~     segments = block columns (CSC),
 //                   activation tile = dY[:, r-block], weight block untransposed
-//
-// (The forward, Y = X . W~^T over block rows, runs on the CTA-pair engine in
-// spmm_pair.cu.  The engine below is written for either orientation -- the
-// TRANS template flag -- and is instantiated for the input gradient only.)
 //
 // (Hugging Face pytorch_block_sparse release note, "Block-Sparse
 // Implementation and Usage": BlockSparseLinear keeps only the nonzero blocks
@@ -112,6 +113,7 @@ struct SpmmArgs {
     const int32_t *grp_ent;    // entries: coordinate | (mask << 24)
     const int32_t *grp_blk;    // BSR block of every present member, entry by entry
     int32_t *sched;            // [1] next unit (zeroed in stream order before every launch)
+    const __nv_bfloat16 *bias; // [nseg * b] added to every output row (forward only; null: none)
     int32_t *status;
     uint64_t timeout_ns;
 };
@@ -520,6 +522,21 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                     const int nz = __shfl_sync(0xffffffffu, mnz, mbr);
                     if (seg < 0) break;
                     uint32_t v[B];
+                    // the bias of the member's b output columns (the same for every row)
+                    float bv[B];
+                    if (args.bias) {
+                        const uint4 *bp = reinterpret_cast<const uint4 *>(args.bias + static_cast<int64_t>(seg) * B);
+#pragma unroll
+                        for (int c = 0; c < B / 8; ++c) {
+                            const uint4 u = __ldg(bp + c);
+                            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                bv[8 * c + 2 * h] = __uint_as_float(w4[h] << 16);
+                                bv[8 * c + 2 * h + 1] = __uint_as_float(w4[h] & 0xFFFF0000u);
+                            }
+                        }
+                    }
                     if (nz) {
                         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                                ar.slot * Cfg::ACC_COLS + s * Cfg::HALF_COLS + mbr * B;
@@ -530,6 +547,10 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                     } else {
 #pragma unroll
                         for (int c = 0; c < B; ++c) v[c] = 0u;
+                    }
+                    if (args.bias) {
+#pragma unroll
+                        for (int c = 0; c < B; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) + bv[c]);
                     }
                     if (lane == 0) bulk_wait_group_read<1>();  // staging chunk `ob` was read out
                     __syncwarp();
@@ -595,16 +616,12 @@ bsl_status run(const CUtensorMap &a, const CUtensorMap &o, const CUtensorMap &w,
 
 }  // namespace
 
-bsl_status launch_spmm_dx(const void *dY, int32_t M, const bsl_bsr *W, void *dX, cudaStream_t s)
+bsl_status launch_spmm_tc(const void *A, int32_t M, int32_t a_cols, const bsl_bsr *W, bool transposed,
+                          const void *bias, void *out, int32_t out_cols, cudaStream_t s)
 {
-    // input gradient: activation operand dY [M, N], output dX [M, K], segments
-    // = block columns through the CSC index (the forward runs on the pair engine)
-    constexpr bool transposed = true;
-    const void *A = dY;
-    void *out = dX;
-    const int32_t a_cols = W->N, out_cols = W->K;
     const int B = W->b;
-    if (W->nnz == 0) return cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(M) * out_cols * 2, s));
+    if (W->nnz == 0 && (transposed || !bias))
+        return cuda_status(cudaMemsetAsync(out, 0, static_cast<size_t>(M) * out_cols * 2, s));
     CUtensorMap ma, mo, mw;
     if (!make_map_2d(&ma, A, a_cols, M, static_cast<uint64_t>(a_cols) * 2, B, 256, 2 * B) ||
         !make_map_2d(&mo, out, out_cols, M, static_cast<uint64_t>(out_cols) * 2, B, 32, 2 * B) ||
@@ -625,9 +642,11 @@ bsl_status launch_spmm_dx(const void *dY, int32_t M, const bsl_bsr *W, void *dX,
     args.grp_ent = transposed ? W->cgrp_ent : W->rgrp_ent;
     args.grp_blk = transposed ? W->cgrp_blk : W->rgrp_blk;
     args.sched = W->sched + (transposed ? 2 : 0);
+    args.bias = transposed ? nullptr : static_cast<const __nv_bfloat16 *>(bias);
     args.status = W->status;
     args.timeout_ns = wait_timeout_ns();
-    return B == 64 ? run<64, true>(ma, mo, mw, args, s) : run<32, true>(ma, mo, mw, args, s);
+    if (B == 64) return transposed ? run<64, true>(ma, mo, mw, args, s) : run<64, false>(ma, mo, mw, args, s);
+    return transposed ? run<32, true>(ma, mo, mw, args, s) : run<32, false>(ma, mo, mw, args, s);
 }
 
 }  // namespace bsl

@@ -227,6 +227,13 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     const int cq1 = share_begin((blockIdx.x + 1) * kStreamWarps, GW, a.nnz);
     const int nblk = q1 > q0 ? q1 - q0 : 0;
     const int nfirst = nblk < Cfg::NSLOT ? nblk : Cfg::NSLOT;
+    if (threadIdx.x == 0) {
+        tma_prefetch_map(&tmW);
+        tma_prefetch_map(&tmX);
+    }
+    // block columns of the share's first 32 blocks, one per lane: the load is
+    // in flight while the weight copies are issued
+    int cidx = q0 + lane < q1 ? a.col_idx[q0 + lane] : 0;
 
     // the weight blocks depend on nothing: their copies go out first, each
     // slot armed for its block and activation slice together
@@ -250,7 +257,6 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     if (nblk > 0) {
         // block columns of 32 consecutive blocks of the share, one per lane
         int cbase = q0;
-        int cidx = q0 + lane < q1 ? a.col_idx[q0 + lane] : 0;
         auto col_of = [&](int p) {  // warp-uniform p; refreshes the lane cache when p leaves it
             if (p >= cbase + 32) {
                 cbase = p;

@@ -147,7 +147,7 @@ def test_repack_in_place_with_a_new_mask():
         assert np.array_equal(getattr(Wp, key)[:nnz].cpu().numpy(), want[key]), key
     assert np.array_equal(bits(Wp.block_values()), want["values"].reshape(nnz, b, b))
     gp, gb, ent, blk = _plan.group_plan(want["row_ptr"], want["col_idx"], oracle.schedule_order(want["row_ptr"]),
-                                        256 // b)
+                                        128 // b)
     assert np.array_equal(Wp.rgrp_ptr.cpu().numpy(), gp)
     assert np.array_equal(Wp.rgrp_ent[:len(ent)].cpu().numpy(), ent)
     ref, S = oracle.forward(second["X"], second["W"], second["mask"], b)
