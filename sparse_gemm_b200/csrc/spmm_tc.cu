@@ -30,10 +30,12 @@
 // let the epilogue of one unit overlap the MMAs of the next.
 //
 // Entry slots.  Each entry in flight owns one shared-memory slot: its
-// activation tile and room for G weight blocks.  The weight blocks of an
-// entry sit contiguously in the pack's plan-ordered copy of the values,
-// stored in the swizzled shared-memory image, so they arrive with one 1-D
-// bulk copy.  The producer also writes the entry's MMA runs (TMEM column,
+// activation tile and room for G weight blocks.  Each present member's
+// block comes straight from the packed values (the weight is stored once,
+// in BSR order) by a 3-D tensor copy that swizzles it on the way into the
+// slot; the group plan lists the BSR block ids of every entry, which the
+// producer warp stages in shared memory a chunk of entries at a time.  The
+// producer also writes the entry's MMA runs (TMEM column,
 // block, instruction descriptor, overwrite flag) into a small slot header:
 // the MMA pipe barely runs ahead of the thread that issues it, so that
 // thread does nothing per entry but wait, read the header and issue.  One
@@ -53,8 +55,8 @@
 // time (they would share the counter).
 //
 // Roles per CTA (persistent grid, one CTA per SM):
-//   warps 0..P-1   producers: TMA tile copy of the activation tile, bulk
-//                  copy of the entry's weight blocks, into the entry's slot
+//   warps 0..P-1   producers: TMA tile copies of the activation tile and of
+//                  the entry's weight blocks, into the entry's slot
 //   warp P         TMEM owner; runs converged, lane 0 issues the MMAs and commits
 //                  (bf16 in, fp32 accumulators in TMEM)
 //   warps P+1..P+4 epilogue: TMEM -> registers -> bf16 (RNE) -> swizzled smem
