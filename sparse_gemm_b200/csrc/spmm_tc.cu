@@ -83,9 +83,12 @@ struct SpmmCfg {
     static constexpr int S = B == 64 ? 4 : 8;           // entry slots (= entries in flight)
     static constexpr int S_LOG = B == 64 ? 2 : 3;
     static constexpr int P = 4;                         // producer warps
-    static constexpr int UR = 16;                       // unit-id ring
+    static constexpr int UR = 16;                       // unit ring (id, entry count)
     static constexpr int W_MMA = P;                     // then 4 epilogue warps
-    static constexpr int THREADS = (P + 5) * 32;
+    static constexpr int W_SCHED = P + 5;               // then the scheduler
+    static constexpr int THREADS = (P + 6) * 32;
+    static constexpr int D = 2;                         // staged chunks of entries
+    static constexpr int CH_BYTES = 16 + 32 * 8 + 32 * G * 4;  // header, entries, aux, block ids
     static constexpr int WARP_OUT = 32 * ROW_BYTES;     // one epilogue warp's staging chunk (32 rows)
     static constexpr int OUT_BYTES = 4 * 2 * WARP_OUT;  // 4 warps x 2 chunks
     static constexpr int ACC = 2;                       // TMEM accumulators
@@ -94,15 +97,15 @@ struct SpmmCfg {
     static constexpr int TMEM_COLS = ACC * ACC_COLS;    // 512
     static constexpr uint32_t LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
     static constexpr uint32_t SBO = 8 * ROW_BYTES;      // stride of 8-row core-matrix groups
-    static constexpr int NUM_BARS = 2 * S + 2 * ACC + 2 * UR + 1;
+    static constexpr int NUM_BARS = 2 * S + 2 * ACC + 2 * UR + 2 * D + 1;
     static constexpr int HDR_V4 = (G + 1) / 2;          // 16-byte header words per slot (two runs each)
     static constexpr int HDR_BYTES = S * HDR_V4 * 16;
-    static constexpr int BLK_IDS = 32 * G;              // block ids of one 32-entry chunk, per producer warp
     static constexpr int SMEM_BYTES =
-        S * SLOT_BYTES + OUT_BYTES + NUM_BARS * 8 + HDR_BYTES + UR * 4 + P * BLK_IDS * 4 + 64 + 1024;
+        S * SLOT_BYTES + OUT_BYTES + NUM_BARS * 8 + HDR_BYTES + UR * 8 + D * CH_BYTES + 64 + 1024;
     static_assert((1 << S_LOG) == S && S % P == 0 && (P & (P - 1)) == 0, "slot ownership");
     static_assert(ACC_COLS == 256 && TMEM_COLS == 512, "TMEM layout");
     static_assert(G <= 8, "member mask is 8 bits");
+    static_assert((D & (D - 1)) == 0 && CH_BYTES % 16 == 0, "chunk ring");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -162,15 +165,17 @@ struct Ring {
     }
 };
 
-// Consumer side of the unit-id ring: the j-th unit id of this CTA (-1: no
-// more units).  Returns false if the wait ran out or the kernel aborted.
+// Consumer side of the unit ring: the j-th unit id of this CTA (-1: no more
+// units) and its entry count.  Returns false if the wait ran out or the
+// kernel aborted.
 template <int UR>
 __device__ __forceinline__ bool unit_take(uint64_t *ufull, uint64_t *uempty, const volatile int *uring, int j,
-                                          int *uid, uint64_t tmo, const volatile int *abort_flag)
+                                          int *uid, int *nent, uint64_t tmo, const volatile int *abort_flag)
 {
     const int s = j % UR;
     if (!mbar_wait(&ufull[s], (j / UR) & 1, tmo, abort_flag)) return false;
-    *uid = uring[s];
+    *uid = uring[2 * s];
+    *nent = uring[2 * s + 1];
     mbar_arrive(&uempty[s]);
     return true;
 }
@@ -190,18 +195,27 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
     uint64_t *empty = full + Cfg::S;       // the entry's MMAs finished: the slot is free
     uint64_t *tfull = empty + Cfg::S;      // accumulator complete
     uint64_t *tempty = tfull + Cfg::ACC;   // accumulator read out
-    uint64_t *ufull = tempty + Cfg::ACC;   // unit id published
-    uint64_t *uempty = ufull + Cfg::UR;    // unit id read by every role
-    uint64_t *drain = uempty + Cfg::UR;
+    uint64_t *ufull = tempty + Cfg::ACC;   // unit published
+    uint64_t *uempty = ufull + Cfg::UR;    // unit read by the MMA issuer and the epilogue
+    uint64_t *cfull = uempty + Cfg::UR;    // chunk of entries staged
+    uint64_t *cempty = cfull + Cfg::D;     // chunk read by every producer
+    uint64_t *drain = cempty + Cfg::D;
     // [S][HDR_V4] MMA runs of the slot's entry, two per 16-byte word: run r is
     // (x, y) = (.x, .y) or (.z, .w) of word r / 2 with x = TMEM column | weight
     // block offset (16-byte units) << 8 | run count (run 0 only) << 24 |
     // overwrite-free flag << 28 and y = the instruction descriptor
     uint4 *hdr = reinterpret_cast<uint4 *>((reinterpret_cast<uintptr_t>(drain + 1) + 15) & ~uintptr_t(15));
+    // [UR][2] unit id (-1: none left) and its entry count
     volatile int *uring = reinterpret_cast<volatile int *>(hdr + Cfg::S * Cfg::HDR_V4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(const_cast<int *>(uring + Cfg::UR));
+    // [D] staged chunks of up to 32 entries of a unit, CH_BYTES each (ints):
+    // [0] entry count (-1: no more units), [1] first output row of the unit,
+    // [4 + i] entry i (coordinate | member mask << 24), [36 + i] members
+    // written by earlier entries of the unit | (offset of the entry's first
+    // block in the chunk's block list << 8), [68 ..] BSR ids of the present
+    // members' blocks, entry by entry
+    int *chunks = const_cast<int *>(uring + 2 * Cfg::UR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(chunks + Cfg::D * (Cfg::CH_BYTES / 4));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int32_t *blk_ids = reinterpret_cast<int32_t *>(tmem_slot + 4);  // [P][BLK_IDS]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
@@ -217,7 +231,11 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         }
         for (int u = 0; u < Cfg::UR; ++u) {
             mbar_init(&ufull[u], 1);
-            mbar_init(&uempty[u], Cfg::P + 5);  // producers, MMA issuer, 4 epilogue warps
+            mbar_init(&uempty[u], 5);  // MMA issuer, 4 epilogue warps
+        }
+        for (int c = 0; c < Cfg::D; ++c) {
+            mbar_init(&cfull[c], 1);
+            mbar_init(&cempty[c], Cfg::P);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -237,140 +255,98 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
 
     if (warp < Cfg::P) {
         // ------------------------------------------------------------ producers
-        // Every producer warp walks all entries of every unit (block offsets
-        // and first-write status are prefix sums over the unit) and issues the
-        // copies of the entries whose slot it owns.  Before the copies it
-        // writes the entry's MMA runs into the slot header, so the issuer only
-        // reads them; the expect_tx arrive publishes the header with the data.
-        // Slot reuse waits for the one MMA commit of the slot's previous
-        // entry, which this warp also issued, so the parity is unambiguous.
+        // The producers walk the entries of the chunks the scheduler staged,
+        // in order, and each issues the copies of the entries whose slot it
+        // owns.  Before the copies it writes the entry's MMA runs into the
+        // slot header, so the issuer only reads them; the expect_tx arrive
+        // publishes the header with the data.  Slot reuse waits for the one
+        // MMA commit of the slot's previous entry, which this warp also
+        // issued, so the parity is unambiguous.
         const int p = warp;
         int e = 0;                  // entries walked so far (all units of this CTA)
         int fills[Cfg::S / Cfg::P]; // fills issued per owned slot
 #pragma unroll
         for (int i = 0; i < Cfg::S / Cfg::P; ++i) fills[i] = 0;
         bool ok = true;
-        for (int j = 0; ok; ++j) {
-            int uid = -1, good = 1;
-            if (lane == 0) {
-                if (p == 0) {
-                    // take the next unit only now that this warp starts it, so a CTA
-                    // never holds more than the units it is working on
-                    const int s = j % Cfg::UR;
-                    if (j >= Cfg::UR && !mbar_wait(&uempty[s], ((j / Cfg::UR) - 1) & 1, tmo, abort_flag)) {
-                        good = 0;
-                    } else {
-                        int ord = atomicAdd(args.sched, 1);
-                        if (ord >= args.units) ord = -1;
-                        uring[s] = ord;
-                        mbar_arrive(&ufull[s]);
-                    }
-                }
-                if (good) good = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag);
-            }
-            good = __shfl_sync(0xffffffffu, good, 0);
-            uid = __shfl_sync(0xffffffffu, uid, 0);
-            if (!good) {
+        for (int cc = 0; ok; ++cc) {
+            const int cs = cc & (Cfg::D - 1);
+            if (__any_sync(0xffffffffu, !mbar_wait(&cfull[cs], (cc / Cfg::D) & 1, tmo, abort_flag))) {
                 ok = false;
                 break;
             }
-            if (uid < 0) break;
-            int mt, g;
-            decode_unit(args, uid, &mt, &g);
-            const int m0 = mt * Cfg::MT;
-            const int z = args.grp_ptr[g], zend = args.grp_ptr[g + 1];
-            int bcur = args.grp_bptr[g];
-            uint32_t seen_carry = 0;  // members present in earlier chunks of this unit
-            for (int eb = z; eb < zend && ok; eb += 32) {
-                const int n = min(32, zend - eb);
-                const int el = lane < n ? args.grp_ent[eb + lane] : 0;
-                const uint32_t ml = static_cast<uint32_t>(el) >> 24;
-                const int kl = __popc(ml);
-                int incl = kl;       // inclusive prefix of block counts over the chunk
-                uint32_t orl = ml;   // inclusive prefix OR of member masks
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                    const uint32_t w = __shfl_up_sync(0xffffffffu, orl, o);
-                    if (lane >= o) {
-                        incl += v;
-                        orl |= w;
-                    }
-                }
-                const int excl = incl - kl;
-                uint32_t seen_ex = __shfl_up_sync(0xffffffffu, orl, 1);
-                seen_ex = (lane == 0 ? 0u : seen_ex) | seen_carry;
-                const int total = __shfl_sync(0xffffffffu, incl, 31);
-                const uint32_t all_or = __shfl_sync(0xffffffffu, orl, 31);
-                // the BSR blocks of the chunk's entries (total <= 32 * G), for the copies
-                int32_t *ids = blk_ids + p * Cfg::BLK_IDS;
-                __syncwarp();  // lane 0 has finished reading the previous chunk's ids
-                for (int i = lane; i < total; i += 32) ids[i] = args.grp_blk[bcur + i];
-                __syncwarp();
-                for (int t = (p - e) & (Cfg::P - 1); t < n; t += Cfg::P) {
-                    const uint32_t ent = static_cast<uint32_t>(__shfl_sync(0xffffffffu, el, t));
-                    const int off = __shfl_sync(0xffffffffu, excl, t);
-                    const uint32_t sb = __shfl_sync(0xffffffffu, seen_ex, t);
-                    // the entry that reuses this slot next: pull its activation tile into L2
-                    const int tn = t + Cfg::S;
-                    const uint32_t entn = static_cast<uint32_t>(__shfl_sync(0xffffffffu, el, tn < n ? tn : 0));
-                    if (lane == 0) {
-                        const int ee = e + t;
-                        const int slot = ee & (Cfg::S - 1);
-                        const int use = ee >> Cfg::S_LOG;
-                        const uint32_t mask = ent >> 24;
-                        const uint32_t k = __popc(mask);
-                        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, tmo, abort_flag)) good = 0;
-                        if (good) {
-                            // runs: consecutive present members with the same first-write
-                            // status; their blocks are consecutive in the slot
-                            uint2 *hr = reinterpret_cast<uint2 *>(hdr + slot * Cfg::HDR_V4);
-                            int nr = 0, mbr = 0;
-                            uint32_t q = 0;
-                            while (mbr < Cfg::G) {
-                                if (!((mask >> mbr) & 1u)) {
-                                    ++mbr;
-                                    continue;
-                                }
-                                const int first = mbr;
-                                const uint32_t q0 = q;
-                                const uint32_t st = (sb >> mbr) & 1u;
-                                int len = 1;
+            const int *ch = chunks + cs * (Cfg::CH_BYTES / 4);
+            const int n = ch[0];
+            if (n < 0) break;  // no more units
+            const int m0 = ch[1];
+            const uint32_t el = lane < n ? static_cast<uint32_t>(ch[4 + lane]) : 0u;
+            const uint32_t ax = lane < n ? static_cast<uint32_t>(ch[36 + lane]) : 0u;
+            const int *ids = ch + 68;
+            int good = 1;
+            for (int t = (p - e) & (Cfg::P - 1); t < n; t += Cfg::P) {
+                const uint32_t ent = __shfl_sync(0xffffffffu, el, t);
+                const uint32_t aux = __shfl_sync(0xffffffffu, ax, t);
+                const int off = static_cast<int>(aux >> 8);
+                const uint32_t sb = aux & 0xFFu;
+                // the entry that reuses this slot next: pull its activation tile into L2
+                const int tn = t + Cfg::S;
+                const uint32_t entn = __shfl_sync(0xffffffffu, el, tn < n ? tn : 0);
+                if (lane == 0) {
+                    const int ee = e + t;
+                    const int slot = ee & (Cfg::S - 1);
+                    const int use = ee >> Cfg::S_LOG;
+                    const uint32_t mask = ent >> 24;
+                    const uint32_t k = __popc(mask);
+                    if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, tmo, abort_flag)) good = 0;
+                    if (good) {
+                        // runs: consecutive present members with the same first-write
+                        // status; their blocks are consecutive in the slot
+                        uint2 *hr = reinterpret_cast<uint2 *>(hdr + slot * Cfg::HDR_V4);
+                        int nr = 0, mbr = 0;
+                        uint32_t q = 0;
+                        while (mbr < Cfg::G) {
+                            if (!((mask >> mbr) & 1u)) {
+                                ++mbr;
+                                continue;
+                            }
+                            const int first = mbr;
+                            const uint32_t q0 = q;
+                            const uint32_t st = (sb >> mbr) & 1u;
+                            int len = 1;
+                            ++mbr;
+                            ++q;
+                            while (mbr < Cfg::G && ((mask >> mbr) & 1u) && ((sb >> mbr) & 1u) == st) {
+                                ++len;
                                 ++mbr;
                                 ++q;
-                                while (mbr < Cfg::G && ((mask >> mbr) & 1u) && ((sb >> mbr) & 1u) == st) {
-                                    ++len;
-                                    ++mbr;
-                                    ++q;
-                                }
-                                hr[nr++] = make_uint2(static_cast<uint32_t>(first * B) |
-                                                          ((q0 * (Cfg::W_BYTES >> 4)) << 8) | (st << 28),
-                                                      make_idesc_bf16(128, len * B, false, TRANS));
                             }
-                            hr[0].x |= static_cast<uint32_t>(nr) << 24;
-                            uint8_t *sp = slots + slot * Cfg::SLOT_BYTES;
-                            mbar_arrive_expect_tx(&full[slot], Cfg::X_BYTES + k * Cfg::W_BYTES);
-                            tma_load_2d(sp, &tmA, &full[slot], static_cast<int>(ent & 0xFFFFFFu) * B, m0);
-                            // the present members' blocks, one swizzled tile each, straight
-                            // from the packed values (stored once, in BSR order)
-                            for (uint32_t qq = 0; qq < k; ++qq)
-                                tma_load_3d(sp + Cfg::X_BYTES + qq * Cfg::W_BYTES, &tmW, &full[slot], 0, 0,
-                                            ids[off + qq]);
-                            if (tn < n) tma_prefetch_2d(&tmA, static_cast<int>(entn & 0xFFFFFFu) * B, m0);
-#pragma unroll
-                            for (int i = 0; i < Cfg::S / Cfg::P; ++i)
-                                if (slot == p + i * Cfg::P) fills[i] = use + 1;
+                            hr[nr++] = make_uint2(static_cast<uint32_t>(first * B) |
+                                                      ((q0 * (Cfg::W_BYTES >> 4)) << 8) | (st << 28),
+                                                  make_idesc_bf16(128, len * B, false, TRANS));
                         }
-                    }
-                    if (!__shfl_sync(0xffffffffu, good, 0)) {
-                        ok = false;
-                        break;
+                        hr[0].x |= static_cast<uint32_t>(nr) << 24;
+                        uint8_t *sp = slots + slot * Cfg::SLOT_BYTES;
+                        mbar_arrive_expect_tx(&full[slot], Cfg::X_BYTES + k * Cfg::W_BYTES);
+                        tma_load_2d(sp, &tmA, &full[slot], static_cast<int>(ent & 0xFFFFFFu) * B, m0);
+                        // the present members' blocks, one swizzled tile each, straight
+                        // from the packed values (stored once, in BSR order)
+                        for (uint32_t qq = 0; qq < k; ++qq)
+                            tma_load_3d(sp + Cfg::X_BYTES + qq * Cfg::W_BYTES, &tmW, &full[slot], 0, 0,
+                                        ids[off + qq]);
+                        if (tn < n) tma_prefetch_2d(&tmA, static_cast<int>(entn & 0xFFFFFFu) * B, m0);
+#pragma unroll
+                        for (int i = 0; i < Cfg::S / Cfg::P; ++i)
+                            if (slot == p + i * Cfg::P) fills[i] = use + 1;
                     }
                 }
-                bcur += total;
-                seen_carry |= all_or;
-                e += n;
+                if (!__shfl_sync(0xffffffffu, good, 0)) {
+                    ok = false;
+                    break;
+                }
             }
+            // every lane is done with the chunk (lane 0 read its block ids)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&cempty[cs]);
+            e += n;
         }
         if (lane == 0) {
             if (!ok) {
@@ -407,10 +383,11 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         constexpr uint32_t KSTEP_W = TRANS ? (16 * Cfg::ROW_BYTES) >> 4 : 2;
         constexpr uint32_t SUB_LO = Cfg::SUB_BYTES >> 4;
         for (int j = 0;; ++j) {
-            int uid = -1, good = 1;
-            if (lane == 0) good = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag);
+            int uid = -1, nent = 0, good = 1;
+            if (lane == 0) good = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, &nent, tmo, abort_flag);
             good = __shfl_sync(0xffffffffu, good, 0);
             uid = __shfl_sync(0xffffffffu, uid, 0);
+            nent = __shfl_sync(0xffffffffu, nent, 0);
             if (!good) {
                 ok = false;
                 break;
@@ -419,14 +396,13 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
             int mt, g;
             decode_unit(args, uid, &mt, &g);
             const bool two = args.M - mt * Cfg::MT > Cfg::BM;  // second 128-row half in range
-            const int z = args.grp_ptr[g], zend = args.grp_ptr[g + 1];
             if (__any_sync(0xffffffffu, !mbar_wait(&tempty[ar.slot], ar.phase ^ 1, tmo, abort_flag))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t d0 = tmem_base + ar.slot * Cfg::ACC_COLS;
-            for (int t = z; t < zend; ++t, ++e) {
+            for (int t = 0; t < nent; ++t, ++e) {
                 const int slot = e & (Cfg::S - 1);
                 // the copies are ordered before the MMAs by the barrier itself (both
                 // are async-proxy accesses), so no tcgen05 fence is needed here
@@ -467,7 +443,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                 any = true;
             }
             if (!ok) break;
-            if (zend > z) umma_commit_lead(lead, &tfull[ar.slot]);
+            if (nent > 0) umma_commit_lead(lead, &tfull[ar.slot]);
             else if (lane == 0) mbar_arrive(&tfull[ar.slot]);
             __syncwarp();
             ar.next(Cfg::ACC);
@@ -481,6 +457,116 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
             if (lane == 0 && !mbar_wait(drain, 0, tmo, nullptr)) set_status(args.status, BSL_ERR_TIMEOUT);
         }
         __syncwarp();
+    } else if (warp == Cfg::W_SCHED) {
+        // ------------------------------------------------------------ scheduler
+        // Takes the units of this CTA from the per-weight counter and stages
+        // each unit's entries, 32 at a time, for the producers: coordinate and
+        // member mask, the members written by earlier entries of the unit
+        // (their MMAs accumulate, the others overwrite), the offset of the
+        // entry's blocks in the chunk and the BSR ids of those blocks.  The
+        // dependent global loads of the plan thus run ahead of the copies.  A
+        // new unit is taken only once a chunk slot is free, so the CTA holds at
+        // most one unit beyond the one its producers are issuing.
+        bool ok = true;
+        int cc = 0;  // chunks staged
+        for (int j = 0; ok; ++j) {
+            int good = 1;
+            if (lane == 0 && cc >= Cfg::D)
+                good = mbar_wait(&cempty[cc & (Cfg::D - 1)], ((cc / Cfg::D) - 1) & 1, tmo, abort_flag);
+            if (!__shfl_sync(0xffffffffu, good, 0)) {
+                ok = false;
+                break;
+            }
+            int ord = -1;
+            if (lane == 0) {
+                ord = atomicAdd(args.sched, 1);
+                if (ord >= args.units) ord = -1;
+            }
+            ord = __shfl_sync(0xffffffffu, ord, 0);
+            int mt = 0, g = 0, z = 0, zend = 0, bcur = 0;
+            if (ord >= 0) {
+                decode_unit(args, ord, &mt, &g);
+                z = args.grp_ptr[g];
+                zend = args.grp_ptr[g + 1];
+                bcur = args.grp_bptr[g];
+            }
+            if (lane == 0) {
+                const int s = j % Cfg::UR;
+                if (j >= Cfg::UR && !mbar_wait(&uempty[s], ((j / Cfg::UR) - 1) & 1, tmo, abort_flag)) {
+                    good = 0;
+                } else {
+                    uring[2 * s] = ord;
+                    uring[2 * s + 1] = zend - z;
+                    mbar_arrive(&ufull[s]);
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, good, 0)) {
+                ok = false;
+                break;
+            }
+            if (ord < 0) break;
+            const int m0 = mt * Cfg::MT;
+            uint32_t seen_carry = 0;  // members present in earlier chunks of this unit
+            for (int eb = z; eb < zend; eb += 32) {
+                const int n = min(32, zend - eb);
+                const uint32_t el = lane < n ? static_cast<uint32_t>(args.grp_ent[eb + lane]) : 0u;
+                const uint32_t ml = el >> 24;
+                const int kl = __popc(ml);
+                int incl = kl;      // inclusive prefix of block counts over the chunk
+                uint32_t orl = ml;  // inclusive prefix OR of member masks
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    const uint32_t w = __shfl_up_sync(0xffffffffu, orl, o);
+                    if (lane >= o) {
+                        incl += v;
+                        orl |= w;
+                    }
+                }
+                uint32_t seen_ex = __shfl_up_sync(0xffffffffu, orl, 1);
+                seen_ex = (lane == 0 ? 0u : seen_ex) | seen_carry;
+                const int total = __shfl_sync(0xffffffffu, incl, 31);
+                const uint32_t all_or = __shfl_sync(0xffffffffu, orl, 31);
+                const int cs = cc & (Cfg::D - 1);
+                if (lane == 0 && cc >= Cfg::D && eb > z)
+                    good = mbar_wait(&cempty[cs], ((cc / Cfg::D) - 1) & 1, tmo, abort_flag);
+                if (!__shfl_sync(0xffffffffu, good, 0)) {
+                    ok = false;
+                    break;
+                }
+                int *ch = chunks + cs * (Cfg::CH_BYTES / 4);
+                if (lane == 0) {
+                    ch[0] = n;
+                    ch[1] = m0;
+                }
+                ch[4 + lane] = static_cast<int>(el);
+                ch[36 + lane] = static_cast<int>(seen_ex | static_cast<uint32_t>(incl - kl) << 8);
+                for (int i = lane; i < total; i += 32) ch[68 + i] = args.grp_blk[bcur + i];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cfull[cs]);
+                bcur += total;
+                seen_carry |= all_or;
+                ++cc;
+            }
+        }
+        if (ok) {  // tell the producers that no unit is left
+            int good = 1;
+            const int cs = cc & (Cfg::D - 1);
+            if (lane == 0) {
+                if (cc >= Cfg::D && !mbar_wait(&cempty[cs], ((cc / Cfg::D) - 1) & 1, tmo, abort_flag)) {
+                    good = 0;
+                } else {
+                    chunks[cs * (Cfg::CH_BYTES / 4)] = -1;
+                    mbar_arrive(&cfull[cs]);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, good, 0) != 0;
+        }
+        if (lane == 0 && !ok) {
+            *abort_flag = 1;
+            set_status(args.status, BSL_ERR_TIMEOUT);
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
         // Each warp drains its own 32 TMEM lanes (tile rows) of every chunk
@@ -492,9 +578,9 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         uint32_t ob = 0;
         bool ok = true;
         for (int j = 0;; ++j) {
-            int uid = -1, go = 1;
+            int uid = -1, nent = 0, go = 1;
             if (lane == 0) {
-                go = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, tmo, abort_flag);
+                go = unit_take<Cfg::UR>(ufull, uempty, uring, j, &uid, &nent, tmo, abort_flag);
                 if (go && uid >= 0) go = mbar_wait(&tfull[ar.slot], ar.phase, tmo, abort_flag);
             }
             go = __shfl_sync(0xffffffffu, go, 0);
