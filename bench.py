@@ -337,7 +337,7 @@ def run_gpu(args):
     Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
     dX = torch.empty((w.M, w.K), dtype=torch.bfloat16, device=dev) if train else None
     dWv = torch.empty((w.nnz, w.b, w.b), dtype=torch.bfloat16, device=dev) if train else None
-    ws = torch.empty(max(16, sg.forward_workspace_bytes(w.M, Wp)), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(16, sg.forward_workspace_bytes(w.M, Wp)), dtype=torch.uint8, device=dev)
     small = w.M <= sg.small_m_max()
 
     kinds = ["fwd", "dx", "dw"] if train else ["fwd"]

@@ -74,6 +74,10 @@ typedef enum {
  * the scratch of bsl_forward_stream_noalloc. */
 #define BSL_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
+/* Length (int32 entries) of bsl_bsr.sbounds: room for the CTA ranges of a
+ * weight-streaming grid of up to 1024 CTAs (one CTA per SM). */
+#define BSL_SBOUNDS_LEN 1026
+
 /* Packed block-sparse weight.  The caller allocates every array (device
  * memory) with the sizes below, R = N/b, C = K/b; bsl_pack fills them. */
 typedef struct {
@@ -108,6 +112,13 @@ typedef struct {
                            * the call's stream before each launch (contents on entry do not
                            * matter).  Two calls of the same contraction on one weight must not
                            * run at the same time: they would share a counter. */
+    int32_t *sbounds;     /* [BSL_SBOUNDS_LEN] block ranges of the weight-streaming forward's CTAs:
+                           * [0] = U, the CTA count of the device bsl_pack ran on (its SM
+                           * count), [1 + c] = first block of CTA c, c = 0..U ([1 + U] = nnz).
+                           * Bound c is the start of the block row holding block
+                           * floor(c * nnz / U) or of the next one, whichever is nearer, when
+                           * that is at most nnz / (4U) blocks away, else floor(c * nnz / U)
+                           * itself: short block rows are never split between CTAs. */
 } bsl_bsr;
 
 /* Human-readable name of a status code (static string). */
@@ -157,10 +168,14 @@ BSL_API bsl_status bsl_forward_tc(const void *X, int32_t M, const bsl_bsr *W, co
 
 /* Weight-streaming forward ("load and sparse expand", lecture summary at
  * 48:12) for 1 <= M <= bsl_small_m_max(): each warp streams a contiguous,
- * equal share of the packed blocks once; block rows split between warps
- * are summed in a fixed order.  workspace: bsl_forward_workspace_bytes(M, W)
- * bytes; contents on entry do not matter.  bias: bf16 [N] or NULL, as for
- * bsl_forward. */
+ * equal share of its CTA's range of packed blocks once (the ranges in
+ * W->sbounds); block rows split between warps or CTAs are summed in a fixed
+ * order.  workspace: bsl_forward_workspace_bytes(M, W) bytes, zeroed once
+ * when it is allocated; every call leaves its counters (at the start of the
+ * workspace, the same place for every M) at zero again, a call that ran out
+ * of time included, so one workspace serves later calls of any M and weight
+ * without being cleared.  Calls that use one workspace must not overlap on
+ * the GPU.  bias: bf16 [N] or NULL, as for bsl_forward. */
 BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y,
                               void *workspace, size_t workspace_bytes, void *stream);
 
@@ -181,7 +196,7 @@ BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W
  * itself and calls no cudaMalloc / cudaFree.  It returns
  * BSL_ERR_SCRATCH_TOO_SMALL, launching nothing, when the call would need more
  * scratch than that.  The need is bsl_forward_workspace_bytes(M, W) =
- * SMs x (2 x b x M' x 4 + 4) bytes, M' = 16 for M <= 16, else 32: at most
+ * about SMs x (4 + 2 x b x M' x 4) bytes, M' = 16 for M <= 16, else 32: at most
  * 2.4 MB on a 148-SM B200 (b = 64, M <= 32), so every supported call fits
  * there; only a device with more than about 1000 SMs would be turned away.
  *
@@ -189,9 +204,9 @@ BSL_API bsl_status bsl_forward_stream(const void *X, int32_t M, const bsl_bsr *W
  * (cudaGetSymbolAddress) and keeps it for the life of the process, so make
  * that first call outside any stream capture; calls after the device's
  * primary context was destroyed and re-created (cudaDeviceReset) are not
- * supported.  Every call on a device shares the one array, which keeps the
- * previous call's contents; nothing in it has to start at zero (each call
- * writes every partial sum before reading it).  Calls whose kernels overlap
+ * supported.  Every call on a device shares the one array, which starts at
+ * zero when it is loaded; each call writes every partial sum before reading
+ * it and leaves the counters at zero again.  Calls whose kernels overlap
  * on the GPU (different streams without ordering between them) race on the
  * array: serialise them.  X, Y, W: as for bsl_forward_stream; the kernels
  * run on the device that owns X. */

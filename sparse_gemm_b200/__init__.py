@@ -49,7 +49,10 @@ class _BSR(ctypes.Structure):
         (name, ctypes.c_void_p) for name in
         ("row_ptr", "col_idx", "values", "col_ptr", "row_idx", "csc_to_bsr", "row_order",
          "col_order", "dw_gptr", "rgrp_ptr", "rgrp_bptr", "rgrp_ent", "rgrp_blk", "cgrp_ptr",
-         "cgrp_bptr", "cgrp_ent", "cgrp_blk", "status", "sched")]
+         "cgrp_bptr", "cgrp_ent", "cgrp_blk", "status", "sched", "sbounds")]
+
+# int32 entries of bsl_bsr.sbounds (BSL_SBOUNDS_LEN in include/bsl.h)
+SBOUNDS_LEN = 1026
 
 
 _lib = None
@@ -139,13 +142,14 @@ class BsrWeight:
         self.cgrp_blk = torch.empty(max(nnz, 1), **i32)
         self.status = torch.zeros(1, **i32)
         self.sched = torch.zeros(8, **i32)
+        self.sbounds = torch.zeros(SBOUNDS_LEN, **i32)
         self._c = _BSR(self.N, self.K, self.b, self.nnz,
                        *[t.data_ptr() for t in (self.row_ptr, self.col_idx, self.values, self.col_ptr,
                                                 self.row_idx, self.csc_to_bsr, self.row_order,
                                                 self.col_order, self.dw_gptr, self.rgrp_ptr,
                                                 self.rgrp_bptr, self.rgrp_ent, self.rgrp_blk,
                                                 self.cgrp_ptr, self.cgrp_bptr, self.cgrp_ent,
-                                                self.cgrp_blk, self.status, self.sched)])
+                                                self.cgrp_blk, self.status, self.sched, self.sbounds)])
 
     @property
     def R(self):
@@ -248,7 +252,7 @@ def forward(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = None,
     Y = _out(M, Wp.N, X) if out is None else out
     nbytes = forward_workspace_bytes(M, Wp)
     if nbytes and workspace is None:
-        workspace = torch.empty(nbytes, dtype=torch.uint8, device=X.device)
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=X.device)
     wptr = workspace.data_ptr() if workspace is not None else None
     wlen = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(library().bsl_forward(X.data_ptr(), M, Wp.cref(), bptr, Y.data_ptr(), wptr, wlen, _stream(X)),
@@ -277,7 +281,7 @@ def forward_stream(X: torch.Tensor, Wp: BsrWeight, out: torch.Tensor | None = No
     Y = _out(M, Wp.N, X) if out is None else out
     nbytes = forward_workspace_bytes(M, Wp)
     if workspace is None:
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=X.device)
+        workspace = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=X.device)
     _check(library().bsl_forward_stream(X.data_ptr(), M, Wp.cref(), bptr, Y.data_ptr(), workspace.data_ptr(),
                                         workspace.numel() * workspace.element_size(), _stream(X)),
            "bsl_forward_stream")

@@ -20,6 +20,9 @@
 //                entry list of the tensor-core kernels (count pass, scan,
 //                fill pass); the kernels read the values themselves from
 //                `values` (stored once) through this list
+//   k_stream_bounds one thread per CTA of the weight-streaming forward: its
+//                first block, moved to the nearest block-row start when that
+//                is close (short rows are then never split between CTAs)
 #include "common.cuh"
 #include "internal.h"
 
@@ -294,6 +297,39 @@ void launch_group_plans(const bsl_bsr *o, cudaStream_t s)
     }
 }
 
+// Block ranges of the U CTAs of the weight-streaming forward.  CTA c starts
+// at t = floor(c * nnz / U), moved to the start of the block row holding
+// block t or of the next row, whichever is nearer, when that is at most
+// q = floor(nnz / (4U)) blocks away.  Every bound stays within q of its equal
+// share, and equal shares are at least 4q apart, so the bounds never
+// decrease; sb[0] = U tells the kernel which grid size they were made for.
+__global__ void k_stream_bounds(const int32_t *__restrict__ row_ptr, int32_t R, int32_t nnz, int32_t U,
+                                int32_t *__restrict__ sb)
+{
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c == 0) sb[0] = U;
+    if (c > U) return;
+    const int t = static_cast<int>(static_cast<int64_t>(c) * nnz / U);
+    const int q = static_cast<int>(nnz / (4LL * U));
+    int bound = t;
+    if (t > 0 && t < nnz && q > 0) {
+        int lo = 0, hi = R;  // the last row lo with row_ptr[lo] <= t (row_ptr[R] = nnz > t)
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (row_ptr[mid] <= t) lo = mid;
+            else hi = mid;
+        }
+        const int da = t - row_ptr[lo], dz = row_ptr[lo + 1] - t;
+        if (da <= dz) {
+            if (da <= q) bound = t - da;
+        } else if (dz <= q) {
+            bound = t + dz;
+        }
+        bound = min(max(bound, t - q), t + q);  // holds even if row_ptr disagrees with nnz
+    }
+    sb[1 + c] = bound;
+}
+
 }  // namespace
 
 bsl_status launch_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *row_ptr, cudaStream_t s)
@@ -324,6 +360,14 @@ bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cud
         const int grid = static_cast<int>(want < 8L * num_sms() ? want : 8L * num_sms());
         k_gather<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(W), o->K, o->b, R, o->row_ptr, o->col_idx,
                                       static_cast<uint4 *>(o->values), nnz);
+    }
+    {
+        const int U = num_sms();
+        if (U <= BSL_SBOUNDS_LEN - 2) {
+            k_stream_bounds<<<(U + 1 + 255) / 256, 256, 0, s>>>(o->row_ptr, R, nnz, U, o->sbounds);
+        } else {  // no room for this grid: the kernel falls back to equal shares
+            cudaMemsetAsync(o->sbounds, 0, sizeof(int32_t), s);
+        }
     }
     k_order<<<(R + 255) / 256, 256, 256 * sizeof(int32_t), s>>>(o->row_ptr, R, o->row_order);
     k_order<<<(C + 255) / 256, 256, 256 * sizeof(int32_t), s>>>(o->col_ptr, C, o->col_order);

@@ -7,10 +7,13 @@
 // blocks, which are already dense b x b tiles, so "expanding" is placing them
 // in shared memory next to the activation slice they multiply.
 //
-// Decomposition: the BSR block list [0, nnz) is cut into equal contiguous
-// shares, one per warp of a one-CTA-per-SM grid (block counts, not block
-// rows, are balanced; the 8 warps of a CTA hold consecutive shares).  Each
-// warp streams its share through its own ring of slots; a slot holds one
+// Decomposition: the BSR block list [0, nnz) is cut into contiguous ranges,
+// one per CTA of a one-CTA-per-SM grid: equal shares, each moved to a
+// nearby block-row start where there is one (the pack computes these
+// bounds), so short block rows never straddle two CTAs and only rows longer
+// than about a quarter of a CTA's share do.  Each CTA's range is cut into
+// equal shares for its 8 warps (block counts, not block rows, are balanced).
+// Each warp streams its share through its own ring of slots; a slot holds one
 // weight block and the activation slice X[0:MP, c*b:(c+1)*b] it multiplies,
 // both brought in by TMA (swizzled rows, rows past M read as zeros).  The
 // weight copies, which depend on nothing, leave first; a ring usually holds
@@ -24,15 +27,16 @@
 //   - a block row cut by share boundaries leaves an fp32 partial.  After all
 //     warps of the CTA are done, the partials sit in their rings and the
 //     CTA's first contributor to each cut row adds them in warp order.  A row
-//     that lies inside the CTA's share is then written; a row that reaches
-//     into other CTAs' shares leaves the CTA's sum in the workspace, and the
-//     last CTA to count itself in on the row's counter adds the CTAs' sums in
-//     CTA order and writes the row.
+//     that lies inside the CTA's range is then written; a (long) row that
+//     reaches into other CTAs' ranges leaves the CTA's sum in the workspace,
+//     and the last CTA to count itself in on the row's counter adds the CTAs'
+//     sums in CTA order and writes the row.
 // Every sum has a fixed order (the same whoever arrives last), so results
 // are identical run to run.  Block rows without blocks are written (bias or
-// zeros) at the end.  The counters are zeroed on the stream before every
-// launch, so nothing in the workspace has to survive from one call to the
-// next.
+// zeros) at the end.  The last CTA to count itself in on a row's counter
+// sets it back to zero, and a warp that gave up waiting still counts itself
+// in, so every call leaves the counters at zero: the workspace is zeroed once
+// when it is allocated and no memset precedes the kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -63,8 +67,9 @@ struct StreamCfg {
 struct StreamArgs {
     __nv_bfloat16 *Y;
     float *ws;                  // [CTAs][2][b*MP] partial sums of rows cut between CTAs
-    int32_t *cnt;               // [CTAs] arrival counters (zero at launch)
+    int32_t *cnt;               // [CTAs] arrival counters (zero between calls)
     const int32_t *row_ptr, *col_idx;
+    const int32_t *sbounds;     // CTA ranges made by the pack ([0] = their CTA count)
     const __nv_bfloat16 *bias;  // [N] added to every output row (null: none)
     int32_t M, N, K, R, C, nnz;
     int32_t *status;
@@ -77,20 +82,95 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
 }
 
 // first block of share u when nnz blocks are split over U shares
+// floor(x / d) for 0 <= x < 2^63, 0 < d < 2^31, in 32-bit arithmetic when x
+// fits (the usual case: a 64-bit division is a long emulated sequence)
+__device__ __forceinline__ int floor_div(uint64_t x, int d)
+{
+    if (x <= 0xFFFFFFFFull) return static_cast<int>(static_cast<uint32_t>(x) / static_cast<uint32_t>(d));
+    return static_cast<int>(x / static_cast<uint64_t>(d));
+}
+
 __device__ __forceinline__ int share_begin(int u, int U, int nnz)
 {
-    return static_cast<int>((static_cast<int64_t>(u) * nnz) / U);
+    return floor_div(static_cast<uint64_t>(u) * static_cast<uint32_t>(nnz), U);
+}
+
+// Count the caller in and return the new count.  Release: the caller's
+// earlier writes are visible before the new count; acquire: the caller's
+// later reads see what the earlier arrivers released.
+__device__ __forceinline__ int arrive_count(int32_t *p)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+    return old + 1;
 }
 
 // the share that holds block p (the last u with share_begin(u) <= p);
 // share_begin(u) = floor(u * nnz / U), so u is within one of floor(p * U / nnz)
 __device__ __forceinline__ int share_of(int p, int U, int nnz)
 {
-    int u = static_cast<int>((static_cast<int64_t>(p) * U) / nnz);
+    int u = floor_div(static_cast<uint64_t>(p) * static_cast<uint32_t>(U), nnz);
     u = u < 0 ? 0 : (u > U - 1 ? U - 1 : u);
     while (u > 0 && share_begin(u, U, nnz) > p) --u;
     while (u + 1 < U && share_begin(u + 1, U, nnz) <= p) ++u;
     return u;
+}
+
+// The block row holding block p (0 <= p < nnz): the last r with
+// row_ptr[r] <= p, by a warp-parallel search (two or three rounds of one
+// load per lane).
+__device__ __forceinline__ int row_holding(const StreamArgs &a, int p, int lane)
+{
+    int lo = 0, hi = a.R;  // row_ptr[lo] <= p < row_ptr[hi]
+    while (hi - lo > 1) {
+        const int step = (hi - lo + 31) / 32;
+        const int probe = lo + lane * step;
+        const bool le = probe < hi && a.row_ptr[probe] <= p;
+        const int last = 31 - __clz(__ballot_sync(0xffffffffu, le));  // lane 0 always qualifies
+        lo = lo + last * step;
+        hi = min(hi, lo + step);
+    }
+    return lo;
+}
+
+// First block of CTA c (0 <= c <= U): the pack's bounds when they were made
+// for this grid size, else the equal share.
+__device__ __forceinline__ int cta_bound(const StreamArgs &a, bool snapped, int c, int U)
+{
+    return snapped ? __ldg(a.sbounds + 1 + c) : share_begin(c, U, a.nnz);
+}
+
+// First block of warp w (0 <= w <= kStreamWarps) of a CTA whose range starts
+// at cq0 and holds n blocks.
+__device__ __forceinline__ int warp_bound(int w, int cq0, int n)
+{
+    return cq0 + static_cast<int>((static_cast<int64_t>(w) * n) / kStreamWarps);
+}
+
+// The warp of the CTA whose share holds block p (cq0 <= p < cq0 + n).
+__device__ __forceinline__ int warp_of(int p, int cq0, int n)
+{
+    int u = floor_div(static_cast<uint64_t>(p - cq0) * kStreamWarps, n);
+    u = u > kStreamWarps - 1 ? kStreamWarps - 1 : u;
+    while (u > 0 && warp_bound(u, cq0, n) > p) --u;
+    while (u + 1 < kStreamWarps && warp_bound(u + 1, cq0, n) <= p) ++u;
+    return u;
+}
+
+// The CTA whose range holds block p (0 <= p < nnz); warp-collective.  A
+// bound made by the pack lies within nnz / (4U) blocks of its equal share and
+// equal shares are at least 4 times that apart, so the CTA is the equal
+// share's CTA or one of its two neighbours: lanes 0..3 look at the bounds of
+// those three in one round of loads.
+__device__ __forceinline__ int cta_of(const StreamArgs &a, bool snapped, int p, int U, int lane)
+{
+    const int c = share_of(p, U, a.nnz);
+    if (!snapped) return c;
+    const int k = c - 1 + lane;
+    const int v = lane < 4 && k >= 0 && k <= U ? __ldg(a.sbounds + 1 + k) : 0;
+    const int vn = __shfl_down_sync(0xffffffffu, v, 1);
+    const unsigned m = __ballot_sync(0xffffffffu, lane < 3 && k >= 0 && k < U && v <= p && p < vn);
+    return m ? c - 1 + (__ffs(m) - 1) : c;
 }
 
 template <int B>
@@ -220,11 +300,24 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStreamWarps * (Cfg::WARP_BYTES + Cfg::OUT_BYTES)) +
                      warp * Cfg::NSLOT;
 
-    const int GW = gridDim.x * kStreamWarps;
+    const int U = gridDim.x;
+    const int GW = U * kStreamWarps;
     const int gw = blockIdx.x * kStreamWarps + warp;
-    const int q0 = share_begin(gw, GW, a.nnz), q1 = share_begin(gw + 1, GW, a.nnz);
-    const int cq0 = share_begin(blockIdx.x * kStreamWarps, GW, a.nnz);          // this CTA's blocks
-    const int cq1 = share_begin((blockIdx.x + 1) * kStreamWarps, GW, a.nnz);
+    // this CTA's blocks [cq0, cq1): the pack's bounds made for this grid size
+    // (the three loads go out together), else equal shares
+    bool snapped = false;
+    int cq0, cq1;
+    {
+        const bool fits = U <= BSL_SBOUNDS_LEN - 2;
+        const int s0 = fits ? __ldg(a.sbounds) : 0;
+        const int b0 = fits ? __ldg(a.sbounds + 1 + blockIdx.x) : 0;
+        const int b1 = fits ? __ldg(a.sbounds + 2 + blockIdx.x) : 0;
+        snapped = s0 == U;
+        cq0 = snapped ? b0 : share_begin(blockIdx.x, U, a.nnz);
+        cq1 = snapped ? b1 : share_begin(blockIdx.x + 1, U, a.nnz);
+    }
+    const int cn = cq1 - cq0;
+    const int q0 = warp_bound(warp, cq0, cn), q1 = warp_bound(warp + 1, cq0, cn);
     const int nblk = q1 > q0 ? q1 - q0 : 0;
     const int nfirst = nblk < Cfg::NSLOT ? nblk : Cfg::NSLOT;
     if (threadIdx.x == 0) {
@@ -251,6 +344,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     acc.zero();
     part0.zero();
     int first_row = 0, last_row = -1;  // rows of blocks q0 and q1 - 1
+    int fr_beg = 0, fr_end = 0, lr_beg = 0, lr_end = 0;  // their block ranges
     bool cut_first = false, cut_last = false, ok = true;
     int issued = nfirst;
 
@@ -271,23 +365,15 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
             if (lane == 0) tma_load_2d(ring + t * Cfg::SLOT + Cfg::W_BLK, &tmX, &bars[t], c * B, 0);
         }
 
-        // first block row of the share: last r with row_ptr[r] <= q0, by a
-        // warp-parallel search (two or three rounds of one load per lane)
-        int lo = 0, hi = a.R;  // row_ptr[lo] <= q0 < row_ptr[hi]
-        while (hi - lo > 1) {
-            const int step = (hi - lo + 31) / 32;
-            const int probe = lo + lane * step;
-            const bool le = probe < hi && a.row_ptr[probe] <= q0;
-            const int last = 31 - __clz(__ballot_sync(0xffffffffu, le));  // lane 0 always qualifies
-            lo = lo + last * step;
-            hi = min(hi, lo + step);
-        }
-        first_row = lo;
-        int r = lo;
+        first_row = row_holding(a, q0, lane);
+        int r = first_row;
         int rbase = r;
         int rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
         int row_end = __shfl_sync(0xffffffffu, rp, 0);
-        cut_first = a.row_ptr[first_row] < q0;
+        int row_beg = a.row_ptr[first_row];
+        fr_beg = row_beg;
+        fr_end = row_end;
+        cut_first = row_beg < q0;
         bool have = false;
         constexpr int KK = B / 16;
 
@@ -301,6 +387,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                     have = false;
                 }
                 ++r;
+                row_beg = row_end;
                 if (r - rbase >= 32) {  // refresh the lane cache of row ends
                     rbase = r;
                     rp = rbase + 1 + lane <= a.R ? a.row_ptr[rbase + 1 + lane] : 0x7fffffff;
@@ -354,6 +441,8 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
         }
         if (ok) {
             last_row = r;
+            lr_beg = row_beg;
+            lr_end = row_end;
             cut_last = row_end > q1;
             if (last_row == first_row && cut_first) {
                 part0 = acc;  // the share lies inside one row cut at its start: one partial
@@ -372,7 +461,16 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                 mbar_wait(&bars[s], (lastt / Cfg::NSLOT) & 1, a.timeout_ns, nullptr);
             }
         }
-        cut_first = cut_last = false;  // nothing of this warp is combined
+        if (nblk > 0) {
+            // the row of the share's last block from the index alone, so that
+            // this warp still counts itself in on every row it shares with
+            // other CTAs and the counters return to zero (its sums are
+            // incomplete; the status word reports the timeout)
+            last_row = row_holding(a, q1 - 1, lane);
+            lr_beg = a.row_ptr[last_row];
+            lr_end = a.row_ptr[last_row + 1];
+            cut_last = lr_end > q1 && !(last_row == first_row && cut_first);
+        }
     }
     // the ring is read out: it now holds the warp's partials, [0] = first row
     // cut at the share's start, [1] = last row cut at its end
@@ -385,23 +483,22 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     // Cut rows.  The CTA's first contributor to a row (the warp whose share
     // holds the row's first block inside this CTA) adds the CTA's partials of
     // that row in warp order.
-    const int w_lo = blockIdx.x * kStreamWarps;
     for (int which = 0; which < 2; ++which) {
         const bool mine = which == 0 ? cut_first : cut_last;
         if (!mine) continue;
         const int r = which == 0 ? first_row : last_row;
-        const int beg = a.row_ptr[r], end = a.row_ptr[r + 1];
-        const int lead = share_of(beg > cq0 ? beg : cq0, GW, a.nnz);
-        if (lead != gw) continue;
+        const int beg = which == 0 ? fr_beg : lr_beg, end = which == 0 ? fr_end : lr_end;
+        const int lead = warp_of(beg > cq0 ? beg : cq0, cq0, cn);
+        if (lead != warp) continue;
         float sum[PER];
 #pragma unroll
         for (int e = 0; e < PER; ++e) sum[e] = 0.f;
-        const int wl = share_of(end - 1 < cq1 - 1 ? end - 1 : cq1 - 1, GW, a.nnz);
-        for (int w = gw; w <= wl; ++w) {
-            const int sb = share_begin(w, GW, a.nnz);
-            if (share_begin(w + 1, GW, a.nnz) == sb) continue;  // empty share: no partial
+        const int wl = warp_of(end - 1 < cq1 - 1 ? end - 1 : cq1 - 1, cq0, cn);
+        for (int w = warp; w <= wl; ++w) {
+            const int sb = warp_bound(w, cq0, cn);
+            if (warp_bound(w + 1, cq0, cn) == sb) continue;  // empty share: no partial
             // slot 0 holds a row that began before the warp's share, slot 1 the rest
-            const float *src = reinterpret_cast<const float *>(smem + (w - w_lo) * Cfg::WARP_BYTES) +
+            const float *src = reinterpret_cast<const float *>(smem + w * Cfg::WARP_BYTES) +
                                (sb > beg ? 0 : Cfg::PART);
 #pragma unroll
             for (int e = 0; e < PER; ++e) sum[e] += src[e * 32 + lane];
@@ -415,27 +512,43 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
         float *mine_ws = a.ws + (static_cast<int64_t>(blockIdx.x) * 2 + (cq0 >= beg ? 0 : 1)) * Cfg::PART;
 #pragma unroll
         for (int e = 0; e < PER; ++e) __stcg(mine_ws + e * 32 + lane, sum[e]);
-        // CTAs holding the row's first and last block (CTA c owns warps 8c .. 8c+7)
-        const int c0 = share_of(beg, GW, a.nnz) / kStreamWarps;
-        const int c1 = share_of(end - 1, GW, a.nnz) / kStreamWarps;
+        // CTAs holding the row's first and last block, and how many of the
+        // CTAs between them hold any block (31 bounds per round of loads)
+        const int c0 = cta_of(a, snapped, beg, U, lane);
+        const int c1 = cta_of(a, snapped, end - 1, U, lane);
         int contributors = 0;
-        for (int c = c0; c <= c1; ++c)
-            contributors += share_begin((c + 1) * kStreamWarps, GW, a.nnz) > share_begin(c * kStreamWarps, GW, a.nnz);
-        __threadfence();  // every lane's part of the sum is visible before the count says so
+        for (int base = c0; base <= c1; base += 31) {
+            const int c = base + lane;
+            const int bc = cta_bound(a, snapped, c < U ? c : U, U);
+            const int bn = __shfl_down_sync(0xffffffffu, bc, 1);
+            contributors += __popc(__ballot_sync(0xffffffffu, lane < 31 && c <= c1 && bn > bc));
+        }
+        // every lane's stores happen before lane 0's release of the count; the
+        // last arriver's acquire orders its reads of the other sums after it
         __syncwarp();
         int last = 0;
-        if (lane == 0) last = atomicAdd(a.cnt + c0, 1) == contributors - 1;
-        if (!__shfl_sync(0xffffffffu, last, 0)) continue;
-        __threadfence();  // the other CTAs' sums are read after their counts
+        if (lane == 0) last = arrive_count(a.cnt + c0) == contributors;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        __syncwarp();
+        if (!last) continue;
 #pragma unroll
         for (int e = 0; e < PER; ++e) sum[e] = 0.f;
-        for (int c = c0; c <= c1; ++c) {
-            const int cb = share_begin(c * kStreamWarps, GW, a.nnz);
-            if (share_begin((c + 1) * kStreamWarps, GW, a.nnz) == cb) continue;  // empty CTA share
-            const float *src = a.ws + (static_cast<int64_t>(c) * 2 + (cb >= beg ? 0 : 1)) * Cfg::PART;
+        for (int base = c0; base <= c1; base += 31) {
+            const int c = base + lane;
+            const int bc = cta_bound(a, snapped, c < U ? c : U, U);
+            const int bn = __shfl_down_sync(0xffffffffu, bc, 1);
+            const unsigned held = __ballot_sync(0xffffffffu, lane < 31 && c <= c1 && bn > bc);
+            // slot 0 of a CTA holds the row when its range starts inside the row
+            const unsigned first = __ballot_sync(0xffffffffu, bc >= beg);
+            for (unsigned m = held; m; m &= m - 1) {
+                const int j = __ffs(m) - 1;
+                const float *src =
+                    a.ws + (static_cast<int64_t>(base + j) * 2 + ((first >> j) & 1u ? 0 : 1)) * Cfg::PART;
 #pragma unroll
-            for (int e = 0; e < PER; ++e) sum[e] += __ldcg(src + e * 32 + lane);
+                for (int e = 0; e < PER; ++e) sum[e] += __ldcg(src + e * 32 + lane);
+            }
         }
+        if (lane == 0) a.cnt[c0] = 0;  // every contributor is in: ready for the next call
         write_row_flat<B, MP>(sum, a, r, stage, lane);
     }
 
@@ -454,9 +567,6 @@ bsl_status run(const void *X, const void *values, StreamArgs a, cudaStream_t s)
 {
     using Cfg = StreamCfg<B, MP>;
     const int grid = num_sms();
-    // counters start at zero on every launch (stream order)
-    cudaError_t e = cudaMemsetAsync(a.cnt, 0, static_cast<size_t>(grid) * sizeof(int32_t), s);
-    if (e != cudaSuccess) return cuda_status(e);
     CUtensorMap mw, mx;
     if (!make_map_2d(&mw, a.nnz > 0 ? values : X, B, static_cast<uint64_t>(a.nnz > 0 ? a.nnz : 1) * B, 2 * B, B, B,
                      2 * B) ||
@@ -477,9 +587,13 @@ size_t partials_bytes(int32_t M, int32_t b)
 
 }  // namespace
 
+// workspace: [CTAs] counters first (their place does not depend on M), then
+// the partial sums
+static size_t counters_bytes() { return (static_cast<size_t>(num_sms()) * 4 + 15) & ~size_t(15); }
+
 size_t stream_workspace_bytes(int32_t M, const bsl_bsr *W)
 {
-    return partials_bytes(M, W->b) + static_cast<size_t>(num_sms()) * sizeof(int32_t);
+    return counters_bytes() + partials_bytes(M, W->b);
 }
 
 bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, void *ws,
@@ -488,9 +602,10 @@ bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, const v
     const int B = W->b;
     StreamArgs a;
     a.Y = static_cast<__nv_bfloat16 *>(Y);
-    a.ws = static_cast<float *>(ws);
-    a.cnt = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + partials_bytes(M, B));
+    a.cnt = static_cast<int32_t *>(ws);
+    a.ws = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + counters_bytes());
     a.row_ptr = W->row_ptr;
+    a.sbounds = W->sbounds;
     a.col_idx = W->col_idx;
     a.bias = static_cast<const __nv_bfloat16 *>(bias);
     a.M = M;

@@ -61,3 +61,29 @@ def dw_group_ptr(col_ptr, group: int) -> np.ndarray:
         n = col_ptr[c + 1] - col_ptr[c]
         out.append(out[-1] + (n + group - 1) // group)
     return np.asarray(out, dtype=np.int32)
+
+
+def stream_bounds(row_ptr, U: int) -> np.ndarray:
+    """CTA ranges of the weight-streaming forward, ``[U, b_0, ..., b_U]``.
+
+    CTA c starts at its equal share t = floor(c * nnz / U), moved to the start
+    of the block row holding block t or of the next row, whichever is nearer
+    (the row's own start on a tie), when that is at most q = floor(nnz / (4U))
+    blocks away; otherwise it starts at t."""
+    row_ptr = [int(v) for v in row_ptr]
+    nnz = row_ptr[-1]
+    q = nnz // (4 * U)
+    out = [U]
+    for c in range(U + 1):
+        t = c * nnz // U
+        bound = t
+        if 0 < t < nnz and q > 0:
+            r = max(i for i in range(len(row_ptr) - 1) if row_ptr[i] <= t)  # the row holding block t
+            da, dz = t - row_ptr[r], row_ptr[r + 1] - t
+            if da <= dz:
+                if da <= q:
+                    bound = t - da
+            elif dz <= q:
+                bound = t + dz
+        out.append(bound)
+    return np.asarray(out, dtype=np.int32)

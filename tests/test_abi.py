@@ -47,7 +47,7 @@ def _bsr(**kw):
 @pytest.mark.parametrize("bad,code", [
     (dict(b=48), 2), (dict(b=16), 2), (dict(N=250), 1), (dict(K=100), 1), (dict(nnz=-1), 1),
     (dict(nnz=65), 1), (dict(row_ptr=0), 1), (dict(values=0), 1), (dict(values=4104), 1),
-    (dict(status=0), 1),
+    (dict(status=0), 1), (dict(sbounds=0), 1),
 ])
 def test_bad_weight_descriptor_is_rejected_on_host(lib, bad, code):
     s = _bsr(**bad)
@@ -72,3 +72,17 @@ def test_status_strings(lib):
     assert lib.bsl_status_string(0) == b"BSL_OK"
     assert lib.bsl_status_string(4) == b"BSL_ERR_TIMEOUT"
     assert lib.bsl_small_m_max() == 32
+
+
+def test_binding_struct_matches_the_header():
+    """The ctypes mirror lists bsl_bsr's fields in the header's order and
+    sizes sbounds as BSL_SBOUNDS_LEN."""
+    import re
+    import sparse_gemm_b200 as sg
+    text = open(os.path.join(ROOT, "include", "bsl.h")).read()
+    body = text[text.index("typedef struct {"):text.index("} bsl_bsr;")]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\*?\s*(\w+)\s*[;,]", body)
+    assert [n for n, _ in sg._BSR._fields_] == names
+    m = re.search(r"#define BSL_SBOUNDS_LEN (\d+)", text)
+    assert m and int(m.group(1)) == sg.SBOUNDS_LEN

@@ -57,6 +57,8 @@ def check_pack(Wp, case, b):
         assert np.array_equal(getattr(Wp, pre + "_bptr").cpu().numpy(), gb), pre
         assert np.array_equal(getattr(Wp, pre + "_ent")[:len(ent)].cpu().numpy(), ent), pre
         assert np.array_equal(getattr(Wp, pre + "_blk")[:nnz].cpu().numpy(), blk), pre
+    U = torch.cuda.get_device_properties(Wp.values.device).multi_processor_count
+    assert np.array_equal(Wp.sbounds[:U + 2].cpu().numpy(), _plan.stream_bounds(want["row_ptr"], U))
     assert sg.device_status(Wp) == 0
 
 
@@ -165,6 +167,73 @@ def test_forward_stream_parity(case_args):
     got = run_forward(sg.forward_stream, case, b, M)
     ref, S = oracle.forward(case["X"], case["W"], case["mask"], b)
     assert_parity(got, ref, S, "forward_stream")
+
+
+def long_row_case(M, R, C, b, long_rows, per_row, seed):
+    """A weight whose rows in ``long_rows`` hold every block column and whose
+    other rows hold ``per_row`` blocks: the long rows reach across the ranges
+    of many CTAs of the weight-streaming forward."""
+    case = synth.random_case(M, R * b, C * b, b, R * per_row, seed)
+    rng = np.random.default_rng(seed)
+    mask = np.zeros((R, C), dtype=np.uint8)
+    for r in range(R):
+        if r in long_rows:
+            mask[r, :] = 1
+        else:
+            mask[r, rng.choice(C, per_row, replace=False)] = 1
+    case["mask"] = mask
+    return case
+
+
+LONG_ROW_CASES = [
+    # (M, R, C, b, long rows, blocks per other row, seed)
+    (16, 32, 256, 32, (0,), 4, 41),          # fewer blocks than 4 per CTA: equal shares
+    (5, 64, 256, 32, (5, 40), 8, 42),        # CTA bounds moved onto nearby row starts
+    (32, 48, 128, 64, (47,), 6, 43),
+]
+
+
+@pytest.mark.parametrize("case_args", LONG_ROW_CASES)
+def test_forward_stream_rows_across_many_ctas(case_args):
+    M, R, C, b, long_rows, per_row, seed = case_args
+    case = long_row_case(M, R, C, b, long_rows, per_row, seed)
+    Wp = pack_dev(case, b)
+    check_pack(Wp, case, b)
+    got = to_f64(sg.forward_stream(to_dev(case["X"]), Wp))
+    assert sg.device_status(Wp) == 0
+    ref, S = oracle.forward(case["X"], case["W"], case["mask"], b)
+    assert_parity(got, ref, S, "forward_stream")
+
+
+def test_forward_stream_replayed_from_a_cuda_graph():
+    # every call leaves the cross-CTA counters at zero, so every replay of a
+    # captured call finds them fresh (a row whose count were carried over
+    # would be left unwritten), with new inputs each time
+    M, R, C, b = 16, 32, 256, 32
+    case = long_row_case(M, R, C, b, (0, 9), 4, 44)
+    Wp = pack_dev(case, b)
+    X = to_dev(case["X"])
+    Y = torch.zeros((M, R * b), dtype=torch.bfloat16, device=X.device)
+    ws = torch.zeros(sg.forward_workspace_bytes(M, Wp), dtype=torch.uint8, device=X.device)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        sg.forward_stream(X, Wp, out=Y, workspace=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        sg.forward_stream(X, Wp, out=Y, workspace=ws)
+    for k in range(3):
+        Xk = synth.random_case(M, R * b, C * b, b, 4, 100 + k)["X"]
+        X.copy_(to_dev(Xk))
+        Y.zero_()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        ref, S = oracle.forward(Xk, case["W"], case["mask"], b)
+        assert_parity(to_f64(Y), ref, S, f"graph replay {k}")
+    assert sg.device_status(Wp) == 0
+    del g
 
 
 BWD_CASES = [

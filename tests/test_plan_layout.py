@@ -2,6 +2,7 @@
 tests hold the device-built plans to).  Each is checked against a property
 found independently: a walk over the stored blocks, not the same formula."""
 import numpy as np
+import pytest
 
 import oracle
 import synth
@@ -64,3 +65,36 @@ def test_dw_group_ptr_by_walking_the_columns():
         starts.append(ngroups)
         col_ptr = np.concatenate([[0], np.cumsum(mask.sum(0))])
         assert np.array_equal(_plan.dw_group_ptr(col_ptr, group), np.array(starts)), group
+
+
+@pytest.mark.parametrize("R,C,nnz,U,seed", [
+    (344, 128, 11008, 148, 1),   # the decode weight's shape and density
+    (224, 64, 1434, 148, 2),
+    (40, 30, 900, 148, 3),       # fewer blocks per CTA than rows are long
+    (12, 7, 50, 148, 4),         # fewer blocks than CTAs: equal shares
+    (64, 64, 4096, 16, 5),       # density 1
+])
+def test_stream_bounds_are_a_partition_that_keeps_short_rows_whole(R, C, nnz, U, seed):
+    mask = synth.mask_uniform(R, C, nnz, np.random.default_rng(seed))
+    mask[0, :] = 0
+    mask[R // 2, :] = 0
+    row_ptr = np.concatenate([[0], np.cumsum(mask.sum(axis=1))]).astype(np.int64)
+    nnz = int(row_ptr[-1])
+    sb = _plan.stream_bounds(row_ptr, U)
+    assert sb[0] == U and len(sb) == U + 2
+    b = sb[1:].astype(np.int64)
+    assert b[0] == 0 and b[-1] == nnz
+    assert np.all(np.diff(b) >= 0)
+    q = nnz // (4 * U)
+    t = np.arange(U + 1) * nnz // U
+    assert np.all(np.abs(b - t) <= q)
+    starts = set(int(v) for v in row_ptr)
+    for c in range(U + 1):
+        if b[c] != t[c]:
+            assert int(b[c]) in starts  # only ever moved onto a row start
+    # a row of at most 2q + 1 blocks always has a row start within q of any
+    # block inside it, so no bound falls strictly inside it
+    for r in range(R):
+        lo, hi = int(row_ptr[r]), int(row_ptr[r + 1])
+        if hi - lo <= 2 * q + 1:
+            assert not np.any((b > lo) & (b < hi)), r
