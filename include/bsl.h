@@ -108,10 +108,11 @@ typedef struct {
     int32_t *cgrp_ent;    /* [nnz] */
     int32_t *cgrp_blk;    /* [nnz] */
     int32_t *status;      /* [1] device status word; must be zeroed once at allocation */
-    int32_t *sched;       /* [8] work counters of the persistent tensor-core kernels, zeroed on
-                           * the call's stream before each launch (contents on entry do not
-                           * matter).  Two calls of the same contraction on one weight must not
-                           * run at the same time: they would share a counter. */
+    int32_t *sched;       /* [8] work counters of the persistent tensor-core kernels: zeroed by
+                           * bsl_pack, and every call (one that ran out of time included) leaves
+                           * them at zero again, so no memset precedes a launch.  Two calls of the
+                           * same contraction on one weight must not run at the same time: they
+                           * would share a counter. */
     int32_t *sbounds;     /* [BSL_SBOUNDS_LEN] block ranges of the weight-streaming forward's CTAs:
                            * [0] = U, the CTA count of the device bsl_pack ran on (its SM
                            * count), [1 + c] = first block of CTA c, c = 0..U ([1 + U] = nnz).

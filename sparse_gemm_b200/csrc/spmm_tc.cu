@@ -46,13 +46,14 @@
 //
 // Scheduling.  Units are taken from a per-weight atomic counter in the
 // order of decode_unit (heaviest first inside chunks of m-tiles), so the SMs
-// stay balanced under skewed block rows.  The first producer warp takes a
-// unit only when it starts issuing it (a CTA never sits on work another SM
-// could do) and publishes it to the other roles through a small ring in
-// shared memory.  The launcher zeroes the counter in stream order before
-// every launch, so a launch that never finished leaves nothing behind; two
-// launches of the same contraction on one weight must not run at the same
-// time (they would share the counter).
+// stay balanced under skewed block rows.  A scheduler warp takes a unit only
+// once a chunk slot is free (the CTA holds at most one unit beyond the one
+// its producers issue) and publishes it to the other roles through a small
+// ring in shared memory.  The CTA that makes the launch's last take past the
+// final unit sets the counter back to zero, and a CTA that ran out of time
+// first takes the remaining units, so every launch leaves the counter at zero
+// and no memset precedes the kernel; two launches of the same contraction on
+// one weight must not run at the same time (they would share the counter).
 //
 // Roles per CTA (persistent grid, one CTA per SM):
 //   warps 0..P-1   producers: TMA tile copies of the activation tile and of
@@ -117,7 +118,7 @@ struct SpmmArgs {
     const int32_t *grp_bptr;   // [ngroups+1] block range per group
     const int32_t *grp_ent;    // entries: coordinate | (mask << 24)
     const int32_t *grp_blk;    // BSR block of every present member, entry by entry
-    int32_t *sched;            // [1] next unit (zeroed in stream order before every launch)
+    int32_t *sched;            // [1] next unit (zero between launches: each launch resets it)
     const __nv_bfloat16 *bias; // [nseg * b] added to every output row (forward only; null: none)
     int32_t *status;
     uint64_t timeout_ns;
@@ -151,6 +152,19 @@ __device__ __forceinline__ void decode_unit(const SpmmArgs &a, int ord, int *mt,
     const int r = ord - ch * per_chunk;
     *g = r / nmt;
     *mt = mt0 + (r - *g * nmt);
+}
+
+// Take the next unit from the per-weight counter (-1: none left).  Every CTA
+// ends with exactly one take past the last unit; the take that returns
+// units + gridDim.x - 1 is the last take of the launch, so that CTA sets the
+// counter back to zero for the next launch (stream order makes the store
+// visible to it).
+__device__ __forceinline__ int take_unit(int32_t *sched, int units)
+{
+    const int ord = atomicAdd(sched, 1);
+    if (ord < units) return ord;
+    if (ord == units + static_cast<int>(gridDim.x) - 1) *reinterpret_cast<volatile int32_t *>(sched) = 0;
+    return -1;
 }
 
 // Ring cursor: slot index + phase parity.
@@ -467,8 +481,8 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         // dependent global loads of the plan thus run ahead of the copies.  A
         // new unit is taken only once a chunk slot is free, so the CTA holds at
         // most one unit beyond the one its producers are issuing.
-        bool ok = true;
-        int cc = 0;  // chunks staged
+        bool ok = true, drained = false;  // drained: this CTA's take past the last unit is done
+        int cc = 0;                       // chunks staged
         for (int j = 0; ok; ++j) {
             int good = 1;
             if (lane == 0 && cc >= Cfg::D)
@@ -479,8 +493,8 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
             }
             int ord = -1;
             if (lane == 0) {
-                ord = atomicAdd(args.sched, 1);
-                if (ord >= args.units) ord = -1;
+                ord = take_unit(args.sched, args.units);
+                drained = ord < 0;
             }
             ord = __shfl_sync(0xffffffffu, ord, 0);
             int mt = 0, g = 0, z = 0, zend = 0, bcur = 0;
@@ -565,6 +579,11 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         if (lane == 0 && !ok) {
             *abort_flag = 1;
             set_status(args.status, BSL_ERR_TIMEOUT);
+            // take the remaining units too (they are left undone: the status
+            // reports the timeout), so that the counter still returns to zero
+            if (!drained)
+                while (take_unit(args.sched, args.units) >= 0) {
+                }
         }
         __syncwarp();
     } else {
@@ -692,11 +711,8 @@ bsl_status run(const CUtensorMap &a, const CUtensorMap &o, const CUtensorMap &w,
     auto kern = k_spmm_tc<B, TRANS>;
     const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(kern), Cfg::SMEM_BYTES);
     if (sa != BSL_OK) return sa;
-    cudaError_t e;
-    // the work counters start at zero on every launch, in stream order, so a
-    // launch that did not finish cannot make a later one skip units
-    e = cudaMemsetAsync(args.sched, 0, 2 * sizeof(int32_t), s);
-    if (e != cudaSuccess) return cuda_status(e);
+    // the work counter is zero here: the pack zeroed it and every launch,
+    // one that ran out of time included, sets it back to zero at its end
     const int grid = args.units < num_sms() ? args.units : num_sms();
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(a, o, w, args);
     return cuda_status(cudaGetLastError());

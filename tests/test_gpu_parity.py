@@ -312,31 +312,68 @@ def test_results_are_deterministic():
         assert torch.equal(u.view(torch.int16), v.view(torch.int16))
 
 
-def test_work_counters_do_not_carry_over_between_launches():
-    """The persistent kernels take units from counters in the packed weight.
-    Each launch starts them from zero in stream order, so whatever a
-    previous launch left there (here: counters poisoned by hand, as a launch
-    that never finished would leave them) cannot make a later launch skip
-    units: results stay bit-identical for any M, ragged or not."""
+def test_work_counters_return_to_zero_after_every_launch():
+    """The persistent kernels take units from counters in the packed weight,
+    and the small-M forward counts CTAs in on rows they share in its
+    workspace.  No memset precedes a launch: every launch leaves its
+    counters at zero, so later launches of any M (ragged or not) take every
+    unit and results stay bit-identical."""
     case = synth.random_case(700, 1024, 768, 64, 120, 44)
     Wp = pack_dev(case, 64)
     X, dY = to_dev(case["X"]), to_dev(case["dY"])
+    ws = torch.zeros(sg.forward_workspace_bytes(32, Wp), dtype=torch.uint8, device=X.device)
     first = None
-    for M, poison in ((700, 0), (256, 5), (1, 10 ** 6), (700, 3)):
-        Wp.sched.fill_(poison)
+    for M in (700, 256, 1, 700, 33, 700):
         y = sg.forward_tc(X[:M].contiguous(), Wp)
-        Wp.sched.fill_(poison)
         dx = sg.backward_input(dY[:M].contiguous(), Wp)
+        ys = sg.forward_stream(X[:min(M, 32)].contiguous(), Wp, workspace=ws)
         torch.cuda.synchronize()
+        assert int(Wp.sched.abs().sum()) == 0, M
+        ncnt = torch.cuda.get_device_properties(X.device).multi_processor_count
+        assert int(ws[:4 * ncnt].view(torch.int32).abs().sum()) == 0, M
         if M == 700:
             if first is None:
-                first = (y.clone(), dx.clone())
+                first = (y.clone(), dx.clone(), ys.clone())
             else:
                 assert torch.equal(y.view(torch.int16), first[0].view(torch.int16))
                 assert torch.equal(dx.view(torch.int16), first[1].view(torch.int16))
+                assert torch.equal(ys.view(torch.int16), first[2].view(torch.int16))
     ref, S = oracle.forward(case["X"], case["W"], case["mask"], 64)
-    assert_parity(to_f64(first[0]), ref, S, "forward after poisoned counters")
+    assert_parity(to_f64(first[0]), ref, S, "forward, repeated launches")
+    ref32, S32 = oracle.forward(case["X"][:32], case["W"], case["mask"], 64)
+    assert_parity(to_f64(first[2]), ref32, S32, "forward_stream, repeated launches")
     assert sg.device_status(Wp) == 0
+
+
+def test_forward_tc_replayed_from_a_cuda_graph():
+    # each replay of a captured call takes every unit again (the counter a
+    # launch used is back at zero when the next one starts)
+    M, N, K, b = 600, 1024, 768, 64
+    case = synth.random_case(M, N, K, b, 120, 45)
+    Wp = pack_dev(case, b)
+    X = to_dev(case["X"])
+    Y = torch.zeros((M, N), dtype=torch.bfloat16, device=X.device)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        sg.forward_tc(X, Wp, out=Y)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        sg.forward_tc(X, Wp, out=Y)
+    for k in range(3):
+        Xk = synth.random_case(M, N, K, b, 4, 200 + k)["X"]
+        X.copy_(to_dev(Xk))
+        Y.zero_()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        rows = np.arange(0, M, 7)
+        ref, S = oracle.forward(Xk, case["W"], case["mask"], b, rows=rows)
+        assert_parity(to_f64(Y)[rows], ref, S, f"graph replay {k}")
+    assert int(Wp.sched.abs().sum()) == 0
+    assert sg.device_status(Wp) == 0
+    del g
 
 
 def test_density_one_matches_cublas():
