@@ -76,6 +76,9 @@ struct SpmmCfg {
     static constexpr int MSUB = 2;                      // MMA row blocks per unit
     static constexpr int MT = BM * MSUB;                // rows of M per unit
     static constexpr int G = 128 / B;                   // members per group
+    // b = 32: every entry is one MMA of all G members (N = 128), absent
+    // members' blocks read as zeros; b = 64: runs of present members only
+    static constexpr bool PAD = B == 32;
     static constexpr int ROW_BYTES = B * 2;             // one tile row: 64 B (b=32) or 128 B (b=64)
     static constexpr int SUB_BYTES = BM * ROW_BYTES;    // one 128-row half of the activation tile
     static constexpr int X_BYTES = MT * ROW_BYTES;      // activation tile
@@ -279,8 +282,12 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         const int p = warp;
         int e = 0;                  // entries walked so far (all units of this CTA)
         int fills[Cfg::S / Cfg::P]; // fills issued per owned slot
+        uint32_t stale[Cfg::S / Cfg::P];  // padded mode: positions of an owned slot that may hold a block
 #pragma unroll
-        for (int i = 0; i < Cfg::S / Cfg::P; ++i) fills[i] = 0;
+        for (int i = 0; i < Cfg::S / Cfg::P; ++i) {
+            fills[i] = 0;
+            stale[i] = (1u << Cfg::G) - 1;  // shared memory starts with anything in it
+        }
         bool ok = true;
         for (int cc = 0; ok; ++cc) {
             const int cs = cc & (Cfg::D - 1);
@@ -304,14 +311,40 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                 // the entry that reuses this slot next: pull its activation tile into L2
                 const int tn = t + Cfg::S;
                 const uint32_t entn = __shfl_sync(0xffffffffu, el, tn < n ? tn : 0);
+                const int ee = e + t;
+                const int slot = ee & (Cfg::S - 1);
+                const int use = ee >> Cfg::S_LOG;
+                const uint32_t mask = ent >> 24;
+                const uint32_t k = __popc(mask);
+                if (lane == 0 && use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, tmo, abort_flag)) good = 0;
+                if (!__shfl_sync(0xffffffffu, good, 0)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *sp = slots + slot * Cfg::SLOT_BYTES;
+                if constexpr (Cfg::PAD) {
+                    // member m's block sits at position m; positions of absent
+                    // members must read as zeros, so the ones that still hold an
+                    // earlier entry's block are cleared (generic-proxy stores, made
+                    // visible to the tensor core before the barrier publishes them)
+                    uint32_t zero = 0;
+#pragma unroll
+                    for (int i = 0; i < Cfg::S / Cfg::P; ++i)
+                        if (slot == p + i * Cfg::P) {
+                            zero = stale[i] & ~mask;
+                            stale[i] = mask;
+                        }
+                    if (zero) {
+                        for (uint32_t z = zero; z; z &= z - 1) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(sp + Cfg::X_BYTES + (__ffs(z) - 1) * Cfg::W_BYTES);
+                            for (int c = lane; c < Cfg::W_BYTES / 16; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+                        }
+                        fence_async_smem();
+                        __syncwarp();
+                    }
+                }
                 if (lane == 0) {
-                    const int ee = e + t;
-                    const int slot = ee & (Cfg::S - 1);
-                    const int use = ee >> Cfg::S_LOG;
-                    const uint32_t mask = ent >> 24;
-                    const uint32_t k = __popc(mask);
-                    if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, tmo, abort_flag)) good = 0;
-                    if (good) {
+                    if constexpr (!Cfg::PAD) {
                         // runs: consecutive present members with the same first-write
                         // status; their blocks are consecutive in the slot
                         uint2 *hr = reinterpret_cast<uint2 *>(hdr + slot * Cfg::HDR_V4);
@@ -338,23 +371,21 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                                                   make_idesc_bf16(128, len * B, false, TRANS));
                         }
                         hr[0].x |= static_cast<uint32_t>(nr) << 24;
-                        uint8_t *sp = slots + slot * Cfg::SLOT_BYTES;
-                        mbar_arrive_expect_tx(&full[slot], Cfg::X_BYTES + k * Cfg::W_BYTES);
-                        tma_load_2d(sp, &tmA, &full[slot], static_cast<int>(ent & 0xFFFFFFu) * B, m0);
-                        // the present members' blocks, one swizzled tile each, straight
-                        // from the packed values (stored once, in BSR order)
-                        for (uint32_t qq = 0; qq < k; ++qq)
-                            tma_load_3d(sp + Cfg::X_BYTES + qq * Cfg::W_BYTES, &tmW, &full[slot], 0, 0,
-                                        ids[off + qq]);
-                        if (tn < n) tma_prefetch_2d(&tmA, static_cast<int>(entn & 0xFFFFFFu) * B, m0);
-#pragma unroll
-                        for (int i = 0; i < Cfg::S / Cfg::P; ++i)
-                            if (slot == p + i * Cfg::P) fills[i] = use + 1;
                     }
-                }
-                if (!__shfl_sync(0xffffffffu, good, 0)) {
-                    ok = false;
-                    break;
+                    mbar_arrive_expect_tx(&full[slot], Cfg::X_BYTES + k * Cfg::W_BYTES);
+                    tma_load_2d(sp, &tmA, &full[slot], static_cast<int>(ent & 0xFFFFFFu) * B, m0);
+                    // the present members' blocks, one swizzled tile each, straight
+                    // from the packed values (stored once, in BSR order): at the
+                    // member's own position (padded) or packed in member order
+                    uint32_t mm = mask;
+                    for (uint32_t qq = 0; qq < k; ++qq, mm &= mm - 1) {
+                        const uint32_t pos = Cfg::PAD ? static_cast<uint32_t>(__ffs(mm) - 1) : qq;
+                        tma_load_3d(sp + Cfg::X_BYTES + pos * Cfg::W_BYTES, &tmW, &full[slot], 0, 0, ids[off + qq]);
+                    }
+                    if (tn < n) tma_prefetch_2d(&tmA, static_cast<int>(entn & 0xFFFFFFu) * B, m0);
+#pragma unroll
+                    for (int i = 0; i < Cfg::S / Cfg::P; ++i)
+                        if (slot == p + i * Cfg::P) fills[i] = use + 1;
                 }
             }
             // every lane is done with the chunk (lane 0 read its block ids)
@@ -426,30 +457,46 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
                 }
                 const uint32_t soff = static_cast<uint32_t>(slot) * (Cfg::SLOT_BYTES >> 4);
                 const uint32_t xlo = xlo0 + soff, wlo = wlo0 + soff;
-                const uint4 *hs = hdr + slot * Cfg::HDR_V4;
-                const uint4 h0 = hs[0];
-                const int nr = static_cast<int>((h0.x >> 24) & 0xFu);
-                auto issue_run = [&](uint32_t x, uint32_t y) {
-                    const uint32_t dcol = d0 + (x & 0xFFu);
-                    const uint32_t blo = wlo + ((x >> 8) & 0xFFFFu);
-                    const uint32_t st = x >> 28;
+                if constexpr (Cfg::PAD) {
+                    // one run of all members; the unit's first entry overwrites
+                    // the whole accumulator, later ones add to it
+                    const uint32_t st = t > 0 ? 1u : 0u;
+                    const uint32_t y = make_idesc_bf16(128, Cfg::G * B, false, TRANS);
 #pragma unroll
                     for (int kk = 0; kk < B / 16; ++kk)
-                        umma_bf16_lo_lead(lead, dcol, xlo + kk * 2, xhi, blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
+                        umma_bf16_lo_lead(lead, d0, xlo + kk * 2, xhi, wlo + kk * KSTEP_W, whi, y, kk ? 1u : st);
                     if (two) {
 #pragma unroll
                         for (int kk = 0; kk < B / 16; ++kk)
-                            umma_bf16_lo_lead(lead, dcol + Cfg::HALF_COLS, xlo + SUB_LO + kk * 2, xhi,
-                                               blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
+                            umma_bf16_lo_lead(lead, d0 + Cfg::HALF_COLS, xlo + SUB_LO + kk * 2, xhi,
+                                               wlo + kk * KSTEP_W, whi, y, kk ? 1u : st);
                     }
-                };
-                issue_run(h0.x, h0.y);
-                if (nr > 1) issue_run(h0.z, h0.w);
-                if constexpr (Cfg::HDR_V4 > 1) {
-                    if (nr > 2) {
-                        const uint4 h1 = hs[1];
-                        issue_run(h1.x, h1.y);
-                        if (nr > 3) issue_run(h1.z, h1.w);
+                } else {
+                    const uint4 *hs = hdr + slot * Cfg::HDR_V4;
+                    const uint4 h0 = hs[0];
+                    const int nr = static_cast<int>((h0.x >> 24) & 0xFu);
+                    auto issue_run = [&](uint32_t x, uint32_t y) {
+                        const uint32_t dcol = d0 + (x & 0xFFu);
+                        const uint32_t blo = wlo + ((x >> 8) & 0xFFFFu);
+                        const uint32_t st = x >> 28;
+#pragma unroll
+                        for (int kk = 0; kk < B / 16; ++kk)
+                            umma_bf16_lo_lead(lead, dcol, xlo + kk * 2, xhi, blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
+                        if (two) {
+#pragma unroll
+                            for (int kk = 0; kk < B / 16; ++kk)
+                                umma_bf16_lo_lead(lead, dcol + Cfg::HALF_COLS, xlo + SUB_LO + kk * 2, xhi,
+                                                   blo + kk * KSTEP_W, whi, y, kk ? 1u : st);
+                        }
+                    };
+                    issue_run(h0.x, h0.y);
+                    if (nr > 1) issue_run(h0.z, h0.w);
+                    if constexpr (Cfg::HDR_V4 > 1) {
+                        if (nr > 2) {
+                            const uint4 h1 = hs[1];
+                            issue_run(h1.x, h1.y);
+                            if (nr > 3) issue_run(h1.z, h1.w);
+                        }
                     }
                 }
                 // the slot is free once these MMAs finish
