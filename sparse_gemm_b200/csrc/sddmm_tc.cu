@@ -10,12 +10,13 @@
 //
 // Tiles.  The block grid is cut into tiles of GR x GC blocks (GR*b = 128 rows
 // of dW, GC*b = 128 columns).  For a tile, every stage brings in 128 rows of
-// M of the dY strips dY[:, r-block] of the tile's block rows and of the X
-// strips X[:, c-block] of its block columns, and one tcgen05.mma of
-// M = 128, N = 128 per 16 rows computes the whole 128 x 128 tile of
-// dY^T . X (fp32 in TMEM).  Only strips of block rows / columns that hold a
-// stored block in the tile are copied (a skipped strip leaves old data in
-// shared memory, which only reaches accumulator entries that are never
+// M of two 64-column strips of dY (the tile's 128 dY columns) and two of X,
+// and one tcgen05.mma of M = 128, N = 128 per 16 rows computes the whole
+// 128 x 128 tile of dY^T . X (fp32 in TMEM).  A strip is one block column
+// for b = 64 and two for b = 32: its 128-byte rows move at the copy engine's
+// full rate, where 64-byte rows move at about 70 % of it.  Only strips that
+// hold a stored block of the tile are copied (a skipped strip leaves old data
+// in shared memory, which only reaches accumulator entries that are never
 // stored), only stored blocks are written out, and tiles without a stored
 // block are skipped.  Each strip is read once per tile instead of once per
 // stored block, and every MMA is full width.
@@ -37,16 +38,19 @@ struct SddmmCfg {
     static constexpr int GR = 128 / B;                   // block rows per tile (MMA M = 128)
     static constexpr int GC = 128 / B;                   // block columns per tile (MMA N = 128)
     static constexpr int MK = 128;                       // rows of M reduced per stage
-    static constexpr int ROW_BYTES = B * 2;
-    static constexpr int T_BYTES = MK * ROW_BYTES;       // one strip tile (MK x b)
-    static constexpr int STAGE_BYTES = (GR + GC) * T_BYTES;
+    static constexpr int SW = 64;                        // strip width (columns): 128-byte rows
+    static constexpr int NS = 128 / SW;                  // strips per operand
+    static constexpr int BPS = SW / B;                   // block columns per strip
+    static constexpr int ROW_BYTES = SW * 2;
+    static constexpr int T_BYTES = MK * ROW_BYTES;       // one strip tile (MK x 64)
+    static constexpr int STAGE_BYTES = 2 * NS * T_BYTES;
     static constexpr int STAGES = 3;
     static constexpr int P = STAGES;                     // producer warps: one per stage slot
     static constexpr int THREADS = (P + 5) * 32;
     static constexpr int ACC = 2;
     static constexpr int ACC_COLS = GC * B;              // 128
     static constexpr int TMEM_COLS = ACC * ACC_COLS;     // 256
-    static constexpr uint32_t LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
+    static constexpr uint32_t LAYOUT = kLayoutSw128;
     static constexpr uint32_t SBO = 8 * ROW_BYTES;
     static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC + 1;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NUM_BARS * 8 + 16 + 1024;
@@ -107,6 +111,18 @@ __device__ __forceinline__ int tile_blocks(const SddmmArgs &a, int t, int lane, 
     return pos;
 }
 
+// Strips holding any of the tile's blocks in `blocks` (bit i = block i).
+template <int B>
+__device__ __forceinline__ uint32_t strip_mask(uint32_t blocks)
+{
+    using Cfg = SddmmCfg<B>;
+    uint32_t m = 0;
+#pragma unroll
+    for (int q = 0; q < Cfg::NS; ++q)
+        if ((blocks >> (q * Cfg::BPS)) & ((1u << Cfg::BPS) - 1u)) m |= 1u << q;
+    return m;
+}
+
 template <int B>
 __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
     k_sddmm_tc(const __grid_constant__ CUtensorMap tmDY, const __grid_constant__ CUtensorMap tmX,
@@ -164,7 +180,8 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
             int rg, cg;
             tile_blocks<B>(args, t, lane, &rm, &cm, &rg, &cg);
             if (!rm) continue;
-            const uint32_t nstrips = __popc(rm) + __popc(cm);
+            const uint32_t rs = strip_mask<B>(rm), cs = strip_mask<B>(cm);
+            const uint32_t nstrips = __popc(rs) + __popc(cs);
             for (int ks = 0; ks < args.ksteps; ++ks, ++i) {
                 if (i % Cfg::P != warp) continue;
                 const int stage = i % Cfg::STAGES;
@@ -177,15 +194,15 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
                         uint8_t *sa = stages + stage * Cfg::STAGE_BYTES;
                         mbar_arrive_expect_tx(&full[stage], nstrips * Cfg::T_BYTES);
 #pragma unroll
-                        for (int q = 0; q < Cfg::GR; ++q)
-                            if ((rm >> q) & 1u)
-                                tma_load_2d(sa + q * Cfg::T_BYTES, &tmDY, &full[stage], (rg * Cfg::GR + q) * B,
-                                            ks * Cfg::MK);
+                        for (int q = 0; q < Cfg::NS; ++q)
+                            if ((rs >> q) & 1u)
+                                tma_load_2d(sa + q * Cfg::T_BYTES, &tmDY, &full[stage],
+                                            rg * Cfg::GR * B + q * Cfg::SW, ks * Cfg::MK);
 #pragma unroll
-                        for (int q = 0; q < Cfg::GC; ++q)
-                            if ((cm >> q) & 1u)
-                                tma_load_2d(sa + (Cfg::GR + q) * Cfg::T_BYTES, &tmX, &full[stage],
-                                            (cg * Cfg::GC + q) * B, ks * Cfg::MK);
+                        for (int q = 0; q < Cfg::NS; ++q)
+                            if ((cs >> q) & 1u)
+                                tma_load_2d(sa + (Cfg::NS + q) * Cfg::T_BYTES, &tmX, &full[stage],
+                                            cg * Cfg::GC * B + q * Cfg::SW, ks * Cfg::MK);
                         issued |= 1u << stage;
                         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     }
@@ -230,9 +247,9 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(stages + stage * Cfg::STAGE_BYTES);
-                const uint32_t x0 = a0 + Cfg::GR * Cfg::T_BYTES;
-                // A: the GR dY strips side by side along M (MN-major, T_BYTES apart);
-                // B: the GC X strips along N; K = 16 rows of M per instruction
+                const uint32_t x0 = a0 + Cfg::NS * Cfg::T_BYTES;
+                // A: the dY strips side by side along M (MN-major, T_BYTES apart);
+                // B: the X strips along N; K = 16 rows of M per instruction
                 const uint64_t ad0 = make_sdesc(a0, Cfg::T_BYTES, Cfg::SBO, Cfg::LAYOUT);
                 const uint64_t xd0 = make_sdesc(x0, Cfg::T_BYTES, Cfg::SBO, Cfg::LAYOUT);
                 const uint32_t alo = static_cast<uint32_t>(ad0), ahi = static_cast<uint32_t>(ad0 >> 32);
@@ -352,8 +369,10 @@ bsl_status launch_sddmm_tc(const void *dY, const void *X, int32_t M, const bsl_b
     const int B = W->b;
     if (W->nnz == 0) return BSL_OK;
     CUtensorMap mdy, mx;
-    if (!make_map_2d(&mdy, dY, W->N, M, static_cast<uint64_t>(W->N) * 2, B, 128, 2 * B) ||
-        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, B, 128, 2 * B))
+    // 64-column strips (128-byte rows, 128-byte swizzle); a strip that reaches
+    // past the last column reads zeros there
+    if (!make_map_2d(&mdy, dY, W->N, M, static_cast<uint64_t>(W->N) * 2, 64, 128, 128) ||
+        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, 64, 128, 128))
         return BSL_ERR_CUDA;
     const int G = 128 / B;
     SddmmArgs args;

@@ -243,6 +243,7 @@ BWD_CASES = [
     (257, 384, 640, 64, 25, 33, (0,), (1, 9)),
     (130, 1024, 512, 32, 512, 34, (), ()),    # density 1
     (64, 768, 1024, 64, 96, 35, (), ()),
+    (40, 96, 32, 32, 2, 36, (), ()),          # one block column, three block rows: strips past the edge
 ]
 
 
