@@ -118,8 +118,9 @@ typedef struct {
                            * count), [1 + c] = first block of CTA c, c = 0..U ([1 + U] = nnz).
                            * Bound c is the start of the block row holding block
                            * floor(c * nnz / U) or of the next one, whichever is nearer, when
-                           * that is at most nnz / (4U) blocks away, else floor(c * nnz / U)
-                           * itself: short block rows are never split between CTAs. */
+                           * that is at most nnz / (2U) blocks away, else floor(c * nnz / U)
+                           * itself: block rows of up to nnz / U + 1 blocks are never split
+                           * between CTAs. */
 } bsl_bsr;
 
 /* Human-readable name of a status code (static string). */

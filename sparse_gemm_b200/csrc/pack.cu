@@ -300,9 +300,10 @@ void launch_group_plans(const bsl_bsr *o, cudaStream_t s)
 // Block ranges of the U CTAs of the weight-streaming forward.  CTA c starts
 // at t = floor(c * nnz / U), moved to the start of the block row holding
 // block t or of the next row, whichever is nearer, when that is at most
-// q = floor(nnz / (4U)) blocks away.  Every bound stays within q of its equal
-// share, and equal shares are at least 4q apart, so the bounds never
-// decrease; sb[0] = U tells the kernel which grid size they were made for.
+// q = floor(nnz / (2U)) blocks away, so no row of up to 2q + 1 blocks is ever
+// split between CTAs.  Every bound stays within q of its equal share, and
+// equal shares are at least 2q apart, so the bounds never decrease; sb[0] = U
+// tells the kernel which grid size they were made for.
 __global__ void k_stream_bounds(const int32_t *__restrict__ row_ptr, int32_t R, int32_t nnz, int32_t U,
                                 int32_t *__restrict__ sb)
 {
@@ -310,7 +311,7 @@ __global__ void k_stream_bounds(const int32_t *__restrict__ row_ptr, int32_t R, 
     if (c == 0) sb[0] = U;
     if (c > U) return;
     const int t = static_cast<int>(static_cast<int64_t>(c) * nnz / U);
-    const int q = static_cast<int>(nnz / (4LL * U));
+    const int q = static_cast<int>(nnz / (2LL * U));
     int bound = t;
     if (t > 0 && t < nnz && q > 0) {
         int lo = 0, hi = R;  // the last row lo with row_ptr[lo] <= t (row_ptr[R] = nnz > t)

@@ -10,8 +10,8 @@
 // Decomposition: the BSR block list [0, nnz) is cut into contiguous ranges,
 // one per CTA of a one-CTA-per-SM grid: equal shares, each moved to a
 // nearby block-row start where there is one (the pack computes these
-// bounds), so short block rows never straddle two CTAs and only rows longer
-// than about a quarter of a CTA's share do.  Each CTA's range is cut into
+// bounds), so block rows of up to a CTA's share never straddle two CTAs and
+// only longer ones do.  Each CTA's range is cut into
 // equal shares for its 8 warps (block counts, not block rows, are balanced).
 // Each warp streams its share through its own ring of slots; a slot holds one
 // weight block and the activation slice X[0:MP, c*b:(c+1)*b] it multiplies,
@@ -158,10 +158,11 @@ __device__ __forceinline__ int warp_of(int p, int cq0, int n)
 }
 
 // The CTA whose range holds block p (0 <= p < nnz); warp-collective.  A
-// bound made by the pack lies within nnz / (4U) blocks of its equal share and
-// equal shares are at least 4 times that apart, so the CTA is the equal
-// share's CTA or one of its two neighbours: lanes 0..3 look at the bounds of
-// those three in one round of loads.
+// bound made by the pack lies within q = floor(nnz / (2U)) blocks of its equal
+// share and equal shares are at least 2q apart (more than q between a share's
+// bound and the next share's), so the CTA is the equal share's CTA or one of
+// its two neighbours: lanes 0..3 look at the bounds of those three in one
+// round of loads.
 __device__ __forceinline__ int cta_of(const StreamArgs &a, bool snapped, int p, int U, int lane)
 {
     const int c = share_of(p, U, a.nnz);
@@ -210,6 +211,24 @@ struct RowAcc {
             for (int j = 0; j < NT; ++j)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) d[i][j][e] = 0.f;
+    }
+    // add a block row stored as floats by store() (element (n, m) at n * MP + m);
+    // cg: read through L2 only (another CTA wrote it)
+    template <bool CG = false>
+    __device__ __forceinline__ void add(const float *src, int lane)
+    {
+        const int g = lane >> 2, c2 = (lane & 3) * 2;
+#pragma unroll
+        for (int i = 0; i < MT; ++i)
+#pragma unroll
+            for (int j = 0; j < NT; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float2 *p = reinterpret_cast<const float2 *>(src + (i * 16 + g + h * 8) * MP + j * 8 + c2);
+                    const float2 v = CG ? __ldcg(p) : *p;
+                    d[i][j][2 * h] += v.x;
+                    d[i][j][2 * h + 1] += v.y;
+                }
     }
     // store as floats, element (feature n, token m) at n * MP + m
     __device__ __forceinline__ void store(float *dst, int lane) const
@@ -269,29 +288,12 @@ __device__ __forceinline__ void write_row(const RowAcc<B, MP> &acc, const Stream
     store_staged<B, MP>(a, stage, r, lane);
 }
 
-// A block row held as floats (n * MP + m, PER = b*MP/32 per lane): bias,
-// bf16, staged, stored.
-template <int B, int MP>
-__device__ __forceinline__ void write_row_flat(const float (&sum)[B * MP / 32], const StreamArgs &a, int r,
-                                               uint8_t *stage, int lane)
-{
-    __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(stage);
-#pragma unroll
-    for (int e = 0; e < B * MP / 32; ++e) {
-        const int idx = e * 32 + lane;
-        const int n = idx / MP, m = idx % MP;
-        s[m * B + n] = __float2bfloat16_rn(sum[e] + bias_of(a, static_cast<int64_t>(r) * B + n));
-    }
-    store_staged<B, MP>(a, stage, r, lane);
-}
-
 template <int B, int MP>
 __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     k_stream_fwd(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const StreamArgs a)
 {
     using Cfg = StreamCfg<B, MP>;
-    constexpr int PER = Cfg::PART / 32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -490,9 +492,8 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
         const int beg = which == 0 ? fr_beg : lr_beg, end = which == 0 ? fr_end : lr_end;
         const int lead = warp_of(beg > cq0 ? beg : cq0, cq0, cn);
         if (lead != warp) continue;
-        float sum[PER];
-#pragma unroll
-        for (int e = 0; e < PER; ++e) sum[e] = 0.f;
+        RowAcc<B, MP> sum;  // the partials added in warp (then CTA) order, from zero
+        sum.zero();
         const int wl = warp_of(end - 1 < cq1 - 1 ? end - 1 : cq1 - 1, cq0, cn);
         for (int w = warp; w <= wl; ++w) {
             const int sb = warp_bound(w, cq0, cn);
@@ -500,18 +501,16 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
             // slot 0 holds a row that began before the warp's share, slot 1 the rest
             const float *src = reinterpret_cast<const float *>(smem + w * Cfg::WARP_BYTES) +
                                (sb > beg ? 0 : Cfg::PART);
-#pragma unroll
-            for (int e = 0; e < PER; ++e) sum[e] += src[e * 32 + lane];
+            sum.add(src, lane);
         }
         if (beg >= cq0 && end <= cq1) {  // the whole row lies in this CTA's share
-            write_row_flat<B, MP>(sum, a, r, stage, lane);
+            write_row<B, MP>(sum, a, r, stage, lane);
             continue;
         }
         // the row reaches into other CTAs: this CTA's sum goes to the workspace;
         // the last CTA to arrive adds all of them in CTA order
         float *mine_ws = a.ws + (static_cast<int64_t>(blockIdx.x) * 2 + (cq0 >= beg ? 0 : 1)) * Cfg::PART;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) __stcg(mine_ws + e * 32 + lane, sum[e]);
+        sum.store(mine_ws, lane);
         // CTAs holding the row's first and last block, and how many of the
         // CTAs between them hold any block (31 bounds per round of loads)
         const int c0 = cta_of(a, snapped, beg, U, lane);
@@ -531,8 +530,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
         last = __shfl_sync(0xffffffffu, last, 0);
         __syncwarp();
         if (!last) continue;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) sum[e] = 0.f;
+        sum.zero();
         for (int base = c0; base <= c1; base += 31) {
             const int c = base + lane;
             const int bc = cta_bound(a, snapped, c < U ? c : U, U);
@@ -544,12 +542,11 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
                 const int j = __ffs(m) - 1;
                 const float *src =
                     a.ws + (static_cast<int64_t>(base + j) * 2 + ((first >> j) & 1u ? 0 : 1)) * Cfg::PART;
-#pragma unroll
-                for (int e = 0; e < PER; ++e) sum[e] += __ldcg(src + e * 32 + lane);
+                sum.template add<true>(src, lane);
             }
         }
         if (lane == 0) a.cnt[c0] = 0;  // every contributor is in: ready for the next call
-        write_row_flat<B, MP>(sum, a, r, stage, lane);
+        write_row<B, MP>(sum, a, r, stage, lane);
     }
 
     // block rows without blocks: bias (or zeros), rows r = gw, gw + GW, ...

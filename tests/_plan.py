@@ -68,11 +68,11 @@ def stream_bounds(row_ptr, U: int) -> np.ndarray:
 
     CTA c starts at its equal share t = floor(c * nnz / U), moved to the start
     of the block row holding block t or of the next row, whichever is nearer
-    (the row's own start on a tie), when that is at most q = floor(nnz / (4U))
+    (the row's own start on a tie), when that is at most q = floor(nnz / (2U))
     blocks away; otherwise it starts at t."""
     row_ptr = [int(v) for v in row_ptr]
     nnz = row_ptr[-1]
-    q = nnz // (4 * U)
+    q = nnz // (2 * U)
     out = [U]
     for c in range(U + 1):
         t = c * nnz // U

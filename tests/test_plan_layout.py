@@ -85,7 +85,7 @@ def test_stream_bounds_are_a_partition_that_keeps_short_rows_whole(R, C, nnz, U,
     b = sb[1:].astype(np.int64)
     assert b[0] == 0 and b[-1] == nnz
     assert np.all(np.diff(b) >= 0)
-    q = nnz // (4 * U)
+    q = nnz // (2 * U)
     t = np.arange(U + 1) * nnz // U
     assert np.all(np.abs(b - t) <= q)
     starts = set(int(v) for v in row_ptr)
