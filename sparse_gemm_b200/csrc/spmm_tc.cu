@@ -26,6 +26,12 @@
 // a "run" whose blocks are stacked along N: per 128-row half and 16-wide K
 // step one tcgen05.mma of N = run * b (runs are split where a member is
 // written for the first time in the unit, since that MMA must overwrite).
+// For b = 32 an MMA costs about the same whatever its N, so every entry is
+// instead one run of all G members (N = 128): each member's block sits at
+// its own slot position, positions of absent members hold zeros, and the
+// unit's first entry overwrites the whole accumulator.  Shared memory is the
+// bound for b = 64: per entry the activation tile is written by TMA and read
+// by both halves' MMAs, the weight blocks written once and read twice.
 // A unit's accumulator is 2 x G*b = 256 fp32 columns of TMEM; two of them
 // let the epilogue of one unit overlap the MMAs of the next.
 //
