@@ -113,8 +113,8 @@ def test_module_matches_oracle_and_sees_in_place_updates():
     assert_parity(to_f64(Y2.reshape(M, N)), ref, S, "module Y after update")
 
 
-def test_repack_in_place_with_a_new_mask():
-    M, N, K, b, nnz = 300, 640, 448, 64, 30
+@pytest.mark.parametrize("M,N,K,b,nnz", [(300, 640, 448, 64, 30), (260, 768, 512, 32, 90)])
+def test_repack_in_place_with_a_new_mask(M, N, K, b, nnz):
     first = synth.random_case(M, N, K, b, nnz, 66)
     second = synth.random_case(M, N, K, b, nnz, 67)
     # same block count, different pattern: block rows 0 and 9 emptied, their
@@ -150,6 +150,8 @@ def test_repack_in_place_with_a_new_mask():
                                         128 // b)
     assert np.array_equal(Wp.rgrp_ptr.cpu().numpy(), gp)
     assert np.array_equal(Wp.rgrp_ent[:len(ent)].cpu().numpy(), ent)
+    U = torch.cuda.get_device_properties(X.device).multi_processor_count
+    assert np.array_equal(Wp.sbounds[:U + 2].cpu().numpy(), _plan.stream_bounds(want["row_ptr"], U))
     ref, S = oracle.forward(second["X"], second["W"], second["mask"], b)
     assert_parity(to_f64(Y), ref, S, "forward after repack")
     assert_parity(to_f64(Ys), ref[:20], S[:20], "stream forward after repack")

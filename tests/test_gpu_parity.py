@@ -194,15 +194,19 @@ LONG_ROW_CASES = [
 
 
 @pytest.mark.parametrize("case_args", LONG_ROW_CASES)
-def test_forward_stream_rows_across_many_ctas(case_args):
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_forward_stream_rows_across_many_ctas(case_args, with_bias):
     M, R, C, b, long_rows, per_row, seed = case_args
     case = long_row_case(M, R, C, b, long_rows, per_row, seed)
     Wp = pack_dev(case, b)
     check_pack(Wp, case, b)
-    got = to_f64(sg.forward_stream(to_dev(case["X"]), Wp))
+    bias = None
+    if with_bias:  # the last CTA on a shared row adds the bias once
+        bias = synth.bf16_bits(np.random.default_rng(seed + 500).standard_normal(R * b, dtype=np.float32))
+    got = to_f64(sg.forward_stream(to_dev(case["X"]), Wp, bias=None if bias is None else to_dev(bias)))
     assert sg.device_status(Wp) == 0
-    ref, S = oracle.forward(case["X"], case["W"], case["mask"], b)
-    assert_parity(got, ref, S, "forward_stream")
+    ref, S = oracle.forward(case["X"], case["W"], case["mask"], b, bias=bias)
+    assert_parity(got, ref, S, "forward_stream" + (" + bias" if with_bias else ""))
 
 
 def test_forward_stream_replayed_from_a_cuda_graph():
