@@ -90,7 +90,6 @@ typedef struct {
     int32_t *csc_to_bsr;  /* [nnz] BSR position of each CSC entry (values are not duplicated) */
     int32_t *row_order;   /* [R] block rows by block count, largest first, ties lower id first */
     int32_t *col_order;   /* [C] block columns, same order rule */
-    int32_t *dw_gptr;     /* [C+1] prefix over columns of ceil(col_count / (128/b)) (weight-gradient groups) */
     /* Work plan of the tensor-core forward: block rows taken G = 128/b at a
      * time in row_order ("row groups", ceil(R/G) of them).  For each group
      * the members' block columns are merged into one ascending list of

@@ -48,7 +48,7 @@ class _BSR(ctypes.Structure):
                 ("nnz", ctypes.c_int32)] + [
         (name, ctypes.c_void_p) for name in
         ("row_ptr", "col_idx", "values", "col_ptr", "row_idx", "csc_to_bsr", "row_order",
-         "col_order", "dw_gptr", "rgrp_ptr", "rgrp_bptr", "rgrp_ent", "rgrp_blk", "cgrp_ptr",
+         "col_order", "rgrp_ptr", "rgrp_bptr", "rgrp_ent", "rgrp_blk", "cgrp_ptr",
          "cgrp_bptr", "cgrp_ent", "cgrp_blk", "status", "sched", "sbounds")]
 
 # int32 entries of bsl_bsr.sbounds (BSL_SBOUNDS_LEN in include/bsl.h)
@@ -129,7 +129,6 @@ class BsrWeight:
         self.csc_to_bsr = torch.empty(max(nnz, 1), **i32)
         self.row_order = torch.empty(R, **i32)
         self.col_order = torch.empty(C, **i32)
-        self.dw_gptr = torch.empty(C + 1, **i32)
         G = 128 // b   # block rows (forward) / block columns (input gradient) per group
         nrg, ncg = (R + G - 1) // G, (C + G - 1) // G
         self.rgrp_ptr = torch.empty(nrg + 1, **i32)
@@ -146,7 +145,7 @@ class BsrWeight:
         self._c = _BSR(self.N, self.K, self.b, self.nnz,
                        *[t.data_ptr() for t in (self.row_ptr, self.col_idx, self.values, self.col_ptr,
                                                 self.row_idx, self.csc_to_bsr, self.row_order,
-                                                self.col_order, self.dw_gptr, self.rgrp_ptr,
+                                                self.col_order, self.rgrp_ptr,
                                                 self.rgrp_bptr, self.rgrp_ent, self.rgrp_blk,
                                                 self.cgrp_ptr, self.cgrp_bptr, self.cgrp_ent,
                                                 self.cgrp_blk, self.status, self.sched, self.sbounds)])

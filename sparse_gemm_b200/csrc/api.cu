@@ -90,7 +90,7 @@ bsl_status check_bsr(const bsl_bsr *W)
     const int64_t R = W->N / W->b, C = W->K / W->b;
     if (W->nnz > R * C) return BSL_ERR_INVALID_ARG;
     if (R >= (1 << 24) || C >= (1 << 24)) return BSL_ERR_UNSUPPORTED;  // plan entries hold 24-bit coordinates
-    const void *ptrs[] = {W->row_ptr, W->col_ptr, W->row_order, W->col_order, W->dw_gptr, W->rgrp_ptr,
+    const void *ptrs[] = {W->row_ptr, W->col_ptr, W->row_order, W->col_order, W->rgrp_ptr,
                           W->rgrp_bptr, W->cgrp_ptr, W->cgrp_bptr, W->status, W->sched, W->sbounds};
     for (const void *p : ptrs)
         if (!p || !aligned(p, 4)) return BSL_ERR_INVALID_ARG;

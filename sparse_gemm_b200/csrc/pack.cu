@@ -10,7 +10,7 @@
 //
 // Kernels, in launch order:
 //   k_counts     one warp per block row / block column: popcount of the mask
-//   k_scan       one CTA: exclusive scans -> row_ptr, col_ptr, dw_gptr; nnz check
+//   k_scan       one CTA: exclusive scans -> row_ptr, col_ptr; nnz check
 //   k_fill_rows  one warp per block row: col_idx (ascending) by ballot prefix
 //   k_fill_cols  one warp per block column: row_idx, csc_to_bsr
 //   k_gather     16-byte vector copy of every kept block into `values`
@@ -81,43 +81,30 @@ __device__ int block_scan_incl(int v, int *sm)
 }
 
 // In-place: ptr[1..n] holds counts; turns ptr[0..n] into the exclusive prefix.
-// If `groups` is set, also writes groups[0..n] = prefix of ceil(count/G).
-__device__ void scan_counts(int32_t *ptr, int32_t n, int32_t *groups, int G, int *sm)
+__device__ void scan_counts(int32_t *ptr, int32_t n, int *sm)
 {
-    int carry = 0, gcarry = 0;
-    if (threadIdx.x == 0) {
-        ptr[0] = 0;
-        if (groups) groups[0] = 0;
-    }
+    int carry = 0;
+    if (threadIdx.x == 0) ptr[0] = 0;
     for (int base = 0; base < n; base += blockDim.x) {
         const int i = base + threadIdx.x;
         const int cnt = i < n ? ptr[i + 1] : 0;
         const int incl = block_scan_incl(cnt, sm) + carry;
-        int gincl = 0;
-        if (groups) gincl = block_scan_incl((cnt + G - 1) / G, sm) + gcarry;
-        if (i < n) {
-            ptr[i + 1] = incl;
-            if (groups) groups[i + 1] = gincl;
-        }
-        // the last thread of the chunk holds the running totals
-        __shared__ int tot[2];
-        if (threadIdx.x == blockDim.x - 1) {
-            tot[0] = incl;
-            tot[1] = gincl;
-        }
+        if (i < n) ptr[i + 1] = incl;
+        // the last thread of the chunk holds the running total
+        __shared__ int tot;
+        if (threadIdx.x == blockDim.x - 1) tot = incl;
         __syncthreads();
-        carry = tot[0];
-        gcarry = tot[1];
+        carry = tot;
         __syncthreads();
     }
 }
 
 __global__ void __launch_bounds__(1024) k_scan(int32_t *row_ptr, int32_t R, int32_t *col_ptr, int32_t C,
-                                               int32_t *dw_gptr, int G, int32_t nnz, int32_t *status)
+                                               int32_t nnz, int32_t *status)
 {
     __shared__ int sm[32];
-    scan_counts(row_ptr, R, nullptr, 1, sm);
-    if (col_ptr) scan_counts(col_ptr, C, dw_gptr, G, sm);
+    scan_counts(row_ptr, R, sm);
+    if (col_ptr) scan_counts(col_ptr, C, sm);
     if (threadIdx.x == 0 && status && nnz >= 0 && row_ptr[R] != nnz) set_status(status, BSL_ERR_NNZ_MISMATCH);
 }
 
@@ -272,10 +259,10 @@ __global__ void __launch_bounds__(1024) k_scan_groups(int32_t *a, int32_t na, in
                                                       int32_t *c, int32_t nc, int32_t *d, int32_t nd)
 {
     __shared__ int sm[32];
-    scan_counts(a, na, nullptr, 1, sm);
-    scan_counts(b, nb_, nullptr, 1, sm);
-    scan_counts(c, nc, nullptr, 1, sm);
-    scan_counts(d, nd, nullptr, 1, sm);
+    scan_counts(a, na, sm);
+    scan_counts(b, nb_, sm);
+    scan_counts(c, nc, sm);
+    scan_counts(d, nd, sm);
 }
 
 template <int G>
@@ -336,14 +323,13 @@ __global__ void k_stream_bounds(const int32_t *__restrict__ row_ptr, int32_t R, 
 bsl_status launch_pack_count(const uint8_t *mask, int32_t R, int32_t C, int32_t *row_ptr, cudaStream_t s)
 {
     k_counts<<<(R + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, row_ptr, nullptr);
-    k_scan<<<1, 1024, 0, s>>>(row_ptr, R, nullptr, 0, nullptr, 1, -1, nullptr);
+    k_scan<<<1, 1024, 0, s>>>(row_ptr, R, nullptr, 0, -1, nullptr);
     return cuda_status(cudaGetLastError());
 }
 
 bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cudaStream_t s)
 {
     const int32_t R = o->N / o->b, C = o->K / o->b, nnz = o->nnz;
-    const int G = 128 / o->b;
     // index arrays start as valid indices (0) even if the mask disagrees with nnz
     if (nnz > 0) {
         cudaMemsetAsync(o->col_idx, 0, sizeof(int32_t) * nnz, s);
@@ -351,7 +337,7 @@ bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cud
         cudaMemsetAsync(o->csc_to_bsr, 0, sizeof(int32_t) * nnz, s);
     }
     k_counts<<<(R + C + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, o->row_ptr, o->col_ptr);
-    k_scan<<<1, 1024, 0, s>>>(o->row_ptr, R, o->col_ptr, C, o->dw_gptr, G, nnz, o->status);
+    k_scan<<<1, 1024, 0, s>>>(o->row_ptr, R, o->col_ptr, C, nnz, o->status);
     k_fill_rows<<<(R + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, o->row_ptr, o->col_idx, nnz);
     k_fill_cols<<<(C + kWarps - 1) / kWarps, kWarps * 32, 0, s>>>(mask, R, C, o->row_ptr, o->col_idx,
                                                                   o->col_ptr, o->row_idx, o->csc_to_bsr, nnz);

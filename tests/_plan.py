@@ -51,18 +51,6 @@ def group_plan(ptr, idx, order, G: int, blk=None):
     return i32(grp_ptr), i32(grp_bptr), i32(ent), i32(blk_list)
 
 
-def dw_group_ptr(col_ptr, group: int) -> np.ndarray:
-    """Start of each block column's weight-gradient groups: the column's
-    blocks are cut into consecutive runs of ``group`` (the last run may be
-    shorter) and the runs are numbered column after column."""
-    col_ptr = [int(v) for v in col_ptr]
-    out = [0]
-    for c in range(len(col_ptr) - 1):
-        n = col_ptr[c + 1] - col_ptr[c]
-        out.append(out[-1] + (n + group - 1) // group)
-    return np.asarray(out, dtype=np.int32)
-
-
 def stream_bounds(row_ptr, U: int) -> np.ndarray:
     """CTA ranges of the weight-streaming forward, ``[U, b_0, ..., b_U]``.
 

@@ -43,30 +43,6 @@ def test_group_plan_covers_every_block_once(oracle_lib):
     assert sorted(blk.tolist()) == list(range(pk["nnz"]))
 
 
-def test_dw_group_ptr_by_walking_the_columns():
-    """Walk the mask column by column, opening a new group at the first
-    block of a column and after every `group` blocks; the group index at
-    which each column starts must be what dw_group_ptr gives."""
-    rng = np.random.default_rng(17)
-    for group in (1, 2, 4):
-        mask = (rng.random((23, 9)) < 0.45).astype(np.uint8)
-        mask[:, 3] = 0            # an empty column
-        mask[:, 5] = 1            # a full column (23 blocks: not a multiple of 2 or 4)
-        starts, ngroups = [], 0
-        for c in range(mask.shape[1]):
-            starts.append(ngroups)
-            in_group = group      # forces a new group at the column's first block
-            for r in range(mask.shape[0]):
-                if mask[r, c]:
-                    if in_group == group:
-                        ngroups += 1
-                        in_group = 0
-                    in_group += 1
-        starts.append(ngroups)
-        col_ptr = np.concatenate([[0], np.cumsum(mask.sum(0))])
-        assert np.array_equal(_plan.dw_group_ptr(col_ptr, group), np.array(starts)), group
-
-
 @pytest.mark.parametrize("R,C,nnz,U,seed", [
     (344, 128, 11008, 148, 1),   # the decode weight's shape and density
     (224, 64, 1434, 148, 2),
