@@ -69,7 +69,10 @@ bsl_status check_device()
 
 // Make the device that owns `p` current for this host thread (this also
 // binds its primary context, which a fresh thread may not have yet), and
-// reject pointers that are not device memory.
+// reject pointers that are not device memory.  The call is made even when the
+// runtime already reports that device: on a thread that has made no runtime
+// call yet (PyTorch's autograd thread, for one) no context is bound, and the
+// driver-level tensor-map encoding would then fail.
 bsl_status bind_device(const void *p)
 {
     cudaPointerAttributes a;
