@@ -16,11 +16,11 @@
 // Each warp streams its share through its own ring of slots; a slot holds one
 // weight block and the activation slice X[0:MP, c*b:(c+1)*b] it multiplies,
 // both brought in by TMA (swizzled rows, rows past M read as zeros).  The
-// weight copies, which depend on nothing, leave first; a ring usually holds
-// the warp's whole share.  The operands go to registers with ldmatrix;
-// mma.sync m16n8k16 (bf16 in, fp32 accumulate) forms
-// Y^T[n][m] = W_blk[n][:] . X[m][:], and the sum of the current block row
-// stays in registers:
+// weight copies, which depend on nothing, leave first; each slot is refilled
+// as soon as it is read, with a few slots per warp (enough to keep DRAM
+// busy).  The operands go to registers with ldmatrix; mma.sync m16n8k16
+// (bf16 in, fp32 accumulate) forms Y^T[n][m] = W_blk[n][:] . X[m][:], and
+// the sum of the current block row stays in registers:
 //   - a block row entirely inside the warp's share is finished there: bias
 //     added, rounded to bf16, staged in shared memory, written to Y with
 //     16-byte stores;
@@ -44,7 +44,11 @@ namespace bsl {
 namespace {
 
 constexpr int kStreamWarps = 8;
-constexpr int kWarpSmem = 24 * 1024;  // ring bytes per warp
+// Copy bytes a warp keeps in flight, at most (two slots at least): 96 KB per
+// SM already covers the DRAM bandwidth-delay product (~6.5 TB/s x ~2 us over
+// 148 SMs); more only queues in the memory system and takes shared memory
+// from L1 (decode forward, 3 KB slots: 8 per warp 12.7 us, 4 per warp 11.0 us).
+constexpr int kWarpInFlight = 12 * 1024;
 
 template <int B, int MP>
 struct StreamCfg {
@@ -52,7 +56,7 @@ struct StreamCfg {
     static constexpr int W_BLK = B * ROW_BYTES;        // one weight block
     static constexpr int X_BLK = MP * ROW_BYTES;       // its activation slice (MP x b)
     static constexpr int SLOT = W_BLK + X_BLK;
-    static constexpr int NSLOT = kWarpSmem / SLOT;
+    static constexpr int NSLOT = kWarpInFlight / SLOT > 2 ? kWarpInFlight / SLOT : 2;
     static constexpr int WARP_BYTES = NSLOT * SLOT;
     static constexpr int OUT_BYTES = MP * ROW_BYTES;   // per-warp bf16 staging of one block row
     static constexpr int PART = B * MP;                // floats of one partial
