@@ -52,7 +52,7 @@ TRAFFIC = {
     ("large_fwd", "fwd"): {"bytes": 287450112, "src_sha": "e4c02bbc81127eb7",
                            "files": ["spmm_tc.cu", "common.cuh"],
                            "profile": "profiles/k_spmm_tc_fwd_large_fwd.md"},
-    ("decode_fwd", "fwd"): {"bytes": 22775040, "src_sha": "0ed3ad13b8d1c89e",
+    ("decode_fwd", "fwd"): {"bytes": 22774528, "src_sha": "ea9cb22b798b0cf0",
                             "files": ["stream_fwd.cu", "common.cuh"],
                             "profile": "profiles/k_stream_fwd_decode_fwd.md"},
     ("enc_train_d1.0", "dx"): {"bytes": 29975296, "src_sha": "e4c02bbc81127eb7",
