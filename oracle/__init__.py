@@ -19,6 +19,13 @@ Sources it restates (page title + section):
 * torchao sparsity README, "Pruning Criteria", out-of-place mask updates:
   the masked weight gradient is dW (.) Mask -> :func:`backward_weight`
   evaluates dW = dY^T X at the mask's blocks only.
+* torchao sparsity README, Table 4.1, row "NVIDIA 2:4 compressed
+  representation" (with the 2:4 semi-structured pattern of the README's
+  introduction and of the "Lecture 11: Sparsity" summary, 8:02 and 12:52: two
+  of every four consecutive elements are zero): the weight kept as a dense
+  matrix of half the width holding the unpruned elements plus 2-bit indices
+  -> :func:`compress24` / :func:`decompress24`; its product is the dense
+  product with the weight it came from -> :func:`semi24_forward`.
 
 The contractions run in ``bsl_oracle.c`` (plain loops, OpenMP over output
 rows/blocks).  The pack and the schedule order are plain Python loops.
@@ -251,3 +258,78 @@ def schedule_order(ptr) -> np.ndarray:
     ptr = [int(v) for v in ptr]
     counts = [ptr[i + 1] - ptr[i] for i in range(len(ptr) - 1)]
     return np.asarray(sorted(range(len(counts)), key=lambda i: (-counts[i], i)), dtype=np.int32)
+
+
+# ---------------------------------------------------------------- 2:4 semi-structured
+
+_SEMI24_CODES = (0x4, 0x8, 0xC, 0x9, 0xD, 0xE)  # i0 | i1 << 2 for the six pairs i0 < i1
+
+
+def compress24(W):
+    """NVIDIA 2:4 compressed representation of a dense weight with zeros in
+    place (torchao sparsity README, Table 4.1, row "NVIDIA 2:4 compressed
+    representation": a compressed dense matrix of half the size holding the
+    unpruned elements, plus 2-bit indices).
+
+    ``W``: bf16 bits (uint16) [N, K], K a multiple of 16.  Every group of four
+    consecutive elements of a row (columns 4g .. 4g+3) may hold at most two
+    nonzeros; +0 and -0 both count as zero.  Returns ``(values, meta)``:
+
+    * ``values`` uint16 [N, K/2]: group g's two kept elements at columns
+      2g and 2g+1, in index order, copied bit for bit;
+    * ``meta`` uint16 [N, K/16]: entry (n, c) holds the kept positions of
+      groups 4c .. 4c+3 of row n, group 4c+j in bits 4j .. 4j+3 as
+      i0 | i1 << 2 (positions inside the group, i0 < i1).
+
+    The kept positions are the nonzero ones; when a group has fewer than two
+    nonzeros the lowest-indexed zeros complete the pair.  Raises ValueError
+    when a group holds more than two nonzeros.
+    """
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    N, K = W.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    v = W.reshape(N, K // 4, 4)
+    nz = (v & 0x7FFF) != 0
+    cnt = nz.sum(axis=2)
+    if (cnt > 2).any():
+        n, g = np.argwhere(cnt > 2)[0]
+        raise ValueError(f"row {n}, group {g} holds {cnt[n, g]} nonzeros: not 2:4")
+    need = 2 - cnt                                   # zeros that complete the pair
+    zero = ~nz
+    zeros_before = np.cumsum(zero, axis=2) - zero    # zeros at lower positions of the group
+    kept = nz | (zero & (zeros_before < need[:, :, None]))
+    pos = np.nonzero(kept)[2].reshape(N, K // 4, 2)  # two kept positions per group, ascending
+    values = np.take_along_axis(v, pos, axis=2).reshape(N, K // 2)
+    code = (pos[:, :, 0] | (pos[:, :, 1] << 2)).astype(np.uint16).reshape(N, K // 16, 4)
+    meta = code[:, :, 0] | (code[:, :, 1] << 4) | (code[:, :, 2] << 8) | (code[:, :, 3] << 12)
+    return values.astype(np.uint16), meta.astype(np.uint16)
+
+
+def decompress24(values, meta):
+    """Dense bf16 bits [N, K] from the compressed form of :func:`compress24`:
+    each kept element back at its position, zeros (+0) elsewhere."""
+    values = np.ascontiguousarray(values, dtype=np.uint16)
+    meta = np.ascontiguousarray(meta, dtype=np.uint16)
+    N, half = values.shape
+    K = 2 * half
+    if meta.shape != (N, K // 16):
+        raise ValueError("meta must be [N, K/16]")
+    code = np.stack([(meta >> (4 * j)) & 0xF for j in range(4)], axis=2).reshape(N, K // 4)
+    i0, i1 = code & 3, code >> 2
+    if ((i0 >= i1)).any():
+        raise ValueError("meta holds a pair that is not ascending")
+    out = np.zeros((N, K // 4, 4), dtype=np.uint16)
+    pair = values.reshape(N, K // 4, 2)
+    np.put_along_axis(out, i0[:, :, None].astype(np.int64), pair[:, :, :1], axis=2)
+    np.put_along_axis(out, i1[:, :, None].astype(np.int64), pair[:, :, 1:], axis=2)
+    return out.reshape(N, K)
+
+
+def semi24_forward(X, values, meta, rows=None, *, Xd=None, bias=None):
+    """Y[rows] = X[rows] W^T (+ bias) in fp64 with W the dense weight that
+    the compressed form stands for: the sparse product is the dense product
+    with zeros in place (torchao sparsity README, introduction).  Returns
+    (Y, Yabs) like :func:`forward`."""
+    Wt = widen(decompress24(values, meta))
+    return forward(X, None, None, None, rows, Xd=Xd, Wt=Wt, bias=bias)

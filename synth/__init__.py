@@ -26,6 +26,7 @@ import torch
 __all__ = [
     "Workload", "WORKLOADS", "bf16_bits", "bits_to_f32", "mask_uniform",
     "zipf_row_counts", "mask_zipf_rows", "make_inputs", "round_half_even",
+    "semi24_weight", "Semi24Workload", "SEMI24_WORKLOADS", "make_semi24_inputs",
 ]
 
 
@@ -222,4 +223,73 @@ def random_case(M: int, N: int, K: int, b: int, nnz: int, seed: int, *,
         "W": draw((N, K), 1.0 / math.sqrt(K)),
         "dY": draw((M, N), 1.0),
         "mask": mask,
+    }
+
+
+# ---------------------------------------------------------------- 2:4 semi-structured weights
+
+_PAIRS = ((0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3))
+
+
+def semi24_weight(N: int, K: int, rng: np.random.Generator, *, std: float = 1.0,
+                  fewer: float = 0.0, integer_values: bool = False) -> np.ndarray:
+    """Dense bf16 weight [N, K] (bit patterns) with zeros in place, at most
+    two nonzeros in every group of four consecutive elements of a row: the
+    2:4 semi-structured pattern.  Each group's two unpruned positions are one
+    of the six pairs, uniformly; the other two are +0.  With ``fewer`` > 0
+    each unpruned value is replaced, with that probability, by +0 or -0 (half
+    each), so groups with one or no nonzero and signed zeros appear.  Values
+    are normal(0, std) rounded to bf16, or integers in {-3..3} without 0 with
+    ``integer_values``."""
+    if K % 4:
+        raise ValueError("K must be a multiple of 4")
+    G = N * (K // 4)
+    pick = rng.integers(0, 6, size=G)
+    pairs = np.asarray(_PAIRS, dtype=np.int64)[pick]          # [G, 2]
+    if integer_values:
+        mag = rng.integers(1, 4, size=(G, 2)).astype(np.float32)
+        val = bf16_bits(mag * np.where(rng.random((G, 2)) < 0.5, -1.0, 1.0).astype(np.float32))
+    else:
+        val = _normal_bf16(rng, (G, 2), std)
+    if fewer > 0:
+        drop = rng.random((G, 2)) < fewer
+        signed = rng.random((G, 2)) < 0.5
+        val = np.where(drop, np.where(signed, np.uint16(0x8000), np.uint16(0)), val).astype(np.uint16)
+    out = np.zeros((G, 4), dtype=np.uint16)
+    rows = np.arange(G)
+    out[rows, pairs[:, 0]] = val[:, 0]
+    out[rows, pairs[:, 1]] = val[:, 1]
+    return out.reshape(N, K)
+
+
+@dataclasses.dataclass(frozen=True)
+class Semi24Workload:
+    """A linear layer whose weight has the 2:4 semi-structured pattern."""
+    name: str
+    M: int
+    N: int
+    K: int
+    seed: int
+    description: str = ""
+
+    def flops(self) -> int:
+        """Algorithmic flops of the forward: 2*M*N*(K/2), the products with
+        the unpruned half of the weight."""
+        return self.M * self.N * self.K
+
+
+SEMI24_WORKLOADS: dict[str, Semi24Workload] = {w.name: w for w in [
+    Semi24Workload("semi24_fwd", 8192, 14336, 4096, 6,
+                   description="LLM-MLP forward, X[8192,4096], W[14336,4096] 2:4 semi-structured"),
+]}
+
+
+def make_semi24_inputs(w: Semi24Workload, *, M: int | None = None):
+    """Seeded X [M,K] and 2:4 weight W [N,K] (bf16 bits) of a 2:4 workload.
+    Sub-streams as for the block-sparse workloads: 0 for X, 2 for W."""
+    M = w.M if M is None else M
+    return {
+        "X": _normal_bf16(np.random.default_rng(w.seed * 10 + 0), (M, w.K), 1.0),
+        "W": semi24_weight(w.N, w.K, np.random.default_rng(w.seed * 10 + 2),
+                           std=1.0 / math.sqrt(w.K / 2)),
     }

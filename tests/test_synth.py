@@ -44,3 +44,25 @@ def test_inputs_are_seeded_and_shaped():
     assert abs(Wf.std() - 1 / 16) < 0.01
     t = torch.from_numpy(a["X"].view(np.int16)).view(torch.bfloat16).float().numpy()
     assert np.array_equal(t, synth.bits_to_f32(a["X"]))
+
+
+def test_semi24_weight_has_at_most_two_nonzeros_per_group():
+    rng = np.random.default_rng(0)
+    W = synth.semi24_weight(64, 256, rng)
+    nz = ((W & 0x7FFF) != 0).reshape(64, 64, 4).sum(axis=2)
+    assert (nz == 2).all()  # no normal draw of std 1 rounds to zero in bf16 here
+    Wf = synth.semi24_weight(64, 256, np.random.default_rng(0), fewer=0.5)
+    nzf = ((Wf & 0x7FFF) != 0).reshape(64, 64, 4).sum(axis=2)
+    assert nzf.max() <= 2 and (nzf == 0).any() and (nzf == 1).any()
+    assert (Wf == 0x8000).any()  # signed zeros appear
+    assert np.array_equal(synth.semi24_weight(8, 16, np.random.default_rng(3)),
+                          synth.semi24_weight(8, 16, np.random.default_rng(3)))
+
+
+def test_semi24_workload_inputs_are_seeded():
+    w = synth.SEMI24_WORKLOADS["semi24_fwd"]
+    a = synth.make_semi24_inputs(w, M=4)
+    b = synth.make_semi24_inputs(w, M=4)
+    assert a["X"].shape == (4, w.K) and a["W"].shape == (w.N, w.K)
+    assert np.array_equal(a["W"], b["W"]) and np.array_equal(a["X"], b["X"])
+    assert w.flops() == 2 * w.M * w.N * (w.K // 2)
