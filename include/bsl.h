@@ -66,8 +66,10 @@ typedef enum {
     BSL_ERR_TIMEOUT = 4,       /* a device-side wait ran out of time (device status) */
     BSL_ERR_NNZ_MISMATCH = 5,  /* mask block count != bsl_bsr.nnz (device status) */
     BSL_ERR_NO_DEVICE = 6,     /* no sm_100 device current */
-    BSL_ERR_SCRATCH_TOO_SMALL = 7  /* bsl_forward_stream_noalloc: the call needs more
+    BSL_ERR_SCRATCH_TOO_SMALL = 7, /* bsl_forward_stream_noalloc: the call needs more
                                       scratch than BSL_NOALLOC_SCRATCH_BYTES */
+    BSL_ERR_NOT_2_4 = 8            /* bsl_semi24_compress: a group of four holds more than
+                                      two nonzeros (device status) */
 } bsl_status;
 
 /* Bytes of device memory that libbsl keeps, on every GPU that loads it, as
@@ -228,6 +230,48 @@ BSL_API bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M,
  * be a multiple of 32; dbias is bf16 [N], 16-byte aligned.  Needs no
  * scratch. */
 BSL_API bsl_status bsl_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, void *stream);
+
+/* ---------------------------------------------------------------- 2:4 semi-structured
+ *
+ * A linear layer whose weight has the 2:4 semi-structured pattern: in every
+ * group of four consecutive elements of a row (along K) at most two are
+ * nonzero (torchao sparsity README, introduction and Table 4.1; "Lecture 11:
+ * Sparsity" summary, 8:02 and 12:52).  The weight is stored in the
+ * compressed form of Table 4.1, row "NVIDIA 2:4 compressed representation":
+ * a dense matrix of half the width holding the unpruned elements, plus
+ * 2-bit indices.  Y = X . W^T runs on the sparse tensor-core MMA. */
+typedef struct {
+    int32_t N, K;       /* dense shape of W: N output features, K input features;
+                         * N a multiple of 8, K a multiple of 64 */
+    void *values;       /* bf16 [N][K/2]: group g of row n (columns 4g .. 4g+3) keeps two
+                         * elements, at values[n][2g] and values[n][2g+1], in column order */
+    uint16_t *meta;     /* [N][K/16]: positions of the kept elements; entry (n, c) covers
+                         * groups 4c .. 4c+3 of row n, group 4c+j in bits 4j .. 4j+3 as
+                         * i0 | i1 << 2, the two positions inside the group with i0 < i1 */
+    int32_t *status;    /* [1] device status word; must be zeroed once at allocation */
+} bsl_semi24;
+
+/* Compress a dense bf16 weight W [N][K] with zeros in place (the handoff
+ * format of the torchao README's introduction) into out->values / out->meta
+ * (caller-allocated, 16-byte aligned).  The kept positions of a group are
+ * its nonzeros (+0 and -0 count as zero), completed by its lowest-indexed
+ * zeros when it has fewer than two; kept elements are copied bit for bit.
+ * A group with more than two nonzeros sets BSL_ERR_NOT_2_4 in the device
+ * status (its outputs are then unspecified); read it with
+ * bsl_semi24_get_status. */
+BSL_API bsl_status bsl_semi24_compress(const void *W, const bsl_semi24 *out, void *stream);
+
+/* Y [M][N] = X [M][K] . W^T (+ bias) with W the weight the compressed form
+ * stands for, in bf16 with fp32 accumulation (the sparse product is the
+ * dense product with zeros in place: torchao README, introduction).  bias is
+ * bf16 [N] added in fp32 before the one rounding to bf16, or NULL.  M >= 1.
+ * Tensor-core kernel (tcgen05.mma.sp), persistent, one CTA per SM. */
+BSL_API bsl_status bsl_semi24_forward(const void *X, int32_t M, const bsl_semi24 *W, const void *bias, void *Y,
+                                      void *stream);
+
+/* SYNCHRONOUS: waits for the stream, copies the device status word of W to
+ * *status_host (a bsl_status value) and resets it to BSL_OK. */
+BSL_API bsl_status bsl_semi24_get_status(const bsl_semi24 *W, int32_t *status_host, void *stream);
 
 /* SYNCHRONOUS: waits for the stream, copies the device status word of W to
  * *status_host (a bsl_status value) and resets it to BSL_OK. */

@@ -25,6 +25,7 @@ __all__ = [
     "device_status", "set_wait_timeout_us", "debug_wait_timeout", "small_m_max",
     "forward_stream_noalloc", "bias_grad",
     "BlockSparseLinearFunction", "BlockSparseLinear",
+    "Semi24Weight", "compress24", "forward24", "semi24_status",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +34,7 @@ LIB_PATH = os.path.join(_HERE, "libbsl.so")
 STATUS_NAMES = {
     0: "BSL_OK", 1: "BSL_ERR_INVALID_ARG", 2: "BSL_ERR_UNSUPPORTED", 3: "BSL_ERR_CUDA",
     4: "BSL_ERR_TIMEOUT", 5: "BSL_ERR_NNZ_MISMATCH", 6: "BSL_ERR_NO_DEVICE",
-    7: "BSL_ERR_SCRATCH_TOO_SMALL",
+    7: "BSL_ERR_SCRATCH_TOO_SMALL", 8: "BSL_ERR_NOT_2_4",
 }
 
 
@@ -51,6 +52,11 @@ class _BSR(ctypes.Structure):
          "col_order", "rgrp_ptr", "rgrp_bptr", "rgrp_ent", "rgrp_blk", "cgrp_ptr",
          "cgrp_bptr", "cgrp_ent", "cgrp_blk", "status", "sched", "sbounds")]
 
+class _SEMI24(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("values", ctypes.c_void_p),
+                ("meta", ctypes.c_void_p), ("status", ctypes.c_void_p)]
+
+
 # int32 entries of bsl_bsr.sbounds (BSL_SBOUNDS_LEN in include/bsl.h)
 SBOUNDS_LEN = 1026
 
@@ -67,6 +73,7 @@ def library() -> ctypes.CDLL:
         lib = ctypes.CDLL(LIB_PATH)
         P, I32, SZ, U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64
         BP = ctypes.POINTER(_BSR)
+        SP = ctypes.POINTER(_SEMI24)
         sig = {
             "bsl_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "bsl_last_cuda_error": (ctypes.c_char_p, []),
@@ -84,6 +91,9 @@ def library() -> ctypes.CDLL:
             "bsl_set_wait_timeout_us": (None, [U64]),
             "bsl_debug_wait_timeout": (ctypes.c_int, [P, U64, P]),
             "bsl_forward_stream_noalloc": (ctypes.c_int, [P, I32, BP, P, P]),
+            "bsl_semi24_compress": (ctypes.c_int, [P, SP, P]),
+            "bsl_semi24_forward": (ctypes.c_int, [P, I32, SP, P, P, P]),
+            "bsl_semi24_get_status": (ctypes.c_int, [SP, ctypes.POINTER(I32), P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -422,3 +432,64 @@ class BlockSparseLinear(torch.nn.Module):
     def extra_repr(self) -> str:
         return (f"in_features={self.in_features}, out_features={self.out_features}, "
                 f"block={self.packed.b}, nnz_blocks={self.packed.nnz}, bias={self.bias is not None}")
+
+
+# ---------------------------------------------------------------- 2:4 semi-structured
+
+
+class Semi24Weight:
+    """A weight with the 2:4 semi-structured pattern in its compressed form
+    (torchao sparsity README, Table 4.1, "NVIDIA 2:4 compressed
+    representation"): ``values`` bf16 [N, K/2], the two kept elements of every
+    group of four, and ``meta`` [N, K/16] (16-bit words held in an int16
+    tensor), their 2-bit positions; layout in include/bsl.h (bsl_semi24)."""
+
+    def __init__(self, N: int, K: int, device):
+        if N <= 0 or K <= 0 or N % 8 or K % 64:
+            raise ValueError("N must be a positive multiple of 8 and K of 64")
+        self.N, self.K = int(N), int(K)
+        self.values = torch.empty((N, K // 2), dtype=torch.bfloat16, device=device)
+        self.meta = torch.empty((N, K // 16), dtype=torch.int16, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self._c = _SEMI24(self.N, self.K, self.values.data_ptr(), self.meta.data_ptr(),
+                          self.status.data_ptr())
+
+    @property
+    def device(self):
+        return self.values.device
+
+    def cref(self):
+        return ctypes.byref(self._c)
+
+
+def compress24(W: torch.Tensor, out: Semi24Weight | None = None) -> Semi24Weight:
+    """Compress a dense bf16 weight [N, K] with zeros in place and at most two
+    nonzeros per group of four along K.  A group with more nonzeros is
+    reported by :func:`semi24_status` (BSL_ERR_NOT_2_4)."""
+    _cuda_bf16_2d(W, "W")
+    N, K = W.shape
+    w = Semi24Weight(N, K, W.device) if out is None else out
+    if (w.N, w.K) != (N, K):
+        raise ValueError(f"out holds a [{w.N}, {w.K}] weight, W is [{N}, {K}]")
+    _check(library().bsl_semi24_compress(W.data_ptr(), w.cref(), _stream(W)), "bsl_semi24_compress")
+    return w
+
+
+def forward24(X: torch.Tensor, w: Semi24Weight, bias: torch.Tensor | None = None,
+              out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T (+ bias) on the sparse tensor-core kernel."""
+    _cuda_bf16_2d(X, "X", w.K)
+    bptr = _bias_ptr(bias, w.N, X)
+    M = X.shape[0]
+    Y = _out(M, w.N, X) if out is None else out
+    _check(library().bsl_semi24_forward(X.data_ptr(), M, w.cref(), bptr, Y.data_ptr(), _stream(X)),
+           "bsl_semi24_forward")
+    return Y
+
+
+def semi24_status(w: Semi24Weight) -> int:
+    """Read and clear the weight's device status word (synchronises the stream)."""
+    out = ctypes.c_int32(0)
+    _check(library().bsl_semi24_get_status(w.cref(), ctypes.byref(out), _stream(w.values)),
+           "bsl_semi24_get_status")
+    return int(out.value)

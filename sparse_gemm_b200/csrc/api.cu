@@ -107,6 +107,16 @@ bsl_status check_bsr(const bsl_bsr *W)
     return BSL_OK;
 }
 
+bsl_status check_semi24(const bsl_semi24 *W)
+{
+    if (!W) return BSL_ERR_INVALID_ARG;
+    if (W->N <= 0 || W->K <= 0 || W->N % 8 || W->K % 64) return BSL_ERR_INVALID_ARG;
+    if (!W->values || !aligned(W->values, 16) || !W->meta || !aligned(W->meta, 16) || !W->status ||
+        !aligned(W->status, 4))
+        return BSL_ERR_INVALID_ARG;
+    return BSL_OK;
+}
+
 namespace {
 thread_local int g_last_cuda_error = 0;  // last CUDA error seen by this host thread
 }
@@ -245,6 +255,7 @@ const char *bsl_status_string(bsl_status s)
     case BSL_ERR_NNZ_MISMATCH: return "BSL_ERR_NNZ_MISMATCH";
     case BSL_ERR_NO_DEVICE: return "BSL_ERR_NO_DEVICE";
     case BSL_ERR_SCRATCH_TOO_SMALL: return "BSL_ERR_SCRATCH_TOO_SMALL";
+    case BSL_ERR_NOT_2_4: return "BSL_ERR_NOT_2_4";
     }
     return "BSL_ERR_UNKNOWN";
 }
@@ -359,6 +370,39 @@ bsl_status bsl_backward_weight(const void *dY, const void *X, int32_t M, const b
 }
 
 bsl_status bsl_get_device_status(const bsl_bsr *W, int32_t *status_host, void *stream)
+{
+    if (!W || !W->status || !status_host) return BSL_ERR_INVALID_ARG;
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(W->status));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    BSL_TRY(cuda_status(cudaMemcpyAsync(status_host, W->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s)));
+    BSL_TRY(cuda_status(cudaMemsetAsync(W->status, 0, sizeof(int32_t), s)));
+    return cuda_status(cudaStreamSynchronize(s));
+}
+
+bsl_status bsl_semi24_compress(const void *W, const bsl_semi24 *out, void *stream)
+{
+    BSL_TRY(check_semi24(out));
+    if (check_matrix(W, out->N) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(W));
+    BSL_TRY(check_device());
+    return launch_compress24(W, out, static_cast<cudaStream_t>(stream));
+}
+
+bsl_status bsl_semi24_forward(const void *X, int32_t M, const bsl_semi24 *W, const void *bias, void *Y,
+                              void *stream)
+{
+    BSL_TRY(check_semi24(W));
+    if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 16)) return BSL_ERR_INVALID_ARG;
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(X));
+    BSL_TRY(check_device());
+    return launch_semi24_fwd(X, M, W, bias, Y, static_cast<cudaStream_t>(stream));
+}
+
+bsl_status bsl_semi24_get_status(const bsl_semi24 *W, int32_t *status_host, void *stream)
 {
     if (!W || !W->status || !status_host) return BSL_ERR_INVALID_ARG;
     DeviceGuard guard;

@@ -48,6 +48,7 @@ private:
 bsl_status set_smem_once(const void *func, int bytes);
 bsl_status check_device();              // current device is sm_100
 bsl_status check_bsr(const bsl_bsr *W);
+bsl_status check_semi24(const bsl_semi24 *W);
 uint64_t wait_timeout_ns();
 bsl_status cuda_status(cudaError_t e);
 void note_driver_error(int code);
@@ -69,6 +70,11 @@ size_t stream_workspace_bytes(int32_t M, const bsl_bsr *W);
 bsl_status launch_stream_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *bias, void *Y, void *ws,
                              cudaStream_t s);
 bsl_status launch_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, cudaStream_t s);
+
+// 2:4 semi-structured weight: compress a dense weight, forward on the sparse MMA.
+bsl_status launch_compress24(const void *W, const bsl_semi24 *out, cudaStream_t s);
+bsl_status launch_semi24_fwd(const void *X, int32_t M, const bsl_semi24 *W, const void *bias, void *Y,
+                             cudaStream_t s);
 
 bsl_status launch_debug_wait(int32_t *status, uint64_t timeout_ns, cudaStream_t s);
 

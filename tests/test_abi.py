@@ -86,3 +86,41 @@ def test_binding_struct_matches_the_header():
     assert [n for n, _ in sg._BSR._fields_] == names
     m = re.search(r"#define BSL_SBOUNDS_LEN (\d+)", text)
     assert m and int(m.group(1)) == sg.SBOUNDS_LEN
+
+
+def _semi24(**kw):
+    import sparse_gemm_b200 as sg
+    s = sg._SEMI24()
+    s.N, s.K = kw.get("N", 256), kw.get("K", 256)
+    for name in ("values", "meta", "status"):
+        setattr(s, name, kw.get(name, 4096))
+    return s
+
+
+@pytest.mark.parametrize("bad", [dict(N=0), dict(N=252), dict(K=96), dict(K=0), dict(values=0),
+                                 dict(values=4104), dict(meta=4100), dict(status=0)])
+def test_bad_semi24_descriptor_is_rejected_on_host(lib, bad):
+    s = _semi24(**bad)
+    assert lib.bsl_semi24_forward(4096, 64, ctypes.byref(s), None, 4096, None) == 1
+    assert lib.bsl_semi24_compress(4096, ctypes.byref(s), None) == 1
+
+
+def test_bad_semi24_matrices_are_rejected_on_host(lib):
+    s = _semi24()
+    assert lib.bsl_semi24_forward(0, 64, ctypes.byref(s), None, 4096, None) == 1      # null X
+    assert lib.bsl_semi24_forward(4096, 0, ctypes.byref(s), None, 4096, None) == 1    # M = 0
+    assert lib.bsl_semi24_forward(4096, 64, ctypes.byref(s), 4100, 4096, None) == 1   # misaligned bias
+    assert lib.bsl_semi24_forward(4096, 64, ctypes.byref(s), None, 0, None) == 1      # null Y
+    assert lib.bsl_semi24_compress(0, ctypes.byref(s), None) == 1                     # null W
+    assert lib.bsl_semi24_get_status(None, ctypes.byref(ctypes.c_int32()), None) == 1
+    assert lib.bsl_status_string(8) == b"BSL_ERR_NOT_2_4"
+
+
+def test_semi24_binding_struct_matches_the_header():
+    import sparse_gemm_b200 as sg
+    text = open(os.path.join(ROOT, "include", "bsl.h")).read()
+    start = text.index("typedef struct {", text.index("2:4 semi-structured"))
+    body = text[start:text.index("} bsl_semi24;")]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = re.findall(r"\*?\s*(\w+)\s*[;,]", body)
+    assert [n for n, _ in sg._SEMI24._fields_] == names
