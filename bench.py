@@ -18,6 +18,10 @@ rank's time.
   python bench.py --impl reference ...   # fp64 CPU oracle on a bounded sample
   python bench.py --kernel-only fwd|dx|dw --workload NAME --reps R
       # runs one contraction R times on one input copy (for ncu captures)
+
+``--workload semi24_fwd`` measures the 2:4 semi-structured layer instead
+(X[8192,4096], W[14336,4096] with two of every four weights kept, compressed
+once before timing; one step is one forward through bsl_semi24_forward).
 """
 from __future__ import annotations
 
@@ -43,6 +47,7 @@ import synth  # noqa: E402
 
 METRIC = "block-sparse GEMM effective TFLOP/s, % roofline, speedup vs dense at 75/90% sparse"
 UNIT = "TFLOP/s"
+METRIC_SEMI24 = "2:4 semi-structured GEMM TFLOP/s of kept products, % roofline, speedup vs dense"
 L2_BYTES_DEFAULT = 126 * 2 ** 20
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture
@@ -61,6 +66,9 @@ TRAFFIC = {
     ("enc_train_d1.0", "dw"): {"bytes": 31493632, "src_sha": "5abcfcfee795d983",
                                "files": ["sddmm_tc.cu", "common.cuh"],
                                "profile": "profiles/k_sddmm_tc_dw_enc_train_d1.md"},
+    ("semi24_fwd", "fwd"): {"bytes": 503706112, "src_sha": "8514e1e4bf6d7d6f",
+                            "files": ["semi24.cu", "common.cuh"],
+                            "profile": "profiles/k_semi24_fwd_semi24_fwd.md"},
 }
 # the kernel source files each contraction's traffic figure depends on
 TRAFFIC_FILES = {"fwd": ["spmm_tc.cu", "common.cuh"], "fwd_small": ["stream_fwd.cu", "common.cuh"],
@@ -641,6 +649,261 @@ def run_gpu(args):
     return out
 
 
+# ----------------------------------------------------------------------------- 2:4 semi-structured
+
+def algorithmic_semi24(w: synth.Semi24Workload):
+    """Flops (products with the kept half of the weight) and minimum HBM bytes
+    (X, compressed values, 2-bit positions and Y each moved once)."""
+    M, N, K = w.M, w.N, w.K
+    return {"flops": w.flops(), "bytes": M * K * 2 + N * (K // 2) * 2 + N * (K // 16) * 2 + M * N * 2}
+
+
+def cpu_sample_semi24(w: synth.Semi24Workload, inp: dict, budget_s: float):
+    """Time the oracle's 2:4 forward on a bounded sample of token rows (the
+    compressed form and the widened operands are prepared outside the timed
+    call).  Flops counted: the kept products, N*K per row.  Returns (flops,
+    seconds, description, threads)."""
+    import oracle
+    oracle.build()
+    v, m = oracle.compress24(inp["W"])
+    Xd = oracle.widen(inp["X"])
+    Wt = oracle.widen(oracle.decompress24(v, m))
+    nthreads = oracle.num_threads()
+    probe = np.arange(min(nthreads, w.M))
+    t0 = time.perf_counter()
+    oracle.forward(None, None, None, None, rows=probe, Xd=Xd, Wt=Wt)
+    t1 = time.perf_counter() - t0
+    n = int(min(w.M, max(1, budget_s / max(t1, 1e-6)) * len(probe)))
+    n = max(1, min(n, w.M))
+    rows = np.random.default_rng(2).choice(w.M, size=n, replace=False)
+    t0 = time.perf_counter()
+    oracle.forward(None, None, None, None, rows=rows, Xd=Xd, Wt=Wt)
+    dt = time.perf_counter() - t0
+    return float(n) * w.N * w.K, dt, f"fwd: {n} of {w.M} token rows", nthreads
+
+
+def run_gpu_semi24(args):
+    """The 2:4 workload: compress once, then K forwards per step graph, timed
+    like the block-sparse workloads (rotating input copies, CUDA-graph
+    replays, median over replays, max over ranks)."""
+    import torch
+    import torch.distributed as dist
+
+    import sparse_gemm_b200 as sg
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from sparse_gemm_b200 import build as _b
+    _b.build()
+
+    w = synth.SEMI24_WORKLOADS[args.workload]
+    inp = synth.make_semi24_inputs(w)
+    pk = peaks()
+    l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", L2_BYTES_DEFAULT) or L2_BYTES_DEFAULT
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    Wd, X0 = dev_bf16(inp["W"]), dev_bf16(inp["X"])
+    stream = torch.cuda.current_stream(dev)
+    w0 = sg.compress24(Wd)
+    torch.cuda.synchronize()
+    ce0, ce1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    comp_ms = []
+    for _ in range(5):
+        ce0.record(stream)
+        sg.compress24(Wd, out=w0)
+        ce1.record(stream)
+        torch.cuda.synchronize()
+        comp_ms.append(ce0.elapsed_time(ce1))
+    if sg.semi24_status(w0) != 0:
+        raise RuntimeError("compress reported a device error")
+
+    in_bytes = X0.numel() * 2 + w.N * (w.K // 2) * 2 + w.N * (w.K // 16) * 2
+    ncopy = int(min(16, max(2, math.ceil(2 * l2 / in_bytes) + 1)))
+    Xs = [X0] + [X0.clone() for _ in range(ncopy - 1)]
+    ws = [w0] + [sg.compress24(Wd) for _ in range(ncopy - 1)]
+    Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        sg.forward24(Xs[i % ncopy], ws[i % ncopy], out=Y)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(device=dev)
+        cs.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cs):
+            for i in range(K):
+                fn(i)
+        stream.wait_stream(cs)
+        torch.cuda.synchronize()
+        return g
+
+    def replay_times(g, reps):
+        g.replay()
+        torch.cuda.synchronize()
+        out = []
+        for _ in range(reps):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            g.replay()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            out.append(ev0.elapsed_time(ev1))
+        return out
+
+    g_step = capture(step)
+    g_warm = capture(lambda i: step(0))
+    clocks = ClockSampler(local)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_times = replay_times(g_step, args.replays)
+    total_ms = statistics.median(step_times)
+    warm_ms = statistics.median(replay_times(g_warm, args.replays))
+    t_end = time.time() + 0.5
+    while time.time() < t_end:
+        g_step.replay()
+        torch.cuda.synchronize()
+    clk = clocks.stop()
+    fwd_ms = total_ms / K
+    total_ms = max_over_ranks(total_ms, world, dev)
+    alg = algorithmic_semi24(w)
+    value = whole_job_value(world, alg["flops"], K, total_ms)
+    ms_per_step = total_ms / K
+
+    # the kept products run at twice the dense rate on the sparse MMA, so the
+    # useful-flop peak of the 2:4 kernel is the dense bf16 peak
+    roof = roofline_entry("fwd", alg, fwd_ms, pk)
+    roof["kernel"] = "k_semi24_fwd"
+    roof["peak_source"] = pk["source"] + (" burst bf16 (useful flops of the 2:4 MMA)"
+                                          if roof["unit"] == "TFLOP/s" else " HBM copy")
+    tr = TRAFFIC.get((w.name, "fwd"))
+    roof["traffic"] = tr["bytes"] if tr and tr.get("src_sha") == src_sha(*tr["files"]) else None
+    roof["algorithmic_bytes"] = alg["bytes"]
+    roof["algorithmic_flops"] = alg["flops"]
+    roof["dense_equivalent_tflops"] = round(2 * alg["flops"] / (fwd_ms * 1e-3) / 1e12, 2)
+    roof["tensor_frac_of_sustained"] = round(alg["flops"] / (fwd_ms * 1e-3) / 1e12
+                                             / pk["bf16_tflops_sustained"], 4)
+
+    # cuBLAS dense on the same weight (zeros in place), same rotation
+    Wds = [Wd] + [Wd.clone() for _ in range(min(ncopy, 3) - 1)]
+
+    def dense_step(i):
+        torch.matmul(Xs[i % ncopy], Wds[i % len(Wds)].t(), out=Y)
+
+    for i in range(max(3, args.warmup)):
+        dense_step(i)
+    torch.cuda.synchronize()
+    dense_ms = statistics.median(replay_times(capture(dense_step), args.replays)) / K
+
+    # end to end through the public API: pinned host X in, Y out, every step;
+    # uploads, layer and downloads pipelined on three streams with two buffer sets
+    hX = torch.empty(X0.shape, dtype=torch.bfloat16, pin_memory=True).copy_(X0.cpu())
+    hY = torch.empty(Y.shape, dtype=torch.bfloat16, pin_memory=True)
+    bufs = [{"X": torch.empty_like(X0), "Y": torch.empty_like(Y)} for _ in range(2)]
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for j in range(2):
+        ev_comp[j].record(s_comp)
+        ev_out[j].record(s_out)
+
+    def e2e_step(i):
+        j = i % 2
+        b = bufs[j]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[j])
+            b["X"].copy_(hX, non_blocking=True)
+            ev_in[j].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[j])
+            s_comp.wait_event(ev_out[j])
+            sg.forward24(b["X"], w0, out=b["Y"])
+            ev_comp[j].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[j])
+            hY.copy_(b["Y"], non_blocking=True)
+            ev_out[j].record(s_out)
+
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    ke = max(3, min(K, 50))
+    if world > 1:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    s_comp.wait_event(t0)
+    s_out.wait_event(t0)
+    for i in range(ke):
+        e2e_step(i)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1) / ke, world, dev)
+    for ww in ws:
+        if sg.semi24_status(ww) != 0:
+            raise RuntimeError("kernels reported a device error")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        done, secs, desc, nthr = cpu_sample_semi24(w, inp, args.cpu_budget)
+        cpu = {"value": round(done / secs / 1e12, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
+               "sample": desc + f" ({secs:.1f} s, fp64 loops over the dense weight with zeros in place)",
+               "cpu_model": cpu_model()}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC_SEMI24, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": w.name, "M": w.M, "N": w.N, "K": w.K, "pattern": "2:4 along K", "seed": w.seed,
+            "contractions_per_step": ["fwd"], "global_batch": w.M * world,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"rotating {ncopy} copies of every input ({ncopy * in_bytes / 2**20:.0f} MiB > 2x L2)",
+            "compress_ms": round(statistics.median(comp_ms), 4),
+            "timing": "cuda-graph",
+        },
+        "timing_spread": {"replays": len(step_times), "min_ms_per_step": round(min(step_times) / K, 5),
+                          "max_ms_per_step": round(max(step_times) / K, 5),
+                          "median_ms_per_step": round(statistics.median(step_times) / K, 5)},
+        "warm_l2": {"ms_per_step": round(warm_ms / K, 5),
+                    "value": round(whole_job_value(1, alg["flops"], K, warm_ms), 3),
+                    "note": "same K steps on one input copy (operands stay in L2); not the headline"},
+        "kernels_ms": {"fwd": round(fwd_ms, 5)},
+        "roofline": roof,
+        "dense_cublas_ms_per_step": round(dense_ms, 5),
+        "speedup_vs_dense": round(dense_ms / ms_per_step, 3),
+        "e2e": {"value": round(whole_job_value(world, alg["flops"], 1, e2e_ms), 3), "unit": UNIT,
+                "h2d_bytes_per_step": X0.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
+                "ms_per_step": round(e2e_ms, 4),
+                "timing": "public API calls, uploads / layer / downloads pipelined on three streams"},
+        "gpu_launches": K,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -650,10 +913,12 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
+    per_step = max(0.5, min(20.0, args.reference_budget / max(1, args.steps + args.warmup)))
+    if args.workload in synth.SEMI24_WORKLOADS:
+        return run_reference_semi24(args, world, per_step)
     w = synth.WORKLOADS[args.workload]
     inp = synth.make_inputs(w)
     kinds = ["fwd", "dx", "dw"] if w.with_dy else ["fwd"]
-    per_step = max(0.5, min(20.0, args.reference_budget / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_sample(w, inp, per_step, kinds)
     done, secs, descs = 0.0, 0.0, []
@@ -678,6 +943,33 @@ def run_reference(args):
     }
 
 
+def run_reference_semi24(args, world, per_step):
+    """The oracle's 2:4 forward on the host cores, a bounded sample of token
+    rows per step; value is TFLOP/s of kept products."""
+    w = synth.SEMI24_WORKLOADS[args.workload]
+    inp = synth.make_semi24_inputs(w)
+    for _ in range(args.warmup):
+        cpu_sample_semi24(w, inp, per_step)
+    done, secs, descs, nthr = 0.0, 0.0, [], 1
+    for _ in range(args.steps):
+        d, s_, desc, nthr = cpu_sample_semi24(w, inp, per_step)
+        done += d
+        secs += s_
+        descs.append(desc)
+    value = done / secs / 1e12
+    return {
+        "impl": "reference", "metric": METRIC_SEMI24, "value": round(value, 8), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "pattern": "2:4 along K", "seed": w.seed},
+        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
+                         "sample": descs[0] + " per step (fp64 loops over the dense weight with zeros in place)",
+                         "cpu_model": cpu_model()},
+        "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_kernel_only(args):
     """One contraction of a workload, `--reps` times, on a single input copy
     (no rotation, no comparison runs): the command the ncu captures use."""
@@ -686,9 +978,25 @@ def run_kernel_only(args):
     import sparse_gemm_b200 as sg
     from sparse_gemm_b200 import build as _b
     _b.build()
+    dev = torch.device("cuda", 0)
+    if args.workload in synth.SEMI24_WORKLOADS:
+        if args.kernel_only != "fwd":
+            raise SystemExit("the 2:4 workload has a forward only")
+        w = synth.SEMI24_WORKLOADS[args.workload]
+        inp = synth.make_semi24_inputs(w)
+        bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        w24 = sg.compress24(bits(inp["W"]))
+        X = bits(inp["X"])
+        for _ in range(args.reps):
+            sg.forward24(X, w24)
+        torch.cuda.synchronize()
+        st = sg.semi24_status(w24)
+        if st != 0:
+            raise RuntimeError(f"device status {st}")
+        print(json.dumps({"kernel_only": "fwd", "workload": w.name, "reps": args.reps}))
+        return
     w = synth.WORKLOADS[args.workload]
     inp = synth.make_inputs(w, with_dy=args.kernel_only != "fwd")
-    dev = torch.device("cuda", 0)
 
     def to_dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -717,7 +1025,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="large_fwd", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="large_fwd",
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.SEMI24_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
     ap.add_argument("--reference-budget", type=float, default=120.0)
@@ -731,7 +1040,12 @@ def main():
     if args.kernel_only:
         run_kernel_only(args)
         return
-    out = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if args.impl == "reference":
+        out = run_reference(args)
+    elif args.workload in synth.SEMI24_WORKLOADS:
+        out = run_gpu_semi24(args)
+    else:
+        out = run_gpu(args)
     if out is not None:
         print(json.dumps(out), flush=True)
 

@@ -13,22 +13,22 @@
 // (tcgen05.mma.sp, kind::f16).  The compressed weight is the MMA's A operand
 // (the operand the instruction takes compressed), so the accumulator holds
 // Y^T: TMEM lane = output feature, column = token.  Persistent, one CTA per
-// SM, tiles of 256 features x 192 tokens (two M = 128 MMA blocks sharing the
+// SM, tiles of 256 features x 224 tokens (two M = 128 MMA blocks sharing the
 // token tile), 64 dense K per stage (two K = 32 sparse MMAs per block).
 // Roles (16 warps):
 //   warp 0      TMA producer: per stage the compressed weight tile
 //               (256 rows x 64 B, 64-byte swizzle) and the activation tile
-//               (192 rows x 128 B, 128-byte swizzle) into a 5-stage ring;
+//               (224 rows x 128 B, 128-byte swizzle) into a 4-stage ring;
 //   warp 1      MMA issuer (lane 0), TMEM owner;
 //   warps 4-7   metadata: per stage, the positions of their 32 TMEM lanes
 //               loaded from global memory, rearranged into the lane layout
-//               the sparse MMA reads (below) and written into an 8-stage
-//               TMEM ring with tcgen05.st;
+//               the sparse MMA reads (below) and written into a 4-stage
+//               TMEM ring with tcgen05.st (the loads run 8 stages ahead);
 //   warps 8-15  epilogue: TMEM -> registers (+ bias) -> bf16, transposed
-//               through a 1 KB staging chunk per warp, TMA store of
-//               16 tokens x 32 features.
-// TMEM: columns 0..383 the two 128 x 192 fp32 accumulators (one buffer),
-// 384..511 the metadata ring, 16 columns per stage: the metadata of block h,
+//               through a 2 KB staging chunk per warp, TMA store of
+//               32 tokens x 32 features.
+// TMEM: columns 0..447 the two 128 x 224 fp32 accumulators (one buffer),
+// 448..511 the metadata ring, 16 columns per stage: the metadata of block h,
 // K step j at column 4(2h + j) of the stage (a sparse MMA's metadata address
 // must be a multiple of 4 columns: an odd one raised a misaligned-address
 // error on B200, and CUTLASS's sparse-MMA metadata fragments assume the same
@@ -102,20 +102,21 @@ __global__ void k_compress24(const uint4 *__restrict__ W, int64_t chunks, uint4 
 
 struct Semi24Cfg {
     static constexpr int BF = 256;                    // features per tile (two M = 128 blocks)
-    static constexpr int BT = 192;                    // tokens per tile (MMA N)
+    static constexpr int BT = 224;                    // tokens per tile (MMA N)
     static constexpr int BK = 64;                     // dense K per stage
-    static constexpr int S = 5;                       // copy stages
+    static constexpr int S = 4;                       // copy stages
     static constexpr int A_BYTES = BF * BK;           // 256 rows x 32 kept bf16
-    static constexpr int B_BYTES = BT * BK * 2;       // 192 rows x 64 bf16
+    static constexpr int B_BYTES = BT * BK * 2;       // 224 rows x 64 bf16
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int MS = 8;                      // metadata ring stages (TMEM)
+    static constexpr int MS = 4;                      // metadata ring stages (TMEM)
     static constexpr int MCOLS = 16;                  // TMEM columns per metadata stage
     static constexpr int META_COL = 2 * BT;           // first metadata column
     static constexpr int TMEM_COLS = 512;
     static constexpr int EPI_WARPS = 8;
-    static constexpr int OUT_CHUNK = 16 * 32 * 2;     // 16 tokens x 32 features bf16
+    static constexpr int OUT_CHUNK = 32 * 32 * 2;     // 32 tokens x 32 features bf16
     static constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_CHUNK;
     static constexpr int W_PROD = 0, W_MMA = 1, W_META = 4, W_EPI = 8;
+    static constexpr int BAND = 16;                   // token tiles per band of the tile order
     static constexpr int THREADS = 16 * 32;
     static constexpr int BAR_BYTES = 1024;
     static constexpr int SMEM_BYTES = 1024 + S * STAGE_BYTES + OUT_BYTES + BAR_BYTES;
@@ -127,6 +128,7 @@ struct Semi24Cfg {
 struct Semi24Args {
     int32_t M, N, K;
     int32_t ntf;    // feature tiles
+    int32_t ntt;    // token tiles
     int32_t tiles;  // feature tiles x token tiles
     int32_t ks;     // stages per tile (K / 64)
     const uint16_t *meta;
@@ -134,6 +136,21 @@ struct Semi24Args {
     int32_t *status;
     uint64_t timeout_ns;
 };
+
+// Tile t of the launch: bands of BAND token tiles in order, and inside a band
+// every feature tile, feature tile major, so the CTAs working at one time
+// share the weight slices of a few feature tiles and the activations of one
+// band, which stay in L2 while the band is processed.
+__device__ __forceinline__ void tile_origin(int t, const Semi24Args &a, int &f0, int &t0)
+{
+    using C = Semi24Cfg;
+    const int band = t / (C::BAND * a.ntf);
+    const int idx = t - band * C::BAND * a.ntf;
+    const int first = band * C::BAND;
+    const int width = a.ntt - first < C::BAND ? a.ntt - first : C::BAND;
+    f0 = (idx / width) * C::BF;
+    t0 = (first + idx % width) * C::BT;
+}
 
 // tcgen05.mma.sp (A compressed, metadata in TMEM), issued by the leader lane
 // of a converged warp.
@@ -146,6 +163,20 @@ __device__ __forceinline__ void umma_sp_lead(uint32_t leader, uint32_t d_tmem, u
         "setp.ne.b32 p, %5, 0;\n\t"
         "@e tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(meta_tmem), "r"(idesc), "r"(accumulate), "r"(leader)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
         : "memory");
 }
 
@@ -212,7 +243,8 @@ __global__ void __launch_bounds__(Semi24Cfg::THREADS, 1)
             bool ok = true;
             int g = 0;  // stages issued
             for (int t = blockIdx.x; ok && t < args.tiles; t += gridDim.x) {
-                const int f0 = (t % args.ntf) * C::BF, t0 = (t / args.ntf) * C::BT;
+                int f0, t0;
+                tile_origin(t, args, f0, t0);
                 for (int k = 0; k < args.ks; ++k, ++g) {
                     const int slot = g % C::S;
                     if (g >= C::S && !mbar_wait(&empty[slot], ((g / C::S) - 1) & 1, tmo, abort_flag)) {
@@ -293,36 +325,54 @@ __global__ void __launch_bounds__(Semi24Cfg::THREADS, 1)
     } else if (warp >= C::W_META && warp < C::W_META + 4) {
         // ------------------------------------------------------------ metadata
         // Lane l loads the 8 bytes of positions (dense K 64k .. 64k+63) of
-        // block row 32q + l, then takes from lanes src_lo / src_hi the 16-bit
-        // halves that its TMEM lane 32q + l holds (layout in the file header).
+        // block row 32q + l of each block, then takes from lanes src_lo /
+        // src_hi the 16-bit halves that its TMEM lane 32q + l holds (layout in
+        // the file header).
         const int q = warp & 3;
         const int src_lo = (lane & 16) | (lane & 7), src_hi = src_lo + 8;
         const bool upper = (lane >> 3) & 1;  // K half kh of the lane
         const size_t row_words = static_cast<size_t>(args.K) / 64;  // 8-byte words per row
         const uint2 *meta = reinterpret_cast<const uint2 *>(args.meta);
+        const uint2 pad = make_uint2(0x44444444u, 0x44444444u);  // rows past N: pairs (0, 1) over zeros
+        // stages of this CTA, all tiles in order: stage g is step g % ks of the
+        // CTA's tile g / ks; the loads run P stages ahead of their use
+        constexpr int P = 8;
+        const int G = (args.tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                      static_cast<int>(gridDim.x) * args.ks;
+        auto load = [&](int g, uint2 &m0, uint2 &m1) {
+            m0 = pad;
+            m1 = pad;
+            if (g >= G) return;
+            const int i = g / args.ks, k = g - i * args.ks;
+            const int t = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+            int f0, t0;
+            tile_origin(t, args, f0, t0);
+            const int r0 = f0 + 32 * q + lane;
+            if (r0 < args.N) m0 = __ldg(meta + static_cast<size_t>(r0) * row_words + k);
+            if (r0 + 128 < args.N) m1 = __ldg(meta + static_cast<size_t>(r0 + 128) * row_words + k);
+        };
+        uint2 b0[P], b1[P];
+#pragma unroll
+        for (int p = 0; p < P; ++p) load(p, b0[p], b1[p]);
         bool ok = true;
-        int g = 0;
-        for (int t = blockIdx.x; ok && t < args.tiles; t += gridDim.x) {
-            const int r0 = (t % args.ntf) * C::BF + 32 * q + lane;
-            const bool valid0 = r0 < args.N, valid1 = r0 + 128 < args.N;
-            const uint2 *row0 = meta + (valid0 ? static_cast<size_t>(r0) * row_words : 0);
-            const uint2 *row1 = meta + (valid1 ? static_cast<size_t>(r0 + 128) * row_words : 0);
-            for (int k = 0; k < args.ks; ++k, ++g) {
+        for (int g0 = 0; ok && g0 < G; g0 += P) {
+#pragma unroll
+            for (int p = 0; p < P; ++p) {
+                const int g = g0 + p;
+                if (g >= G) break;
                 const int ms = g % C::MS;
-                // rows past N read as pairs (0, 1), over zero values
-                const uint2 m0 = valid0 ? __ldg(row0 + k) : make_uint2(0x44444444u, 0x44444444u);
-                const uint2 m1 = valid1 ? __ldg(row1 + k) : make_uint2(0x44444444u, 0x44444444u);
                 uint32_t w[4];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const uint32_t x = h ? (j ? m1.y : m1.x) : (j ? m0.y : m0.x);
+                        const uint32_t x = h ? (j ? b1[p].y : b1[p].x) : (j ? b0[p].y : b0[p].x);
                         const uint32_t lo = __shfl_sync(0xffffffffu, x, src_lo);
                         const uint32_t hi = __shfl_sync(0xffffffffu, x, src_hi);
                         w[2 * h + j] = (upper ? lo >> 16 : lo & 0xFFFFu) | (upper ? hi & 0xFFFF0000u : hi << 16);
                     }
                 }
+                load(g + P, b0[p], b1[p]);
                 if (g >= C::MS &&
                     __any_sync(0xffffffffu, !mbar_wait(&mempty[ms], ((g / C::MS) - 1) & 1, tmo, abort_flag))) {
                     ok = false;
@@ -346,27 +396,29 @@ __global__ void __launch_bounds__(Semi24Cfg::THREADS, 1)
     } else if (warp >= C::W_EPI) {
         // ------------------------------------------------------------ epilogue
         // Warp e reads block h = e / 4, TMEM lanes 32q .. 32q+31 (features),
-        // 16 token columns at a time.  Neighbouring lanes swap values so each
+        // 32 token columns at a time.  Neighbouring lanes swap values so each
         // writes one 32-bit word (two features of one token) into the
-        // [16 tokens][32 features] staging chunk, stored by TMA.
+        // [32 tokens][32 features] staging chunk, stored by TMA.
         const int e = warp - C::W_EPI, q = warp & 3, h = e >> 2;
         uint8_t *wbuf = outbuf + e * 2 * C::OUT_CHUNK;
         const bool odd = lane & 1;
         bool ok = true;
         int it = 0, ob = 0;
         for (int t = blockIdx.x; ok && t < args.tiles; t += gridDim.x, ++it) {
-            const int f0 = (t % args.ntf) * C::BF + h * 128 + 32 * q, t0 = (t / args.ntf) * C::BT;
+            int f0, t0;
+            tile_origin(t, args, f0, t0);
+            f0 += h * 128 + 32 * q;
             const float bv = (args.bias && f0 + lane < args.N) ? __bfloat162float(args.bias[f0 + lane]) : 0.f;
             const int left = args.M - t0;
-            const int nch = left >= C::BT ? C::BT / 16 : (left + 15) / 16;
+            const int nch = left >= C::BT ? C::BT / 32 : (left + 31) / 32;
             if (__any_sync(0xffffffffu, !mbar_wait(afull, it & 1, tmo, abort_flag))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             for (int c = 0; c < nch; ++c) {
-                uint32_t v[16];
-                tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + h * C::BT + c * 16, v);
+                uint32_t v[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + h * C::BT + c * 32, v);
                 tmem_wait_ld();
                 if (c == nch - 1) {  // this warp's last TMEM read of the tile
                     tc_fence_before();
@@ -378,7 +430,7 @@ __global__ void __launch_bounds__(Semi24Cfg::THREADS, 1)
                 __syncwarp();
                 uint8_t *dst = wbuf + ob * C::OUT_CHUNK;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 16; ++u) {
                     const float a = __uint_as_float(v[2 * u]) + bv, b = __uint_as_float(v[2 * u + 1]) + bv;
                     const float other = __shfl_xor_sync(0xffffffffu, odd ? a : b, 1);
                     const uint32_t word = odd ? pack_bf16x2(other, b) : pack_bf16x2(a, other);
@@ -387,7 +439,7 @@ __global__ void __launch_bounds__(Semi24Cfg::THREADS, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmY, dst, f0, t0 + 16 * c);
+                    tma_store_2d(&tmY, dst, f0, t0 + 32 * c);
                     bulk_commit_group();
                 }
                 ob ^= 1;
@@ -430,14 +482,15 @@ bsl_status launch_semi24_fwd(const void *X, int32_t M, const bsl_semi24 *W, cons
     CUtensorMap ma, mx, my;
     if (!make_map_2d(&ma, W->values, W->K / 2, W->N, static_cast<uint64_t>(W->K), C::BK / 2, C::BF, 64) ||
         !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, C::BK, C::BT, 128) ||
-        !make_map_2d(&my, Y, W->N, M, static_cast<uint64_t>(W->N) * 2, 32, 16, 0))
+        !make_map_2d(&my, Y, W->N, M, static_cast<uint64_t>(W->N) * 2, 32, 32, 0))
         return BSL_ERR_CUDA;
     Semi24Args args;
     args.M = M;
     args.N = W->N;
     args.K = W->K;
     args.ntf = (W->N + C::BF - 1) / C::BF;
-    const int64_t tiles = static_cast<int64_t>(args.ntf) * ((M + C::BT - 1) / C::BT);
+    args.ntt = (M + C::BT - 1) / C::BT;
+    const int64_t tiles = static_cast<int64_t>(args.ntf) * args.ntt;
     if (tiles > 0x7FFFFFFF) return BSL_ERR_UNSUPPORTED;
     args.tiles = static_cast<int32_t>(tiles);
     args.ks = W->K / C::BK;

@@ -61,8 +61,19 @@ def test_reported_bound(name, kind, bound):
 
 def test_traffic_entries_name_their_sources():
     for (wname, kind), t in bench.TRAFFIC.items():
-        assert wname in synth.WORKLOADS and kind in ("fwd", "dx", "dw")
+        assert (wname in synth.WORKLOADS or wname in synth.SEMI24_WORKLOADS) and kind in ("fwd", "dx", "dw")
         assert t["bytes"] > 0 and len(t["src_sha"]) == 16
         assert os.path.exists(os.path.join(ROOT, t["profile"]))
         for f in t["files"]:
             assert os.path.exists(os.path.join(ROOT, "sparse_gemm_b200", "csrc", f))
+
+
+def test_semi24_work_bytes_and_bound():
+    """2:4 forward: kept products 2·M·N·(K/2); bytes X + half-width values +
+    4 bits of positions per group + Y; at the LLM-MLP size it is tensor-bound
+    against the dense peak (the kept products run at twice the dense rate)."""
+    w = synth.SEMI24_WORKLOADS["semi24_fwd"]
+    alg = bench.algorithmic_semi24(w)
+    assert alg["flops"] == 2 * w.M * w.N * (w.K // 2)
+    assert alg["bytes"] == w.M * w.K * 2 + w.N * w.K + w.N * w.K // 8 + w.M * w.N * 2
+    assert bench.roofline_entry("fwd", alg, 0.5, PEAKS)["bound"] == "tensor"

@@ -3,9 +3,9 @@
 The compressed form (values and positions) must match the oracle bit for
 bit; the forward must match the oracle's product element by element within
 the bound of tests/_parity.py.  Shapes span several tiles (256 features x
-192 tokens) with ragged tails, one token, more tiles than SMs (so a CTA
+224 tokens) with ragged tails, one token, more tiles than SMs (so a CTA
 walks several tiles and the rings wrap), and the full workload size on
-sampled rows (the first and last token of every 192-token tile).
+sampled rows (the first and last token of every 224-token tile).
 """
 import numpy as np
 import pytest
@@ -63,11 +63,11 @@ FWD_CASES = [
     # M, N, K, bias, seed
     (1, 8, 64, False, 10),
     (5, 200, 128, True, 11),
-    (192, 256, 64, False, 12),
-    (193, 264, 192, True, 13),
+    (224, 256, 64, False, 12),
+    (225, 264, 192, True, 13),
     (400, 520, 320, True, 14),
     (700, 1032, 1024, False, 15),   # 16 stages per tile: the metadata ring wraps
-    (3000, 2560, 128, True, 16),    # 160 tiles: CTAs walk several tiles
+    (3400, 2560, 128, True, 16),    # 160 tiles: CTAs walk several tiles
 ]
 
 
@@ -129,7 +129,7 @@ def test_full_workload_sampled_rows():
     Y = sg.forward24(to_dev(X), w)
     torch.cuda.synchronize()
     assert sg.semi24_status(w) == 0
-    rows = sorted({r for t in range(0, wl.M, 192) for r in (t, min(t + 191, wl.M - 1))})
+    rows = sorted({r for t in range(0, wl.M, 224) for r in (t, min(t + 223, wl.M - 1))})
     v, m = oracle.compress24(W)
     ref, refabs = oracle.semi24_forward(X, v, m, rows=np.asarray(rows))
     assert_parity(to_f64(Y[rows]), ref, refabs, "semi24 forward, full size, sampled rows")
