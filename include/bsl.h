@@ -269,6 +269,34 @@ BSL_API bsl_status bsl_semi24_compress(const void *W, const bsl_semi24 *out, voi
 BSL_API bsl_status bsl_semi24_forward(const void *X, int32_t M, const bsl_semi24 *W, const void *bias, void *Y,
                                       void *stream);
 
+/* ---------------------------------------------------------------- 2:4 inside blocks
+ *
+ * A block-sparse weight (bsl_bsr, packed by bsl_pack) whose kept blocks carry
+ * the 2:4 pattern along K: the "50% sparse pattern within blocks" of the
+ * release note's "Future Development Roadmap" and the "blocks of 2:4" of the
+ * "Lecture 11: Sparsity" summary (43:51).  The kept blocks are stored
+ * compressed beside the packed weight:
+ *   values24  bf16 [nnz + 1][b][b/2]: block p in BSR order, each row's two kept
+ *             elements of every group of four in column order; block nnz is
+ *             zeros (written by bsl_bsr24_compress);
+ *   meta24    uint16 [nnz][b][b/16]: the positions, per row as bsl_semi24.meta.
+ * Both caller-allocated, 16-byte aligned. */
+
+/* Compress the packed weight's kept blocks (W->values) into values24 and
+ * meta24, with the kept positions chosen as bsl_semi24_compress does.  A
+ * group with more than two nonzeros sets BSL_ERR_NOT_2_4 in W's device status
+ * (read it with bsl_get_device_status). */
+BSL_API bsl_status bsl_bsr24_compress(const bsl_bsr *W, void *values24, uint16_t *meta24, void *stream);
+
+/* Y [M][N] = X [M][K] . W~^T (+ bias), W~ the block-sparse weight with zeros
+ * outside its blocks, the blocks read from values24 / meta24 (the dense
+ * product with zeros in place: torchao README, introduction).  bf16 in, fp32
+ * accumulation, bias bf16 [N] or NULL.  b must be 64 (BSL_ERR_UNSUPPORTED
+ * otherwise).  Sparse tensor-core kernel driven by W's row-group plan,
+ * persistent, one CTA per SM. */
+BSL_API bsl_status bsl_bsr24_forward(const void *X, int32_t M, const bsl_bsr *W, const void *values24,
+                                     const uint16_t *meta24, const void *bias, void *Y, void *stream);
+
 /* SYNCHRONOUS: waits for the stream, copies the device status word of W to
  * *status_host (a bsl_status value) and resets it to BSL_OK. */
 BSL_API bsl_status bsl_semi24_get_status(const bsl_semi24 *W, int32_t *status_host, void *stream);

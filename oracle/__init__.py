@@ -326,6 +326,18 @@ def decompress24(values, meta):
     return out.reshape(N, K)
 
 
+def compress24_blocks(values):
+    """2:4 compressed form of packed b x b blocks ([nnz, b, b] bf16 bits, as
+    :func:`pack` returns them), block by block along each block row: the
+    "50% sparse pattern within blocks" of the Hugging Face release note
+    ("Future Development Roadmap") stored as Table 4.1's compressed
+    representation.  Returns (values [nnz, b, b/2], meta [nnz, b, b/16])."""
+    values = np.ascontiguousarray(values, dtype=np.uint16)
+    nnz, b, _ = values.shape
+    v, m = compress24(values.reshape(nnz * b, b))
+    return v.reshape(nnz, b, b // 2), m.reshape(nnz, b, b // 16)
+
+
 def semi24_forward(X, values, meta, rows=None, *, Xd=None, bias=None):
     """Y[rows] = X[rows] W^T (+ bias) in fp64 with W the dense weight that
     the compressed form stands for: the sparse product is the dense product

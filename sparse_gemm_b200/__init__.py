@@ -26,6 +26,7 @@ __all__ = [
     "forward_stream_noalloc", "bias_grad",
     "BlockSparseLinearFunction", "BlockSparseLinear",
     "Semi24Weight", "compress24", "forward24", "semi24_status",
+    "Bsr24Weight", "compress_bsr24", "forward_bsr24",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -94,6 +95,8 @@ def library() -> ctypes.CDLL:
             "bsl_semi24_compress": (ctypes.c_int, [P, SP, P]),
             "bsl_semi24_forward": (ctypes.c_int, [P, I32, SP, P, P, P]),
             "bsl_semi24_get_status": (ctypes.c_int, [SP, ctypes.POINTER(I32), P]),
+            "bsl_bsr24_compress": (ctypes.c_int, [BP, P, P, P]),
+            "bsl_bsr24_forward": (ctypes.c_int, [P, I32, BP, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -493,3 +496,47 @@ def semi24_status(w: Semi24Weight) -> int:
     _check(library().bsl_semi24_get_status(w.cref(), ctypes.byref(out), _stream(w.values)),
            "bsl_semi24_get_status")
     return int(out.value)
+
+
+# ---------------------------------------------------------------- 2:4 inside blocks
+
+
+class Bsr24Weight:
+    """The kept blocks of a packed block-sparse weight in 2:4 compressed form
+    ("50% sparse pattern within blocks", release note, "Future Development
+    Roadmap"): ``values`` bf16 [nnz + 1, b, b/2] (the last block zeros) and
+    ``meta`` [nnz, b, b/16] (16-bit position words held in an int16 tensor),
+    beside the packed weight whose index and plan drive the kernel."""
+
+    def __init__(self, packed: BsrWeight):
+        b, nnz = packed.b, packed.nnz
+        self.packed = packed
+        self.values = torch.zeros((nnz + 1, b, b // 2), dtype=torch.bfloat16, device=packed.device)
+        self.meta = torch.zeros((max(nnz, 1), b, b // 16), dtype=torch.int16, device=packed.device)
+
+    @property
+    def nnz(self):
+        return self.packed.nnz
+
+
+def compress_bsr24(Wp: BsrWeight, out: Bsr24Weight | None = None) -> Bsr24Weight:
+    """Compress the kept blocks of ``Wp`` (2:4 along K inside each block).  A
+    group with more than two nonzeros is reported by :func:`device_status`
+    (BSL_ERR_NOT_2_4)."""
+    w = Bsr24Weight(Wp) if out is None else out
+    _check(library().bsl_bsr24_compress(Wp.cref(), w.values.data_ptr(), w.meta.data_ptr(),
+                                        _stream(Wp.values)), "bsl_bsr24_compress")
+    return w
+
+
+def forward_bsr24(X: torch.Tensor, w: Bsr24Weight, bias: torch.Tensor | None = None,
+                  out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W^T (+ bias) for a block-sparse weight with 2:4 blocks (b = 64)."""
+    Wp = w.packed
+    _cuda_bf16_2d(X, "X", Wp.K)
+    bptr = _bias_ptr(bias, Wp.N, X)
+    M = X.shape[0]
+    Y = _out(M, Wp.N, X) if out is None else out
+    _check(library().bsl_bsr24_forward(X.data_ptr(), M, Wp.cref(), w.values.data_ptr(), w.meta.data_ptr(),
+                                       bptr, Y.data_ptr(), _stream(X)), "bsl_bsr24_forward")
+    return Y

@@ -200,6 +200,28 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
     return r == CUDA_SUCCESS;
 }
 
+bool make_map_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
+                 uint64_t stride2, uint32_t box0, uint32_t box1, int swizzle_bytes)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        note_driver_error(999);
+        return false;
+    }
+    const cuuint64_t dims[3] = {d0, d1, d2 > 0 ? d2 : 1};
+    const cuuint64_t strides[2] = {stride1, stride2};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                        : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) note_driver_error(static_cast<int>(r));
+    return r == CUDA_SUCCESS;
+}
+
 bool make_block_map(CUtensorMap *map, const void *values, int32_t b, int32_t nblocks, uint32_t box_rows)
 {
     EncodeTiledFn fn = encode_fn();
@@ -400,6 +422,32 @@ bsl_status bsl_semi24_forward(const void *X, int32_t M, const bsl_semi24 *W, con
     BSL_TRY(guard.bind(X));
     BSL_TRY(check_device());
     return launch_semi24_fwd(X, M, W, bias, Y, static_cast<cudaStream_t>(stream));
+}
+
+bsl_status bsl_bsr24_compress(const bsl_bsr *W, void *values24, uint16_t *meta24, void *stream)
+{
+    BSL_TRY(check_bsr(W));
+    if (!values24 || !aligned(values24, 16) || (W->nnz > 0 && (!meta24 || !aligned(meta24, 16))))
+        return BSL_ERR_INVALID_ARG;
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(values24));
+    BSL_TRY(check_device());
+    return launch_bsr24_compress(W, values24, meta24, static_cast<cudaStream_t>(stream));
+}
+
+bsl_status bsl_bsr24_forward(const void *X, int32_t M, const bsl_bsr *W, const void *values24,
+                             const uint16_t *meta24, const void *bias, void *Y, void *stream)
+{
+    BSL_TRY(check_bsr(W));
+    if (W->b != 64) return BSL_ERR_UNSUPPORTED;
+    if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
+    if (!values24 || !aligned(values24, 16) || (W->nnz > 0 && (!meta24 || !aligned(meta24, 16))))
+        return BSL_ERR_INVALID_ARG;
+    if (bias && !aligned(bias, 16)) return BSL_ERR_INVALID_ARG;
+    DeviceGuard guard;
+    BSL_TRY(guard.bind(X));
+    BSL_TRY(check_device());
+    return launch_bsr24_fwd(X, M, W, values24, meta24, bias, Y, static_cast<cudaStream_t>(stream));
 }
 
 bsl_status bsl_semi24_get_status(const bsl_semi24 *W, int32_t *status_host, void *stream)

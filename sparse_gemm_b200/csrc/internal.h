@@ -16,6 +16,11 @@ namespace bsl {
 bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                  uint32_t box_inner, uint32_t box_outer, int swizzle_bytes);
 
+// Encode a 3-D bf16 tensor map: d0 contiguous elements, d1 rows `stride1`
+// bytes apart, d2 planes `stride2` bytes apart; box of box0 x box1 x 1.
+bool make_map_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1,
+                 uint64_t stride2, uint32_t box0, uint32_t box1, int swizzle_bytes);
+
 // Encode the packed weight values bf16 [nblocks][b][b] as a 3-D tensor map
 // (x = column inside a block, y = row inside a block, z = block) with a
 // box of b columns x box_rows rows x 1 block, swizzled like the kernels'
@@ -75,6 +80,12 @@ bsl_status launch_bias_grad(const void *dY, int32_t M, int32_t N, void *dbias, c
 bsl_status launch_compress24(const void *W, const bsl_semi24 *out, cudaStream_t s);
 bsl_status launch_semi24_fwd(const void *X, int32_t M, const bsl_semi24 *W, const void *bias, void *Y,
                              cudaStream_t s);
+
+// Block-sparse weight with 2:4 inside its blocks: compress the kept blocks,
+// forward on the sparse MMA driven by the row-group plan.
+bsl_status launch_bsr24_compress(const bsl_bsr *W, void *values24, uint16_t *meta24, cudaStream_t s);
+bsl_status launch_bsr24_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *values24,
+                            const uint16_t *meta24, const void *bias, void *Y, cudaStream_t s);
 
 bsl_status launch_debug_wait(int32_t *status, uint64_t timeout_ns, cudaStream_t s);
 

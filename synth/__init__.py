@@ -27,6 +27,7 @@ __all__ = [
     "Workload", "WORKLOADS", "bf16_bits", "bits_to_f32", "mask_uniform",
     "zipf_row_counts", "mask_zipf_rows", "make_inputs", "round_half_even",
     "semi24_weight", "Semi24Workload", "SEMI24_WORKLOADS", "make_semi24_inputs",
+    "BSR24_WORKLOADS", "make_bsr24_inputs",
 ]
 
 
@@ -292,4 +293,24 @@ def make_semi24_inputs(w: Semi24Workload, *, M: int | None = None):
         "X": _normal_bf16(np.random.default_rng(w.seed * 10 + 0), (M, w.K), 1.0),
         "W": semi24_weight(w.N, w.K, np.random.default_rng(w.seed * 10 + 2),
                            std=1.0 / math.sqrt(w.K / 2)),
+    }
+
+
+# ---------------------------------------------------------------- block-sparse with 2:4 blocks
+
+BSR24_WORKLOADS: dict[str, Workload] = {w.name: w for w in [
+    Workload("bsr24_fwd", 8192, 14336, 4096, 64, 0.1, 7, mask_kind="zipf",
+             description="LLM-MLP forward, 90% block-sparse (Zipf rows), 2:4 inside the kept blocks"),
+]}
+
+
+def make_bsr24_inputs(w: Workload, *, M: int | None = None):
+    """Seeded X [M,K], block mask and a dense weight W [N,K] with the 2:4
+    pattern along K everywhere (the mask then keeps whole blocks of it), as
+    bf16 bits.  Sub-streams as :func:`make_inputs`: 0 X, 1 mask, 2 W."""
+    M = w.M if M is None else M
+    return {
+        "X": _normal_bf16(np.random.default_rng(w.seed * 10 + 0), (M, w.K), 1.0),
+        "mask": make_mask(w),
+        "W": semi24_weight(w.N, w.K, np.random.default_rng(w.seed * 10 + 2), std=math.sqrt(2.0 / w.K)),
     }

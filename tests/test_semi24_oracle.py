@@ -152,3 +152,29 @@ def test_brute_force_pin_catches_planted_mistakes(name):
         v, m = MUTANTS[name](*oracle.compress24(W))
     bv, bm = brute_compress(W)
     assert not (np.array_equal(v, bv) and np.array_equal(m, bm))
+
+
+def test_block_compression_is_the_dense_compression_restricted_to_blocks():
+    """For a block-sparse weight with 2:4 along K (b a multiple of 16), the
+    compressed form of each kept block is the matching slice of the
+    compressed form of the whole weight with zeros outside the blocks."""
+    b, R, C = 16, 3, 4
+    rng = np.random.default_rng(14)
+    W = synth.semi24_weight(R * b, C * b, rng, fewer=0.3)
+    mask = synth.mask_uniform(R, C, 7, rng)
+    packed = oracle.pack(W, mask, b)
+    v, m = oracle.compress24_blocks(packed["values"])
+    Wz = W.copy()
+    for r in range(R):
+        for c in range(C):
+            if not mask[r, c]:
+                Wz[r * b:(r + 1) * b, c * b:(c + 1) * b] = 0
+    dv, dm = oracle.compress24(Wz)
+    p = 0
+    for r in range(R):
+        for c in range(C):
+            if mask[r, c]:
+                assert np.array_equal(v[p], dv[r * b:(r + 1) * b, c * b // 2:(c + 1) * b // 2])
+                assert np.array_equal(m[p], dm[r * b:(r + 1) * b, c * b // 16:(c + 1) * b // 16])
+                p += 1
+    assert p == packed["nnz"]
