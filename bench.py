@@ -21,7 +21,9 @@ rank's time.
 
 ``--workload semi24_fwd`` measures the 2:4 semi-structured layer instead
 (X[8192,4096], W[14336,4096] with two of every four weights kept, compressed
-once before timing; one step is one forward through bsl_semi24_forward).
+once before timing; one step is one forward through bsl_semi24_forward), and
+``--workload bsr24_fwd`` the block-sparse layer with 2:4 inside its kept
+blocks (the large workload's shape and mask kind; bsl_bsr24_forward).
 """
 from __future__ import annotations
 
@@ -48,6 +50,7 @@ import synth  # noqa: E402
 METRIC = "block-sparse GEMM effective TFLOP/s, % roofline, speedup vs dense at 75/90% sparse"
 UNIT = "TFLOP/s"
 METRIC_SEMI24 = "2:4 semi-structured GEMM TFLOP/s of kept products, % roofline, speedup vs dense"
+METRIC_BSR24 = "block-sparse GEMM with 2:4 blocks, TFLOP/s of kept products, % roofline, speedup vs dense"
 L2_BYTES_DEFAULT = 126 * 2 ** 20
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture
@@ -69,6 +72,9 @@ TRAFFIC = {
     ("semi24_fwd", "fwd"): {"bytes": 503706112, "src_sha": "8514e1e4bf6d7d6f",
                             "files": ["semi24.cu", "common.cuh"],
                             "profile": "profiles/k_semi24_fwd_semi24_fwd.md"},
+    ("bsr24_fwd", "fwd"): {"bytes": 297211904, "src_sha": "64a4794252670688",
+                           "files": ["bsr24.cu", "common.cuh"],
+                           "profile": "profiles/k_bsr24_fwd_bsr24_fwd.md"},
 }
 # the kernel source files each contraction's traffic figure depends on
 TRAFFIC_FILES = {"fwd": ["spmm_tc.cu", "common.cuh"], "fwd_small": ["stream_fwd.cu", "common.cuh"],
@@ -682,9 +688,29 @@ def cpu_sample_semi24(w: synth.Semi24Workload, inp: dict, budget_s: float):
     return float(n) * w.N * w.K, dt, f"fwd: {n} of {w.M} token rows", nthreads
 
 
-def run_gpu_semi24(args):
-    """The 2:4 workload: compress once, then K forwards per step graph, timed
-    like the block-sparse workloads (rotating input copies, CUDA-graph
+def algorithmic_bsr24(w: synth.Workload, nnz: int):
+    """Block-sparse weight with 2:4 blocks: flops of the kept products
+    (2*M*b*b*nnz / 2); bytes X + compressed blocks + their position words +
+    the BSR index + Y."""
+    b, M, N, K = w.b, w.M, w.N, w.K
+    R = N // b
+    return {"flops": M * b * b * nnz,
+            "bytes": M * K * 2 + nnz * b * (b // 2) * 2 + nnz * b * (b // 16) * 2 + (R + 1 + nnz) * 4 + M * N * 2}
+
+
+def cpu_sample_bsr24(w: synth.Workload, inp: dict, budget_s: float):
+    """The oracle's block-skipping forward on a bounded sample of token rows
+    of the 2:4-block workload; flops counted are the kept products
+    (b*b per stored block and token)."""
+    f, secs, desc = cpu_sample_blockskip(w, inp, budget_s)
+    import oracle
+    return f / 2, secs, desc, oracle.num_threads()
+
+
+def run_gpu_2of4(args):
+    """The 2:4 workloads (plain 2:4, and 2:4 inside the blocks of a
+    block-sparse weight): compress once, then K forwards per step graph,
+    timed like the block-sparse workloads (rotating input copies, CUDA-graph
     replays, median over replays, max over ranks)."""
     import torch
     import torch.distributed as dist
@@ -702,37 +728,65 @@ def run_gpu_semi24(args):
     from sparse_gemm_b200 import build as _b
     _b.build()
 
-    w = synth.SEMI24_WORKLOADS[args.workload]
-    inp = synth.make_semi24_inputs(w)
     pk = peaks()
     l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", L2_BYTES_DEFAULT) or L2_BYTES_DEFAULT
 
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    Wd, X0 = dev_bf16(inp["W"]), dev_bf16(inp["X"])
     stream = torch.cuda.current_stream(dev)
-    w0 = sg.compress24(Wd)
+    if args.workload in synth.SEMI24_WORKLOADS:
+        w = synth.SEMI24_WORKLOADS[args.workload]
+        inp = synth.make_semi24_inputs(w)
+        Wd, X0 = dev_bf16(inp["W"]), dev_bf16(inp["X"])
+        compress = lambda out=None: sg.compress24(Wd, out=out)  # noqa: E731
+        forward = lambda x, ww, out=None: sg.forward24(x, ww, out=out)  # noqa: E731
+        status = sg.semi24_status
+        Wdense = Wd
+        alg = algorithmic_semi24(w)
+        wbytes = w.N * (w.K // 2) * 2 + w.N * (w.K // 16) * 2
+        kernel, metric = "k_semi24_fwd", METRIC_SEMI24
+        extra = {"pattern": "2:4 along K"}
+        cpu_fn = cpu_sample_semi24
+        cpu_what = "fp64 loops over the dense weight with zeros in place"
+    else:
+        w = synth.BSR24_WORKLOADS[args.workload]
+        inp = synth.make_bsr24_inputs(w)
+        Wd, X0 = dev_bf16(inp["W"]), dev_bf16(inp["X"])
+        mask = torch.from_numpy(inp["mask"]).to(dev)
+        Wp = sg.pack(Wd, mask, w.b, nnz=w.nnz)
+        compress = lambda out=None: sg.compress_bsr24(Wp, out=out)  # noqa: E731
+        forward = lambda x, ww, out=None: sg.forward_bsr24(x, ww, out=out)  # noqa: E731
+        status = lambda ww: sg.device_status(ww.packed)  # noqa: E731
+        Wdense = Wd * torch.repeat_interleave(torch.repeat_interleave(mask.to(torch.bfloat16), w.b, 0), w.b, 1)
+        alg = algorithmic_bsr24(w, w.nnz)
+        wbytes = w.nnz * w.b * (w.b // 2) * 2 + w.nnz * w.b * (w.b // 16) * 2
+        kernel, metric = "k_bsr24_fwd", METRIC_BSR24
+        extra = {"b": w.b, "nnz": w.nnz, "density": round(w.nnz / (w.R * w.C), 5), "mask": w.mask_kind,
+                 "pattern": "2:4 along K inside the kept blocks"}
+        cpu_fn = cpu_sample_bsr24
+        cpu_what = "fp64 loops over the stored blocks only"
+    w0 = compress()
     torch.cuda.synchronize()
     ce0, ce1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     comp_ms = []
     for _ in range(5):
         ce0.record(stream)
-        sg.compress24(Wd, out=w0)
+        compress(out=w0)
         ce1.record(stream)
         torch.cuda.synchronize()
         comp_ms.append(ce0.elapsed_time(ce1))
-    if sg.semi24_status(w0) != 0:
+    if status(w0) != 0:
         raise RuntimeError("compress reported a device error")
 
-    in_bytes = X0.numel() * 2 + w.N * (w.K // 2) * 2 + w.N * (w.K // 16) * 2
+    in_bytes = X0.numel() * 2 + wbytes
     ncopy = int(min(16, max(2, math.ceil(2 * l2 / in_bytes) + 1)))
     Xs = [X0] + [X0.clone() for _ in range(ncopy - 1)]
-    ws = [w0] + [sg.compress24(Wd) for _ in range(ncopy - 1)]
+    ws = [w0] + [compress() for _ in range(ncopy - 1)]
     Y = torch.empty((w.M, w.N), dtype=torch.bfloat16, device=dev)
 
     def step(i):
-        sg.forward24(Xs[i % ncopy], ws[i % ncopy], out=Y)
+        forward(Xs[i % ncopy], ws[i % ncopy], out=Y)
 
     for i in range(args.warmup):
         step(i)
@@ -783,14 +837,13 @@ def run_gpu_semi24(args):
     clk = clocks.stop()
     fwd_ms = total_ms / K
     total_ms = max_over_ranks(total_ms, world, dev)
-    alg = algorithmic_semi24(w)
     value = whole_job_value(world, alg["flops"], K, total_ms)
     ms_per_step = total_ms / K
 
     # the kept products run at twice the dense rate on the sparse MMA, so the
     # useful-flop peak of the 2:4 kernel is the dense bf16 peak
     roof = roofline_entry("fwd", alg, fwd_ms, pk)
-    roof["kernel"] = "k_semi24_fwd"
+    roof["kernel"] = kernel
     roof["peak_source"] = pk["source"] + (" burst bf16 (useful flops of the 2:4 MMA)"
                                           if roof["unit"] == "TFLOP/s" else " HBM copy")
     tr = TRAFFIC.get((w.name, "fwd"))
@@ -802,7 +855,7 @@ def run_gpu_semi24(args):
                                              / pk["bf16_tflops_sustained"], 4)
 
     # cuBLAS dense on the same weight (zeros in place), same rotation
-    Wds = [Wd] + [Wd.clone() for _ in range(min(ncopy, 3) - 1)]
+    Wds = [Wdense] + [Wdense.clone() for _ in range(min(ncopy, 3) - 1)]
 
     def dense_step(i):
         torch.matmul(Xs[i % ncopy], Wds[i % len(Wds)].t(), out=Y)
@@ -835,7 +888,7 @@ def run_gpu_semi24(args):
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(ev_in[j])
             s_comp.wait_event(ev_out[j])
-            sg.forward24(b["X"], w0, out=b["Y"])
+            forward(b["X"], w0, out=b["Y"])
             ev_comp[j].record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_comp[j])
@@ -858,26 +911,25 @@ def run_gpu_semi24(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1) / ke, world, dev)
     for ww in ws:
-        if sg.semi24_status(ww) != 0:
+        if status(ww) != 0:
             raise RuntimeError("kernels reported a device error")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        done, secs, desc, nthr = cpu_sample_semi24(w, inp, args.cpu_budget)
+        done, secs, desc, nthr = cpu_fn(w, inp, args.cpu_budget)
         cpu = {"value": round(done / secs / 1e12, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
-               "sample": desc + f" ({secs:.1f} s, fp64 loops over the dense weight with zeros in place)",
-               "cpu_model": cpu_model()}
+               "sample": desc + f" ({secs:.1f} s, {cpu_what})", "cpu_model": cpu_model()}
 
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return None
     return {
-        "metric": METRIC_SEMI24, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": metric, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {
-            "workload": w.name, "M": w.M, "N": w.N, "K": w.K, "pattern": "2:4 along K", "seed": w.seed,
+            "workload": w.name, "M": w.M, "N": w.N, "K": w.K, **extra, "seed": w.seed,
             "contractions_per_step": ["fwd"], "global_batch": w.M * world,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "l2": f"rotating {ncopy} copies of every input ({ncopy * in_bytes / 2**20:.0f} MiB > 2x L2)",
@@ -914,8 +966,8 @@ def run_reference(args):
     if rank != 0:
         return None
     per_step = max(0.5, min(20.0, args.reference_budget / max(1, args.steps + args.warmup)))
-    if args.workload in synth.SEMI24_WORKLOADS:
-        return run_reference_semi24(args, world, per_step)
+    if args.workload in synth.SEMI24_WORKLOADS or args.workload in synth.BSR24_WORKLOADS:
+        return run_reference_2of4(args, world, per_step)
     w = synth.WORKLOADS[args.workload]
     inp = synth.make_inputs(w)
     kinds = ["fwd", "dx", "dw"] if w.with_dy else ["fwd"]
@@ -943,29 +995,37 @@ def run_reference(args):
     }
 
 
-def run_reference_semi24(args, world, per_step):
-    """The oracle's 2:4 forward on the host cores, a bounded sample of token
-    rows per step; value is TFLOP/s of kept products."""
-    w = synth.SEMI24_WORKLOADS[args.workload]
-    inp = synth.make_semi24_inputs(w)
+def run_reference_2of4(args, world, per_step):
+    """The oracle's forward of a 2:4 workload on the host cores, a bounded
+    sample of token rows per step; value is TFLOP/s of kept products."""
+    if args.workload in synth.SEMI24_WORKLOADS:
+        w = synth.SEMI24_WORKLOADS[args.workload]
+        inp = synth.make_semi24_inputs(w)
+        fn, metric, what = cpu_sample_semi24, METRIC_SEMI24, "fp64 loops over the dense weight with zeros in place"
+        cfg = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "pattern": "2:4 along K", "seed": w.seed}
+    else:
+        w = synth.BSR24_WORKLOADS[args.workload]
+        inp = synth.make_bsr24_inputs(w)
+        fn, metric, what = cpu_sample_bsr24, METRIC_BSR24, "fp64 loops over the stored blocks only"
+        cfg = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "b": w.b, "nnz": w.nnz,
+               "density": round(w.nnz / (w.R * w.C), 5), "mask": w.mask_kind,
+               "pattern": "2:4 along K inside the kept blocks", "seed": w.seed}
     for _ in range(args.warmup):
-        cpu_sample_semi24(w, inp, per_step)
+        fn(w, inp, per_step)
     done, secs, descs, nthr = 0.0, 0.0, [], 1
     for _ in range(args.steps):
-        d, s_, desc, nthr = cpu_sample_semi24(w, inp, per_step)
+        d, s_, desc, nthr = fn(w, inp, per_step)
         done += d
         secs += s_
         descs.append(desc)
     value = done / secs / 1e12
     return {
-        "impl": "reference", "metric": METRIC_SEMI24, "value": round(value, 8), "unit": UNIT,
+        "impl": "reference", "metric": metric, "value": round(value, 8), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "pattern": "2:4 along K", "seed": w.seed},
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
         "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": nthr, "kind": "oracle",
-                         "sample": descs[0] + " per step (fp64 loops over the dense weight with zeros in place)",
-                         "cpu_model": cpu_model()},
+                         "sample": descs[0] + f" per step ({what})", "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -991,6 +1051,23 @@ def run_kernel_only(args):
             sg.forward24(X, w24)
         torch.cuda.synchronize()
         st = sg.semi24_status(w24)
+        if st != 0:
+            raise RuntimeError(f"device status {st}")
+        print(json.dumps({"kernel_only": "fwd", "workload": w.name, "reps": args.reps}))
+        return
+    if args.workload in synth.BSR24_WORKLOADS:
+        if args.kernel_only != "fwd":
+            raise SystemExit("the 2:4-block workload has a forward only")
+        w = synth.BSR24_WORKLOADS[args.workload]
+        inp = synth.make_bsr24_inputs(w)
+        bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        Wp = sg.pack(bits(inp["W"]), torch.from_numpy(inp["mask"]).to(dev), w.b, nnz=w.nnz)
+        w24 = sg.compress_bsr24(Wp)
+        X = bits(inp["X"])
+        for _ in range(args.reps):
+            sg.forward_bsr24(X, w24)
+        torch.cuda.synchronize()
+        st = sg.device_status(Wp)
         if st != 0:
             raise RuntimeError(f"device status {st}")
         print(json.dumps({"kernel_only": "fwd", "workload": w.name, "reps": args.reps}))
@@ -1026,7 +1103,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_fwd",
-                    choices=sorted(synth.WORKLOADS) + sorted(synth.SEMI24_WORKLOADS))
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.SEMI24_WORKLOADS)
+                    + sorted(synth.BSR24_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
     ap.add_argument("--reference-budget", type=float, default=120.0)
@@ -1042,8 +1120,8 @@ def main():
         return
     if args.impl == "reference":
         out = run_reference(args)
-    elif args.workload in synth.SEMI24_WORKLOADS:
-        out = run_gpu_semi24(args)
+    elif args.workload in synth.SEMI24_WORKLOADS or args.workload in synth.BSR24_WORKLOADS:
+        out = run_gpu_2of4(args)
     else:
         out = run_gpu(args)
     if out is not None:

@@ -61,7 +61,8 @@ def test_reported_bound(name, kind, bound):
 
 def test_traffic_entries_name_their_sources():
     for (wname, kind), t in bench.TRAFFIC.items():
-        assert (wname in synth.WORKLOADS or wname in synth.SEMI24_WORKLOADS) and kind in ("fwd", "dx", "dw")
+        assert (wname in synth.WORKLOADS or wname in synth.SEMI24_WORKLOADS or wname in synth.BSR24_WORKLOADS) \
+            and kind in ("fwd", "dx", "dw")
         assert t["bytes"] > 0 and len(t["src_sha"]) == 16
         assert os.path.exists(os.path.join(ROOT, t["profile"]))
         for f in t["files"]:
@@ -77,3 +78,14 @@ def test_semi24_work_bytes_and_bound():
     assert alg["flops"] == 2 * w.M * w.N * (w.K // 2)
     assert alg["bytes"] == w.M * w.K * 2 + w.N * w.K + w.N * w.K // 8 + w.M * w.N * 2
     assert bench.roofline_entry("fwd", alg, 0.5, PEAKS)["bound"] == "tensor"
+
+
+def test_bsr24_work_and_bytes():
+    """2:4 inside blocks: kept products M*b*b*nnz; bytes X + compressed blocks
+    (b*b/2 values and b*b/16 words each) + BSR index + Y."""
+    w = synth.BSR24_WORKLOADS["bsr24_fwd"]
+    alg = bench.algorithmic_bsr24(w, w.nnz)
+    assert alg["flops"] == bench.algorithmic(w, w.nnz)["fwd"]["flops"] // 2
+    b, R = w.b, w.N // w.b
+    assert alg["bytes"] == (w.M * w.K * 2 + w.nnz * b * b + w.nnz * b * b // 8 + (R + 1 + w.nnz) * 4
+                            + w.M * w.N * 2)
