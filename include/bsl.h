@@ -291,9 +291,8 @@ BSL_API bsl_status bsl_bsr24_compress(const bsl_bsr *W, void *values24, uint16_t
 /* Y [M][N] = X [M][K] . W~^T (+ bias), W~ the block-sparse weight with zeros
  * outside its blocks, the blocks read from values24 / meta24 (the dense
  * product with zeros in place: torchao README, introduction).  bf16 in, fp32
- * accumulation, bias bf16 [N] or NULL.  b must be 64 (BSL_ERR_UNSUPPORTED
- * otherwise).  Sparse tensor-core kernel driven by W's row-group plan,
- * persistent, one CTA per SM. */
+ * accumulation, bias bf16 [N] or NULL.  b = 32 or 64.  Sparse tensor-core
+ * kernel driven by W's row-group plan, persistent, one CTA per SM. */
 BSL_API bsl_status bsl_bsr24_forward(const void *X, int32_t M, const bsl_bsr *W, const void *values24,
                                      const uint16_t *meta24, const void *bias, void *Y, void *stream);
 

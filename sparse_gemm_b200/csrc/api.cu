@@ -192,6 +192,7 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                                         : CU_TENSOR_MAP_SWIZZLE_NONE;
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -214,6 +215,7 @@ bool make_map_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, u
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                                         : CU_TENSOR_MAP_SWIZZLE_NONE;
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -439,7 +441,6 @@ bsl_status bsl_bsr24_forward(const void *X, int32_t M, const bsl_bsr *W, const v
                              const uint16_t *meta24, const void *bias, void *Y, void *stream)
 {
     BSL_TRY(check_bsr(W));
-    if (W->b != 64) return BSL_ERR_UNSUPPORTED;
     if (M <= 0 || check_matrix(X, M) != BSL_OK || check_matrix(Y, M) != BSL_OK) return BSL_ERR_INVALID_ARG;
     if (!values24 || !aligned(values24, 16) || (W->nnz > 0 && (!meta24 || !aligned(meta24, 16))))
         return BSL_ERR_INVALID_ARG;

@@ -18,7 +18,8 @@
 // 224 tokens.  Per entry one stage holds the members' compressed blocks (a
 // zero block for absent members), the activation tile X[t0:t0+224, c*b:(c+1)*b]
 // and the present members' position words, all by TMA.  b = 64: 2 members,
-// two K = 32 MMAs of N = 224 per entry.  Persistent, one CTA per SM; tiles
+// two K = 32 MMAs of N = 224 per entry, 64-byte weight rows; b = 32: 4
+// members, one MMA per entry, 32-byte weight rows (32-byte swizzle).  Persistent, one CTA per SM; tiles
 // token-tile major, every group (heaviest first) inside, taken round robin.
 // Roles (16 warps):
 //   warp 2      plan: reads each tile's plan 32 entries at a time (lane i
@@ -53,20 +54,27 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+constexpr int kBsr24Tokens = 224;  // tokens per tile (MMA N)
+
+template <int B_>
 struct Bsr24Cfg {
-    static constexpr int B = 64;                     // block size
+    static constexpr int B = B_;                     // block size: 64 or 32
     static constexpr int G = 128 / B;                // block rows per group
-    static constexpr int BT = 224;                   // tokens per tile (MMA N)
-    static constexpr int S = 5;                      // copy stages, one entry each
-    static constexpr int A_BLOCK = B * (B / 2) * 2;  // one compressed block: B rows x B/2 bf16
-    static constexpr int A_BYTES = G * A_BLOCK;      // 128 rows x 64 B
-    static constexpr int B_BYTES = BT * B * 2;       // 224 rows x 128 B
+    static constexpr int KSTEPS = B / 32;            // K = 32 sparse MMAs per entry
+    static constexpr int BT = kBsr24Tokens;
+    static constexpr int S = B == 64 ? 5 : 8;        // copy stages, one entry each
+    static constexpr int A_ROW = B;                  // bytes of a compressed block row (B/2 bf16)
+    static constexpr uint32_t A_LAYOUT = B == 64 ? kLayoutSw64 : kLayoutSw32;
+    static constexpr uint32_t X_LAYOUT = B == 64 ? kLayoutSw128 : kLayoutSw64;
+    static constexpr int A_BLOCK = B * A_ROW;        // one compressed block
+    static constexpr int A_BYTES = G * A_BLOCK;      // 128 rows
+    static constexpr int B_BYTES = BT * B * 2;       // 224 rows of B activations
     static constexpr int META_BLOCK = B * (B / 16) * 2;  // one block's position words
     static constexpr int META_OFF = A_BYTES + B_BYTES;
     static constexpr int HDR_OFF = META_OFF + G * META_BLOCK;
     static constexpr int STAGE_BYTES = (HDR_OFF + 16 + 1023) / 1024 * 1024;
     static constexpr int MS = 8;                     // metadata ring stages (TMEM)
-    static constexpr int MCOLS = 8;                  // TMEM columns per metadata stage
+    static constexpr int MCOLS = 4 * KSTEPS;         // TMEM columns per metadata stage
     static constexpr int ACC = 2;                    // accumulator buffers
     static constexpr int META_COL = ACC * BT;
     static constexpr int TMEM_COLS = 512;
@@ -87,7 +95,7 @@ struct Bsr24Cfg {
     static_assert(META_COL + MCOLS * MS <= TMEM_COLS, "TMEM columns");
     static_assert((2 * S + 2 * MS + 2 * ACC + 2 * D + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-    static_assert(B == 64, "the K = 32 steps and the 64-byte operand rows assume b = 64");
+    static_assert(B == 64 || B == 32, "block size");
 };
 
 struct Bsr24Args {
@@ -138,7 +146,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 // running at one time work on one or two token tiles across every group, so
 // the activations they read (a few MB) and the compressed weight stay in L2.
 __device__ __forceinline__ int tile_group(int t, const Bsr24Args &a) { return t % a.ngroups; }
-__device__ __forceinline__ int tile_token0(int t, const Bsr24Args &a) { return (t / a.ngroups) * Bsr24Cfg::BT; }
+__device__ __forceinline__ int tile_token0(int t, const Bsr24Args &a) { return (t / a.ngroups) * kBsr24Tokens; }
 
 // Entries of tile t's group (0 past the last tile).
 __device__ __forceinline__ int tile_entries(int t, const Bsr24Args &a)
@@ -148,19 +156,20 @@ __device__ __forceinline__ int tile_entries(int t, const Bsr24Args &a)
     return __ldg(a.grp_ptr + grp + 1) - __ldg(a.grp_ptr + grp);
 }
 
-// Block row of member m of tile t's group, or -1 (no such member or tile).
-__device__ __forceinline__ int tile_block_row(int t, int m, const Bsr24Args &a)
+// Block row of member m of tile t's group (G members), or -1 (no such member or tile).
+__device__ __forceinline__ int tile_block_row(int t, int m, int G, const Bsr24Args &a)
 {
     if (t >= a.tiles) return -1;
-    const int gi = tile_group(t, a) * Bsr24Cfg::G + m;
+    const int gi = tile_group(t, a) * G + m;
     return gi < a.R ? __ldg(a.row_order + gi) : -1;
 }
 
-__global__ void __launch_bounds__(Bsr24Cfg::THREADS, 1)
+template <int B>
+__global__ void __launch_bounds__(Bsr24Cfg<B>::THREADS, 1)
     k_bsr24_fwd(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
                 const __grid_constant__ CUtensorMap tmY, const uint8_t *__restrict__ meta, const Bsr24Args args)
 {
-    using C = Bsr24Cfg;
+    using C = Bsr24Cfg<B>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *stages = align1024(smem_raw);
     uint8_t *outbuf = stages + C::S * C::STAGE_BYTES;
@@ -387,9 +396,9 @@ __global__ void __launch_bounds__(Bsr24Cfg::THREADS, 1)
                 const uint32_t a_base = smem_u32(stages + slot * C::STAGE_BYTES);
                 const uint32_t b_base = a_base + C::A_BYTES;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint64_t ad = make_sdesc(a_base + j * 32, 16, 512, kLayoutSw64);
-                    const uint64_t bd = make_sdesc(b_base + j * 64, 16, 1024, kLayoutSw128);
+                for (int j = 0; j < C::KSTEPS; ++j) {
+                    const uint64_t ad = make_sdesc(a_base + j * 32, 16, 8 * C::A_ROW, C::A_LAYOUT);
+                    const uint64_t bd = make_sdesc(b_base + j * 64, 16, 8 * 2 * C::B, C::X_LAYOUT);
                     umma_sp_lead(lead, tmem + acc * C::BT, ad, bd, tmem + C::META_COL + ms * C::MCOLS + j * 4,
                                  idesc, (k | j) != 0);
                 }
@@ -414,15 +423,15 @@ __global__ void __launch_bounds__(Bsr24Cfg::THREADS, 1)
         __syncwarp();
     } else if (warp >= C::W_META && warp < C::W_META + 4) {
         // ------------------------------------------------------------ metadata
-        // Warp q covers TMEM lanes 32q .. 32q+31: member m = q / 2, rows
-        // 32(q % 2) .. 32(q % 2)+31 of its block.  Lane l reads its row's
-        // 8 bytes of position words (K 0..63 of the entry), then takes the
-        // 16-bit halves its TMEM lane holds from lanes src_lo / src_hi.
-        const int q = warp & 3, m = q >> 1;
-        const int row = (q & 1) * 32 + lane;
+        // Warp q covers TMEM lanes 32q .. 32q+31: member m = 32q / b, rows
+        // 32q % b .. +31 of its block.  Lane l reads its row's b/8 bytes of
+        // position words (one 32-bit word per K = 32 step of the entry), then
+        // takes the 16-bit halves its TMEM lane holds from lanes src_lo / src_hi.
+        const int q = warp & 3, m = (32 * q) / B;
+        const int row = (32 * q) % B + lane;
         const int src_lo = (lane & 16) | (lane & 7), src_hi = src_lo + 8;
         const bool upper = (lane >> 3) & 1;
-        const uint2 pad = make_uint2(0x44444444u, 0x44444444u);  // absent member: pairs (0, 1) over zeros
+        constexpr uint32_t pad = 0x44444444u;  // absent member: pairs (0, 1) over zeros
         bool ok = true;
         int g = 0;
         int nent_next = tile_entries(blockIdx.x, args);
@@ -437,13 +446,13 @@ __global__ void __launch_bounds__(Bsr24Cfg::THREADS, 1)
                 }
                 const uint8_t *st = stages + slot * C::STAGE_BYTES;
                 const uint32_t mj = *reinterpret_cast<const volatile uint32_t *>(st + C::HDR_OFF);
-                const uint2 v = ((mj >> m) & 1u)
-                                    ? *reinterpret_cast<const uint2 *>(st + C::META_OFF + m * C::META_BLOCK + row * 8)
-                                    : pad;
-                uint32_t w[2];
+                const uint32_t *src =
+                    reinterpret_cast<const uint32_t *>(st + C::META_OFF + m * C::META_BLOCK + row * (B / 8));
+                const bool present = (mj >> m) & 1u;
+                uint32_t w[C::KSTEPS];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint32_t x = j ? v.y : v.x;
+                for (int j = 0; j < C::KSTEPS; ++j) {
+                    const uint32_t x = present ? src[j] : pad;
                     const uint32_t lo = __shfl_sync(0xffffffffu, x, src_lo);
                     const uint32_t hi = __shfl_sync(0xffffffffu, x, src_hi);
                     w[j] = (upper ? lo >> 16 : lo & 0xFFFFu) | (upper ? hi & 0xFFFF0000u : hi << 16);
@@ -455,8 +464,8 @@ __global__ void __launch_bounds__(Bsr24Cfg::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + C::META_COL + ms * C::MCOLS;
-                tmem_st1(taddr, w[0]);
-                tmem_st1(taddr + 4, w[1]);
+#pragma unroll
+                for (int j = 0; j < C::KSTEPS; ++j) tmem_st1(taddr + 4 * j, w[j]);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -480,15 +489,15 @@ __global__ void __launch_bounds__(Bsr24Cfg::THREADS, 1)
         bool ok = true;
         int it = 0, ob = 0;
         int nent_next = tile_entries(blockIdx.x, args);
-        int row_next = tile_block_row(blockIdx.x, q >> 1, args);
+        int row_next = tile_block_row(blockIdx.x, (32 * q) / B, C::G, args);
         for (int t = blockIdx.x; ok && t < args.tiles; t += gridDim.x, ++it) {
             const int t0 = tile_token0(t, args);
             const int nent = nent_next, brow = row_next;
             nent_next = tile_entries(t + gridDim.x, args);  // used one tile later
-            row_next = tile_block_row(t + gridDim.x, q >> 1, args);
+            row_next = tile_block_row(t + gridDim.x, (32 * q) / B, C::G, args);
             const int acc = it & 1;
             const bool member = brow >= 0;
-            const int f0 = member ? brow * C::B + (q & 1) * 32 : 0;
+            const int f0 = member ? brow * C::B + (32 * q) % B : 0;
             const float bv = (args.bias && member) ? __bfloat162float(args.bias[f0 + lane]) : 0.f;
             const int left = args.M - t0;
             const int nch = left >= C::BT ? C::BT / 32 : (left + 31) / 32;
@@ -557,12 +566,13 @@ __global__ void __launch_bounds__(Bsr24Cfg::THREADS, 1)
 }
 
 // Compressed blocks [nnz + 1][b][b/2] bf16 (the last one zero) as a 3-D map:
-// x = kept value in a row, y = row in the block, z = block; 64-byte swizzle.
+// x = kept value in a row, y = row in the block, z = block; the rows are b
+// bytes, swizzled over b bytes.
 bool make_block24_map(CUtensorMap *map, const void *values, int32_t b, int32_t nblocks)
 {
     return make_map_3d(map, values, static_cast<uint64_t>(b) / 2, static_cast<uint64_t>(b),
                        static_cast<uint64_t>(nblocks), static_cast<uint64_t>(b),
-                       static_cast<uint64_t>(b) * b, static_cast<uint32_t>(b) / 2, static_cast<uint32_t>(b), 64);
+                       static_cast<uint64_t>(b) * b, static_cast<uint32_t>(b) / 2, static_cast<uint32_t>(b), b);
 }
 
 }  // namespace
@@ -585,19 +595,21 @@ bsl_status launch_bsr24_compress(const bsl_bsr *W, void *values24, uint16_t *met
     return cuda_status(cudaMemsetAsync(static_cast<uint8_t *>(values24) + W->nnz * block_bytes, 0, block_bytes, s));
 }
 
-bsl_status launch_bsr24_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *values24,
-                            const uint16_t *meta24, const void *bias, void *Y, cudaStream_t s)
+namespace {
+
+template <int B>
+bsl_status run_bsr24(const void *X, int32_t M, const bsl_bsr *W, const void *values24, const uint16_t *meta24,
+                     const void *bias, void *Y, cudaStream_t s)
 {
-    using C = Bsr24Cfg;
-    if (W->b != C::B) return BSL_ERR_UNSUPPORTED;
+    using C = Bsr24Cfg<B>;
     CUtensorMap ma, mx, my;
-    if (!make_block24_map(&ma, values24, W->b, W->nnz + 1) ||
-        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, C::B, C::BT, 128) ||
+    if (!make_block24_map(&ma, values24, B, W->nnz + 1) ||
+        !make_map_2d(&mx, X, W->K, M, static_cast<uint64_t>(W->K) * 2, B, C::BT, 2 * B) ||
         !make_map_2d(&my, Y, W->N, M, static_cast<uint64_t>(W->N) * 2, 32, 32, 0))
         return BSL_ERR_CUDA;
     Bsr24Args args;
     args.M = M;
-    args.R = W->N / W->b;
+    args.R = W->N / B;
     args.nnz = W->nnz;
     args.ntt = (M + C::BT - 1) / C::BT;
     args.ngroups = (args.R + C::G - 1) / C::G;
@@ -612,12 +624,22 @@ bsl_status launch_bsr24_fwd(const void *X, int32_t M, const bsl_bsr *W, const vo
     args.bias = static_cast<const __nv_bfloat16 *>(bias);
     args.status = W->status;
     args.timeout_ns = wait_timeout_ns();
-    const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(k_bsr24_fwd), C::SMEM_BYTES);
+    auto kern = k_bsr24_fwd<B>;
+    const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (sa != BSL_OK) return sa;
     const int grid = args.tiles < num_sms() ? args.tiles : num_sms();
-    k_bsr24_fwd<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ma, mx, my, reinterpret_cast<const uint8_t *>(meta24),
-                                                         args);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ma, mx, my, reinterpret_cast<const uint8_t *>(meta24), args);
     return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+bsl_status launch_bsr24_fwd(const void *X, int32_t M, const bsl_bsr *W, const void *values24,
+                            const uint16_t *meta24, const void *bias, void *Y, cudaStream_t s)
+{
+    if (W->b == 64) return run_bsr24<64>(X, M, W, values24, meta24, bias, Y, s);
+    if (W->b == 32) return run_bsr24<32>(X, M, W, values24, meta24, bias, Y, s);
+    return BSL_ERR_UNSUPPORTED;
 }
 
 }  // namespace bsl

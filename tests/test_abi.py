@@ -131,6 +131,6 @@ def test_bsr24_entry_points_check_arguments_on_host(lib):
     assert lib.bsl_bsr24_forward(4096, 64, ctypes.byref(s), 0, 4096, None, 4096, None) == 1     # null values24
     assert lib.bsl_bsr24_forward(4096, 64, ctypes.byref(s), 4096, 4100, None, 4096, None) == 1  # misaligned meta
     assert lib.bsl_bsr24_forward(4096, 0, ctypes.byref(s), 4096, 4096, None, 4096, None) == 1   # M = 0
-    assert lib.bsl_bsr24_forward(4096, 64, ctypes.byref(_bsr(b=32)), 4096, 4096, None, 4096, None) == 2
+    assert lib.bsl_bsr24_forward(4096, 64, ctypes.byref(_bsr(b=48)), 4096, 4096, None, 4096, None) == 2
     assert lib.bsl_bsr24_compress(ctypes.byref(s), 4104, 4096, None) == 1                         # misaligned
     assert lib.bsl_bsr24_compress(ctypes.byref(_bsr(b=48)), 4096, 4096, None) == 2

@@ -3,11 +3,11 @@
 The compressed blocks must match the oracle bit for bit (block by block, the
 zero block after them); the forward must match the oracle's block-sparse
 product (the dense product with zeros outside the kept blocks) element by
-element within the bound of tests/_parity.py.  Cases: one token, ragged
-token tiles (224 tokens per tile), empty block rows (a group without
-entries, whose rows must come out as the bias alone), an odd number of block
-rows (the last group has one member), more tiles than SMs, and the full
-workload on sampled rows.
+element within the bound of tests/_parity.py.  Cases, for block sizes 64
+and 32: one token, ragged token tiles (224 tokens per tile), empty block rows
+(a group without entries, whose rows must come out as the bias alone), a
+block-row count that leaves the last group short, more tiles than SMs, and
+the full workload on sampled rows.
 """
 import numpy as np
 import pytest
@@ -22,12 +22,10 @@ pytestmark = pytest.mark.gpu
 
 sg = pytest.importorskip("sparse_gemm_b200")
 
-B = 64
 
-
-def case(M, N, K, nnz, seed, *, empty_rows=(), fewer=0.2):
+def case(M, N, K, nnz, seed, *, b=64, empty_rows=(), fewer=0.2):
     rng = np.random.default_rng(seed)
-    mask = synth.mask_uniform(N // B, K // B, nnz, rng)
+    mask = synth.mask_uniform(N // b, K // b, nnz, rng)
     for r in empty_rows:
         mask[r, :] = 0
     W = synth.semi24_weight(N, K, rng, std=(2.0 / K) ** 0.5, fewer=fewer)
@@ -36,8 +34,8 @@ def case(M, N, K, nnz, seed, *, empty_rows=(), fewer=0.2):
     return X, W, mask, bias
 
 
-def run(X, W, mask, bias=None):
-    Wp = sg.pack(to_dev(W), mask_dev(mask), B)
+def run(X, W, mask, bias=None, b=64):
+    Wp = sg.pack(to_dev(W), mask_dev(mask), b)
     w24 = sg.compress_bsr24(Wp)
     Y = sg.forward_bsr24(to_dev(X), w24, bias=None if bias is None else to_dev(bias))
     torch.cuda.synchronize()
@@ -45,8 +43,8 @@ def run(X, W, mask, bias=None):
     return Wp, w24, Y
 
 
-def check_blocks(W, mask, w24):
-    packed = oracle.pack(W, mask, B)
+def check_blocks(W, mask, w24, b=64):
+    packed = oracle.pack(W, mask, b)
     v, m = oracle.compress24_blocks(packed["values"])
     nnz = packed["nnz"]
     got_v = bits(w24.values)
@@ -57,47 +55,41 @@ def check_blocks(W, mask, w24):
 
 
 FWD_CASES = [
-    # M, N, K, nnz, bias, empty block rows, seed
-    (1, 256, 256, 5, False, (), 30),
-    (225, 512, 384, 20, True, (), 31),
-    (300, 640, 1024, 40, True, (0, 1, 6), 32),   # block rows 0 and 1 form an empty group
-    (448, 320, 512, 12, False, (), 33),          # 5 block rows: the last group has one member
-    (5000, 1024, 512, 60, True, (), 34),         # 8 groups x 23 token tiles > SMs
+    # b, M, N, K, nnz, bias, empty block rows, seed
+    (64, 1, 256, 256, 5, False, (), 30),
+    (64, 225, 512, 384, 20, True, (), 31),
+    (64, 300, 640, 1024, 40, True, (0, 1, 6), 32),  # block rows 0 and 1 form an empty group
+    (64, 448, 320, 512, 12, False, (), 33),         # 5 block rows: the last group has one member
+    (64, 5000, 1024, 512, 60, True, (), 34),        # 8 groups x 23 token tiles > SMs
+    (32, 1, 128, 128, 5, False, (), 40),
+    (32, 225, 512, 384, 60, True, (), 41),
+    (32, 300, 640, 1024, 120, True, (0, 1, 2, 3, 9), 42),  # rows 0-3: an empty group of four
+    (32, 448, 224, 512, 30, False, (), 43),         # 7 block rows: the last group has three members
+    (32, 5000, 2048, 256, 200, True, (), 44),       # 16 groups x 23 token tiles > SMs
 ]
 
 
-@pytest.mark.parametrize("M,N,K,nnz,with_bias,empty,seed", FWD_CASES)
-def test_forward_parity(M, N, K, nnz, with_bias, empty, seed):
-    X, W, mask, bias = case(M, N, K, nnz, seed, empty_rows=empty)
-    Wp, w24, Y = run(X, W, mask, bias if with_bias else None)
-    check_blocks(W, mask, w24)
-    ref, refabs = oracle.forward(X, W, mask, B, bias=bias if with_bias else None)
-    assert_parity(to_f64(Y), ref, refabs, f"2:4-block forward M={M} N={N} K={K} nnz={nnz}")
+@pytest.mark.parametrize("b,M,N,K,nnz,with_bias,empty,seed", FWD_CASES)
+def test_forward_parity(b, M, N, K, nnz, with_bias, empty, seed):
+    X, W, mask, bias = case(M, N, K, nnz, seed, b=b, empty_rows=empty)
+    Wp, w24, Y = run(X, W, mask, bias if with_bias else None, b=b)
+    check_blocks(W, mask, w24, b=b)
+    ref, refabs = oracle.forward(X, W, mask, b, bias=bias if with_bias else None)
+    assert_parity(to_f64(Y), ref, refabs, f"2:4-block forward b={b} M={M} N={N} K={K} nnz={nnz}")
 
 
 def test_compress_reports_groups_with_more_than_two_nonzeros():
     X, W, mask, _ = case(8, 256, 256, 6, 35)
     r, c = np.argwhere(mask)[0]
-    W[r * B + 3, c * B + 8:c * B + 12] = [0x3F80, 0x4000, 0xBF80, 0]
-    Wp = sg.pack(to_dev(W), mask_dev(mask), B)
+    W[r * 64 + 3, c * 64 + 8:c * 64 + 12] = [0x3F80, 0x4000, 0xBF80, 0]
+    Wp = sg.pack(to_dev(W), mask_dev(mask), 64)
     sg.compress_bsr24(Wp)
     assert sg.device_status(Wp) == 8  # BSL_ERR_NOT_2_4
 
 
-def test_block_size_32_is_unsupported():
-    rng = np.random.default_rng(36)
-    mask = synth.mask_uniform(4, 4, 5, rng)
-    W = synth.semi24_weight(128, 128, rng)
-    Wp = sg.pack(to_dev(W), mask_dev(mask), 32)
-    w24 = sg.compress_bsr24(Wp)
-    X = to_dev(synth.bf16_bits(rng.standard_normal((16, 128)).astype(np.float32)))
-    with pytest.raises(sg.BslError, match="UNSUPPORTED"):
-        sg.forward_bsr24(X, w24)
-
-
 def test_deterministic_and_replays_from_a_cuda_graph():
     X, W, mask, bias = case(700, 768, 1024, 50, 37)
-    Wp = sg.pack(to_dev(W), mask_dev(mask), B)
+    Wp = sg.pack(to_dev(W), mask_dev(mask), 64)
     w24 = sg.compress_bsr24(Wp)
     Xd, bd = to_dev(X), to_dev(bias)
     Y1 = sg.forward_bsr24(Xd, w24, bias=bd)
@@ -127,5 +119,5 @@ def test_full_workload_sampled_rows():
     Wp, w24, Y = run(X, W, mask)
     check_blocks(W, mask, w24)
     rows = sorted({r for t in range(0, wl.M, 224) for r in (t, min(t + 223, wl.M - 1))})
-    ref, refabs = oracle.forward(X, W, mask, B, rows=np.asarray(rows))
+    ref, refabs = oracle.forward(X, W, mask, wl.b, rows=np.asarray(rows))
     assert_parity(to_f64(Y[rows]), ref, refabs, "2:4-block forward, full size, sampled rows")
