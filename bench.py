@@ -72,7 +72,7 @@ TRAFFIC = {
     ("semi24_fwd", "fwd"): {"bytes": 503706112, "src_sha": "8514e1e4bf6d7d6f",
                             "files": ["semi24.cu", "common.cuh"],
                             "profile": "profiles/k_semi24_fwd_semi24_fwd.md"},
-    ("bsr24_fwd", "fwd"): {"bytes": 297211904, "src_sha": "64a4794252670688",
+    ("bsr24_fwd", "fwd"): {"bytes": 296873984, "src_sha": "ecebceabf4a22b60",
                            "files": ["bsr24.cu", "common.cuh"],
                            "profile": "profiles/k_bsr24_fwd_bsr24_fwd.md"},
 }

@@ -56,6 +56,10 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p)
 
 constexpr int kBsr24Tokens = 224;  // tokens per tile (MMA N)
 
+// Shared-memory descriptor layout code of the 32-byte swizzle (the b = 32
+// compressed rows are 32 bytes); 64- and 128-byte are kLayoutSw64 / kLayoutSw128.
+constexpr uint32_t kLayoutSw32 = 6;
+
 template <int B_>
 struct Bsr24Cfg {
     static constexpr int B = B_;                     // block size: 64 or 32

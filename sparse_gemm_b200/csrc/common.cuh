@@ -304,8 +304,8 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn, 
 }
 
 // Shared-memory matrix descriptor (sm_100 version 1).  Layout codes:
-// 2 = 128-byte swizzle, 4 = 64-byte swizzle, 6 = 32-byte swizzle.  lbo / sbo in bytes.
-enum : uint32_t { kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6 };
+// 2 = 128-byte swizzle, 4 = 64-byte swizzle.  lbo / sbo in bytes.
+enum : uint32_t { kLayoutSw128 = 2, kLayoutSw64 = 4 };
 
 __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout)
 {
