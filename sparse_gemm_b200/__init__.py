@@ -25,7 +25,7 @@ __all__ = [
     "device_status", "set_wait_timeout_us", "debug_wait_timeout", "small_m_max",
     "forward_stream_noalloc", "bias_grad",
     "BlockSparseLinearFunction", "BlockSparseLinear",
-    "Semi24Weight", "compress24", "forward24", "semi24_status",
+    "Semi24Weight", "compress24", "forward24", "semi24_status", "Semi24Linear",
     "Bsr24Weight", "compress_bsr24", "forward_bsr24",
 ]
 
@@ -496,6 +496,44 @@ def semi24_status(w: Semi24Weight) -> int:
     _check(library().bsl_semi24_get_status(w.cref(), ctypes.byref(out), _stream(w.values)),
            "bsl_semi24_get_status")
     return int(out.value)
+
+
+class Semi24Linear(torch.nn.Module):
+    """Inference ``nn.Linear`` with a 2:4 semi-structured weight: the torchao
+    sparsity README's flow (introduction and its example) converts a trained
+    linear layer's weight, pruned to two nonzeros in every four along K, into
+    the compressed form and multiplies with the sparse tensor cores.  Built
+    with :meth:`from_dense`; inputs may have any leading dimensions."""
+
+    def __init__(self, weight24: Semi24Weight, bias: torch.Tensor | None = None):
+        super().__init__()
+        self.weight24 = weight24
+        self.in_features, self.out_features = weight24.K, weight24.N
+        if bias is not None:
+            if bias.shape != (weight24.N,):
+                raise ValueError("bias must have out_features entries")
+            bias = bias.detach().to(device=weight24.device, dtype=torch.bfloat16).contiguous()
+        self.register_buffer("bias", bias)
+
+    @classmethod
+    def from_dense(cls, weight: torch.Tensor, bias: torch.Tensor | None = None) -> "Semi24Linear":
+        """Compress a [out_features, in_features] weight with at most two
+        nonzeros in every group of four along in_features; raises BslError
+        (BSL_ERR_NOT_2_4) if a group holds more."""
+        w24 = compress24(weight.detach().to(torch.bfloat16).contiguous())
+        st = semi24_status(w24)
+        if st != 0:
+            raise BslError(st, "Semi24Linear.from_dense")
+        return cls(w24, bias)
+
+    @torch.no_grad()
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        x2 = x.reshape(-1, self.in_features)
+        if x2.dtype != torch.bfloat16:
+            x2 = x2.to(torch.bfloat16)
+        y = forward24(x2.contiguous(), self.weight24, bias=self.bias)
+        return y.reshape(*lead, self.out_features)
 
 
 # ---------------------------------------------------------------- 2:4 inside blocks

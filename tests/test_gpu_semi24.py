@@ -133,3 +133,21 @@ def test_full_workload_sampled_rows():
     v, m = oracle.compress24(W)
     ref, refabs = oracle.semi24_forward(X, v, m, rows=np.asarray(rows))
     assert_parity(to_f64(Y[rows]), ref, refabs, "semi24 forward, full size, sampled rows")
+
+
+def test_semi24_linear_module():
+    """The inference module: leading dimensions kept, bias added, output equal
+    to the oracle within the bound; a weight that is not 2:4 is refused."""
+    rng = np.random.default_rng(22)
+    W = synth.semi24_weight(136, 192, rng, std=0.1)
+    bias = synth.bf16_bits(rng.standard_normal(136).astype(np.float32))
+    X = synth.bf16_bits(rng.standard_normal((2 * 3 * 5, 192)).astype(np.float32))
+    mod = sg.Semi24Linear.from_dense(to_dev(W), bias=to_dev(bias))
+    y = mod(to_dev(X).reshape(2, 3, 5, 192))
+    assert y.shape == (2, 3, 5, 136)
+    ref, refabs = oracle.semi24_forward(X, *oracle.compress24(W), bias=bias)
+    assert_parity(to_f64(y.reshape(30, 136)), ref, refabs, "Semi24Linear")
+    bad = W.copy()
+    bad[0, 0:4] = [0x3F80, 0x3F80, 0x3F80, 0]
+    with pytest.raises(sg.BslError, match="NOT_2_4"):
+        sg.Semi24Linear.from_dense(to_dev(bad))
