@@ -58,23 +58,17 @@ L2_BYTES_DEFAULT = 126 * 2 ** 20
 # entry is only used while the kernel source still hashes to `src_sha`.
 TRAFFIC = {
     ("large_fwd", "fwd"): {"bytes": 287450112, "src_sha": "e4c02bbc81127eb7",
-                           "files": ["spmm_tc.cu", "common.cuh"],
-                           "profile": "profiles/k_spmm_tc_fwd_large_fwd.md"},
+                           "files": ["spmm_tc.cu", "common.cuh"]},
     ("decode_fwd", "fwd"): {"bytes": 22774528, "src_sha": "ea9cb22b798b0cf0",
-                            "files": ["stream_fwd.cu", "common.cuh"],
-                            "profile": "profiles/k_stream_fwd_decode_fwd.md"},
+                            "files": ["stream_fwd.cu", "common.cuh"]},
     ("enc_train_d1.0", "dx"): {"bytes": 29975296, "src_sha": "e4c02bbc81127eb7",
-                               "files": ["spmm_tc.cu", "common.cuh"],
-                               "profile": "profiles/k_spmm_tc_dx_enc_train_d1.md"},
+                               "files": ["spmm_tc.cu", "common.cuh"]},
     ("enc_train_d1.0", "dw"): {"bytes": 31493632, "src_sha": "5abcfcfee795d983",
-                               "files": ["sddmm_tc.cu", "common.cuh"],
-                               "profile": "profiles/k_sddmm_tc_dw_enc_train_d1.md"},
+                               "files": ["sddmm_tc.cu", "common.cuh"]},
     ("semi24_fwd", "fwd"): {"bytes": 503706112, "src_sha": "8514e1e4bf6d7d6f",
-                            "files": ["semi24.cu", "common.cuh"],
-                            "profile": "profiles/k_semi24_fwd_semi24_fwd.md"},
+                            "files": ["semi24.cu", "common.cuh"]},
     ("bsr24_fwd", "fwd"): {"bytes": 296873984, "src_sha": "ecebceabf4a22b60",
-                           "files": ["bsr24.cu", "common.cuh"],
-                           "profile": "profiles/k_bsr24_fwd_bsr24_fwd.md"},
+                           "files": ["bsr24.cu", "common.cuh"]},
 }
 # the kernel source files each contraction's traffic figure depends on
 TRAFFIC_FILES = {"fwd": ["spmm_tc.cu", "common.cuh"], "fwd_small": ["stream_fwd.cu", "common.cuh"],

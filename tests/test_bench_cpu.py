@@ -64,7 +64,7 @@ def test_traffic_entries_name_their_sources():
         assert (wname in synth.WORKLOADS or wname in synth.SEMI24_WORKLOADS or wname in synth.BSR24_WORKLOADS) \
             and kind in ("fwd", "dx", "dw")
         assert t["bytes"] > 0 and len(t["src_sha"]) == 16
-        assert os.path.exists(os.path.join(ROOT, t["profile"]))
+        assert set(t) == {"bytes", "src_sha", "files"}
         for f in t["files"]:
             assert os.path.exists(os.path.join(ROOT, "sparse_gemm_b200", "csrc", f))
 
