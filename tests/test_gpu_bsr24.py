@@ -121,3 +121,15 @@ def test_full_workload_sampled_rows():
     rows = sorted({r for t in range(0, wl.M, 224) for r in (t, min(t + 223, wl.M - 1))})
     ref, refabs = oracle.forward(X, W, mask, wl.b, rows=np.asarray(rows))
     assert_parity(to_f64(Y[rows]), ref, refabs, "2:4-block forward, full size, sampled rows")
+
+
+@pytest.mark.parametrize("b", [64, 32])
+def test_weight_without_blocks_gives_the_bias_exactly(b):
+    """Degenerate mask: no kept block, so every group is empty and the forward
+    writes the bias alone (exactly) without any MMA."""
+    M, N, K = 300, 256, 256
+    X, W, mask, bias = case(M, N, K, 1, 45, b=b)
+    mask[:] = 0
+    Wp, w24, Y = run(X, W, mask, bias, b=b)
+    assert Wp.nnz == 0
+    assert np.array_equal(bits(Y), np.broadcast_to(bias, (M, N)))

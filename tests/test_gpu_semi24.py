@@ -151,3 +151,19 @@ def test_semi24_linear_module():
     bad[0, 0:4] = [0x3F80, 0x3F80, 0x3F80, 0]
     with pytest.raises(sg.BslError, match="NOT_2_4"):
         sg.Semi24Linear.from_dense(to_dev(bad))
+
+
+def test_all_zero_weight_gives_the_bias_exactly():
+    """Degenerate weight: every group has no nonzero (kept pair (0, 1) over
+    zeros); the output is the bias alone, exactly, or exact zeros."""
+    M, N, K = 230, 264, 128
+    rng = np.random.default_rng(23)
+    W = np.zeros((N, K), dtype=np.uint16)
+    X = synth.bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    bias = synth.bf16_bits(rng.standard_normal(N).astype(np.float32))
+    w = sg.compress24(to_dev(W))
+    check_compress(W, w)
+    Y0 = sg.forward24(to_dev(X), w)
+    Yb = sg.forward24(to_dev(X), w, bias=to_dev(bias))
+    assert not Y0.float().abs().max().item()
+    assert np.array_equal(bits(Yb), np.broadcast_to(bias, (M, N)))
