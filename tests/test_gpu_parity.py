@@ -156,6 +156,7 @@ STREAM_CASES = [
     (32, 1024, 768, 64, 96, 25, ()),
     (7, 2048, 4096, 32, 1, 26, ()),           # one block: most warps idle
     (16, 4096, 4096, 32, 5000, 27, ()),       # rows cut across many warp shares
+    (9, 512, 416, 32, 30, 28, (1,)),          # K = 13 block columns, an empty block row
 ]
 
 
