@@ -19,15 +19,16 @@
 // zero block for absent members), the activation tile X[t0:t0+224, c*b:(c+1)*b]
 // and the present members' position words, all by TMA.  b = 64: 2 members,
 // two K = 32 MMAs of N = 224 per entry, 64-byte weight rows; b = 32: 4
-// members, one MMA per entry, 32-byte weight rows (32-byte swizzle).  Persistent, one CTA per SM; tiles
-// token-tile major, every group (heaviest first) inside, taken round robin.
+// members, one MMA per entry, 32-byte weight rows (32-byte swizzle).
+// Persistent, one CTA per SM; tiles token-tile major, every group (heaviest
+// first) inside, taken round robin.
 // Roles (16 warps):
 //   warp 2      plan: reads each tile's plan 32 entries at a time (lane i
 //               entry i: column, member mask, block ids by a warp prefix sum
 //               of the member counts) into a 4-chunk shared-memory ring;
 //   warps 0, 3  producers (lane 0 each, alternate stages): issue each staged
-//               entry's copies into a 5-stage ring and write the entry's
-//               member mask in the stage;
+//               entry's copies into a 5-stage (b = 64) or 8-stage (b = 32)
+//               ring and write the entry's member mask in the stage;
 //   warp 1      MMA issuer (lane 0), TMEM owner;
 //   warps 4-7   metadata: per stage, their 32 TMEM lanes' position words from
 //               shared memory into the lane layout of the sparse MMA, written
@@ -36,7 +37,8 @@
 //               chunks: TMEM -> registers (+ bias) -> bf16, transposed through
 //               a 2 KB staging chunk per warp, TMA store at the member's rows.
 // TMEM: two 128 x 224 fp32 accumulators (columns 0..447), so a tile's epilogue
-// overlaps the next tile's MMAs; the metadata ring at columns 448..511.
+// overlaps the next tile's MMAs; the metadata ring from column 448 (8 or 4
+// columns per stage for b = 64 or 32).
 // Sparse-MMA metadata layout in TMEM (measured on B200, selector 0): for rows
 // 16q .. 16q+15, lane 16q + 8kh + i holds the positions of K half kh: bits
 // 0-15 for row 16q + i, bits 16-31 for row 16q + 8 + i.
