@@ -569,7 +569,7 @@ def compress_bsr24(Wp: BsrWeight, out: Bsr24Weight | None = None) -> Bsr24Weight
 
 def forward_bsr24(X: torch.Tensor, w: Bsr24Weight, bias: torch.Tensor | None = None,
                   out: torch.Tensor | None = None) -> torch.Tensor:
-    """Y = X W^T (+ bias) for a block-sparse weight with 2:4 blocks (b = 64)."""
+    """Y = X W^T (+ bias) for a block-sparse weight with 2:4 blocks (b = 32 or 64)."""
     Wp = w.packed
     _cuda_bf16_2d(X, "X", Wp.K)
     bptr = _bias_ptr(bias, Wp.N, X)

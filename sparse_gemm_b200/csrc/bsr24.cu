@@ -195,6 +195,7 @@ __global__ void __launch_bounds__(Bsr24Cfg<B>::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
+    dependents_may_launch();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::S; ++s) {
@@ -228,6 +229,7 @@ __global__ void __launch_bounds__(Bsr24Cfg<B>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    wait_for_prior_grid();  // set-up above touched no global memory
 
     if (warp == C::W_PLAN) {
         // ------------------------------------------------------------ plan
@@ -634,8 +636,8 @@ bsl_status run_bsr24(const void *X, int32_t M, const bsl_bsr *W, const void *val
     const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (sa != BSL_OK) return sa;
     const int grid = args.tiles < num_sms() ? args.tiles : num_sms();
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ma, mx, my, reinterpret_cast<const uint8_t *>(meta24), args);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_dependent(kern, grid, C::THREADS, C::SMEM_BYTES, s, ma, mx, my,
+                                        reinterpret_cast<const uint8_t *>(meta24), args));
 }
 
 }  // namespace

@@ -26,6 +26,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Kernels launched by launch_dependent (internal.h) may start while the
+// kernel before them in the stream is finishing.  Each calls dependents_may_launch
+// at its start (the next such kernel may then be placed on SMs as they free
+// up) and wait_for_prior_grid before its first global memory access, which
+// returns once the grid before it has completed and its writes are visible:
+// the same ordering as a plain launch, with the launch and the set-up that
+// touches no global memory (barriers, TMEM, descriptor prefetch) overlapped.
+
+__device__ __forceinline__ void dependents_may_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void wait_for_prior_grid()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- smem / mbarrier
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)

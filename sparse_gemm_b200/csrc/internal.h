@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "bsl.h"
 
 namespace bsl {
@@ -48,6 +50,27 @@ public:
 private:
     int prev_ = 0;
 };
+
+// Launch a kernel that may begin while the previous kernel in the stream is
+// finishing (programmatic stream serialization).  The kernel must wait for
+// the prior grid (wait_for_prior_grid, common.cuh) before its first global
+// memory access; results and ordering are those of a plain launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                             Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and device.
 bsl_status set_smem_once(const void *func, int bytes);

@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
+    dependents_may_launch();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -166,6 +167,7 @@ __global__ void __launch_bounds__(SddmmCfg<B>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    wait_for_prior_grid();  // set-up above touched no global memory
 
     if (warp < Cfg::P) {
         // ------------------------------------------------------------ producers
@@ -358,8 +360,7 @@ bsl_status run(const CUtensorMap &dy, const CUtensorMap &x, const SddmmArgs &arg
     const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(kern), Cfg::SMEM_BYTES);
     if (sa != BSL_OK) return sa;
     const int grid = args.ntiles < num_sms() ? args.ntiles : num_sms();
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(dy, x, args);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_dependent(kern, grid, Cfg::THREADS, Cfg::SMEM_BYTES, s, dy, x, args));
 }
 
 }  // namespace

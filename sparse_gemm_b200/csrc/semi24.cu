@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(Semi24Cfg::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
+    dependents_may_launch();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::S; ++s) {
@@ -236,6 +237,7 @@ __global__ void __launch_bounds__(Semi24Cfg::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    wait_for_prior_grid();  // set-up above touched no global memory
 
     if (warp == C::W_PROD) {
         // ------------------------------------------------------------ producer
@@ -501,8 +503,7 @@ bsl_status launch_semi24_fwd(const void *X, int32_t M, const bsl_semi24 *W, cons
     const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(k_semi24_fwd), C::SMEM_BYTES);
     if (sa != BSL_OK) return sa;
     const int grid = args.tiles < num_sms() ? args.tiles : num_sms();
-    k_semi24_fwd<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ma, mx, my, args);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_dependent(k_semi24_fwd, grid, C::THREADS, C::SMEM_BYTES, s, ma, mx, my, args));
 }
 
 }  // namespace bsl

@@ -244,6 +244,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t tmo = args.timeout_ns;
+    dependents_may_launch();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::S; ++s) {
@@ -277,6 +278,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    wait_for_prior_grid();  // set-up above touched no global memory
 
     if (warp < Cfg::P) {
         // ------------------------------------------------------------ producers
@@ -769,8 +771,7 @@ bsl_status run(const CUtensorMap &a, const CUtensorMap &o, const CUtensorMap &w,
     // the work counter is zero here: the pack zeroed it and every launch,
     // one that ran out of time included, sets it back to zero at its end
     const int grid = args.units < num_sms() ? args.units : num_sms();
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, s>>>(a, o, w, args);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_dependent(kern, grid, Cfg::THREADS, Cfg::SMEM_BYTES, s, a, o, w, args));
 }
 
 }  // namespace

@@ -306,6 +306,8 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStreamWarps * (Cfg::WARP_BYTES + Cfg::OUT_BYTES)) +
                      warp * Cfg::NSLOT;
 
+    dependents_may_launch();
+    wait_for_prior_grid();  // every step below reads or writes global memory
     const int U = gridDim.x;
     const int GW = U * kStreamWarps;
     const int gw = blockIdx.x * kStreamWarps + warp;
@@ -576,8 +578,7 @@ bsl_status run(const void *X, const void *values, StreamArgs a, cudaStream_t s)
     auto kern = k_stream_fwd<B, MP>;
     const bsl_status sa = set_smem_once(reinterpret_cast<const void *>(kern), Cfg::SMEM_BYTES);
     if (sa != BSL_OK) return sa;
-    kern<<<grid, kStreamWarps * 32, Cfg::SMEM_BYTES, s>>>(mw, mx, a);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(launch_dependent(kern, grid, kStreamWarps * 32, Cfg::SMEM_BYTES, s, mw, mx, a));
 }
 
 size_t partials_bytes(int32_t M, int32_t b)
