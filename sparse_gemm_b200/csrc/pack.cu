@@ -20,9 +20,10 @@
 //                entry list of the tensor-core kernels (count pass, scan,
 //                fill pass); the kernels read the values themselves from
 //                `values` (stored once) through this list
-//   k_stream_bounds one thread per CTA of the weight-streaming forward: its
-//                first block, moved to the nearest block-row start when that
-//                is close (short rows are then never split between CTAs)
+//   k_stream_bounds one CTA: the weight-streaming forward's CTA ranges, each
+//                bound on a block-row start near its equal share (short rows
+//                are never split between CTAs), chosen to minimise the
+//                largest range
 #include "common.cuh"
 #include "internal.h"
 
@@ -284,38 +285,113 @@ void launch_group_plans(const bsl_bsr *o, cudaStream_t s)
     }
 }
 
-// Block ranges of the U CTAs of the weight-streaming forward.  CTA c starts
-// at t = floor(c * nnz / U), moved to the start of the block row holding
-// block t or of the next row, whichever is nearer, when that is at most
-// q = floor(nnz / (2U)) blocks away, so no row of up to 2q + 1 blocks is ever
-// split between CTAs.  Every bound stays within q of its equal share, and
-// equal shares are at least 2q apart, so the bounds never decrease; sb[0] = U
-// tells the kernel which grid size they were made for.
-__global__ void k_stream_bounds(const int32_t *__restrict__ row_ptr, int32_t R, int32_t nnz, int32_t U,
-                                int32_t *__restrict__ sb)
+// Block ranges of the U CTAs of the weight-streaming forward, sb[0] = U (the
+// grid size they were made for), sb[1 + c] = first block of CTA c.  Bound c
+// lies within q = floor(nnz / (2U)) blocks of its equal share
+// t = floor(c * nnz / U) (the kernel finds a block's CTA from that), on a
+// block-row start when the window [t - q, t + q] holds one, else at t; equal
+// shares are at least 2q apart, so windows are ordered and no row of up to
+// 2q + 1 blocks is ever split.  Among those choices the bounds minimise the
+// largest CTA range: the smallest L for which choosing, CTA by CTA, the
+// largest allowed bound at most L past the previous one reaches the end
+// (larger bounds only relax what follows, so that choice succeeds whenever
+// any does).  With q = 0 the bounds are the equal shares.
+
+// index of the last row start <= x among row_ptr[lo..hi], given row_ptr[lo] <= x
+// (row_ptr non-decreasing)
+__device__ int last_start_le(const int32_t *__restrict__ row_ptr, int lo, int hi, int64_t x)
 {
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c == 0) sb[0] = U;
-    if (c > U) return;
-    const int t = static_cast<int>(static_cast<int64_t>(c) * nnz / U);
-    const int q = static_cast<int>(nnz / (2LL * U));
-    int bound = t;
-    if (t > 0 && t < nnz && q > 0) {
-        int lo = 0, hi = R;  // the last row lo with row_ptr[lo] <= t (row_ptr[R] = nnz > t)
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (row_ptr[mid] <= t) lo = mid;
-            else hi = mid;
-        }
-        const int da = t - row_ptr[lo], dz = row_ptr[lo + 1] - t;
-        if (da <= dz) {
-            if (da <= q) bound = t - da;
-        } else if (dz <= q) {
-            bound = t + dz;
-        }
-        bound = min(max(bound, t - q), t + q);  // holds even if row_ptr disagrees with nnz
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(row_ptr + mid) <= x) lo = mid;
+        else hi = mid - 1;
     }
-    sb[1 + c] = bound;
+    return lo;
+}
+
+struct BoundsCtx {
+    const int32_t *row_ptr;
+    int64_t nnz, q;
+    int U;
+    const int *wlo, *whi;  // [U] row-index range of the row starts inside CTA c's window (wlo > whi: none)
+};
+
+// the largest allowed bound of CTA c that is <= x, or -1
+__device__ int64_t largest_bound(const BoundsCtx &k, int c, int64_t x)
+{
+    const int64_t t = static_cast<int64_t>(c) * k.nnz / k.U;
+    const int lo = k.wlo[c], hi = k.whi[c];
+    if (lo > hi) return t <= x ? t : -1;  // no row start in the window
+    if (__ldg(k.row_ptr + lo) > x) return -1;
+    return __ldg(k.row_ptr + last_start_le(k.row_ptr, lo, hi, x));
+}
+
+// the bounds for the largest range L (written to sb when given); false if
+// they cannot reach nnz
+__device__ bool bounds_for(const BoundsCtx &k, int64_t L, int32_t *sb)
+{
+    int64_t prev = 0;
+    if (sb) sb[1] = 0;
+    for (int c = 1; c < k.U; ++c) {
+        const int64_t v = largest_bound(k, c, prev + L);
+        if (v < prev) return false;
+        prev = v;
+        if (sb) sb[1 + c] = static_cast<int32_t>(v);
+    }
+    if (sb) sb[1 + k.U] = static_cast<int32_t>(k.nnz);
+    return k.nnz - prev <= L;
+}
+
+// One CTA (U <= 1024): each CTA's window located once, then the smallest
+// feasible L by rounds of parallel probes (each round tests evenly spaced
+// values below the smallest L known to work), then thread 0 writes the bounds.
+__global__ void __launch_bounds__(1024) k_stream_bounds(const int32_t *__restrict__ row_ptr, int32_t R,
+                                                        int32_t nnz, int32_t U, int32_t *__restrict__ sb)
+{
+    __shared__ int wlo[1024], whi[1024];
+    __shared__ unsigned long long best;
+    const int64_t q = nnz / (2LL * U);
+    if (threadIdx.x == 0) sb[0] = U;
+    if (q == 0) {
+        for (int c = threadIdx.x; c <= U; c += blockDim.x)
+            sb[1 + c] = static_cast<int32_t>(static_cast<int64_t>(c) * nnz / U);
+        return;
+    }
+    for (int c = threadIdx.x; c < U; c += blockDim.x) {
+        const int64_t t = static_cast<int64_t>(c) * nnz / U;
+        const int hi = last_start_le(row_ptr, 0, R, t + q);  // row_ptr[0] = 0 <= t + q
+        int lo = hi;  // the first start >= t - q, searched back from hi
+        if (__ldg(row_ptr + hi) < t - q) {
+            lo = hi + 1;  // none inside the window
+        } else {
+            int a = 0, b = hi;  // first index in [a, b] with row_ptr >= t - q (b qualifies)
+            while (a < b) {
+                const int mid = (a + b) >> 1;
+                if (__ldg(row_ptr + mid) >= t - q) b = mid;
+                else a = mid + 1;
+            }
+            lo = a;
+        }
+        wlo[c] = lo;
+        whi[c] = hi;
+    }
+    __syncthreads();
+    const BoundsCtx k{row_ptr, nnz, q, U, wlo, whi};
+    int64_t lo = (static_cast<int64_t>(nnz) + U - 1) / U, hi = nnz;  // hi always works; the answer is in [lo, hi]
+    while (lo < hi) {
+        const int64_t step = (hi - lo + blockDim.x - 1) / blockDim.x;
+        if (threadIdx.x == 0) best = static_cast<unsigned long long>(hi);
+        __syncthreads();
+        const int64_t L = lo + static_cast<int64_t>(threadIdx.x) * step;
+        if (L < hi && bounds_for(k, L, nullptr)) atomicMin(&best, static_cast<unsigned long long>(L));
+        __syncthreads();
+        const int64_t b = static_cast<int64_t>(best);
+        // b is the smallest working probe (or hi); the probe a step below it failed
+        lo = b - step + 1 > lo ? b - step + 1 : lo;
+        hi = b;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) bounds_for(k, lo, sb);
 }
 
 }  // namespace
@@ -351,7 +427,7 @@ bsl_status launch_pack(const void *W, const uint8_t *mask, const bsl_bsr *o, cud
     {
         const int U = num_sms();
         if (U <= BSL_SBOUNDS_LEN - 2) {
-            k_stream_bounds<<<(U + 1 + 255) / 256, 256, 0, s>>>(o->row_ptr, R, nnz, U, o->sbounds);
+            k_stream_bounds<<<1, 1024, 0, s>>>(o->row_ptr, R, nnz, U, o->sbounds);
         } else {  // no room for this grid: the kernel falls back to equal shares
             cudaMemsetAsync(o->sbounds, 0, sizeof(int32_t), s);
         }

@@ -311,6 +311,9 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
     const int U = gridDim.x;
     const int GW = U * kStreamWarps;
     const int gw = blockIdx.x * kStreamWarps + warp;
+    // whether block row gw is empty (written at the end, bias or zeros): the
+    // load leaves now rather than after the share is streamed
+    const bool gw_empty = gw < a.R && a.row_ptr[gw + 1] == a.row_ptr[gw];
     // this CTA's blocks [cq0, cq1): the pack's bounds made for this grid size
     // (the three loads go out together), else equal shares
     bool snapped = false;
@@ -557,7 +560,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 1)
 
     // block rows without blocks: bias (or zeros), rows r = gw, gw + GW, ...
     for (int r = gw; r < a.R; r += GW) {
-        if (a.row_ptr[r + 1] != a.row_ptr[r]) continue;
+        if (r == gw ? !gw_empty : a.row_ptr[r + 1] != a.row_ptr[r]) continue;
         __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(stage);
         for (int idx = lane; idx < MP * B; idx += 32)
             s[idx] = __float2bfloat16_rn(bias_of(a, static_cast<int64_t>(r) * B + (idx % B)));

@@ -9,6 +9,8 @@ group counts found by walking the columns).
 """
 from __future__ import annotations
 
+import bisect
+
 import numpy as np
 
 
@@ -54,24 +56,41 @@ def group_plan(ptr, idx, order, G: int, blk=None):
 def stream_bounds(row_ptr, U: int) -> np.ndarray:
     """CTA ranges of the weight-streaming forward, ``[U, b_0, ..., b_U]``.
 
-    CTA c starts at its equal share t = floor(c * nnz / U), moved to the start
-    of the block row holding block t or of the next row, whichever is nearer
-    (the row's own start on a tie), when that is at most q = floor(nnz / (2U))
-    blocks away; otherwise it starts at t."""
+    Bound c stays within q = floor(nnz / (2U)) blocks of its equal share
+    t = floor(c * nnz / U): on one of the block-row starts inside the window
+    [t - q, t + q] when there is any, else at t itself.  Among those choices
+    the bounds are the ones that reach the end with the smallest largest
+    range L, taking for each CTA in turn the largest allowed bound at most L
+    past the previous one.  With q = 0 the bounds are the equal shares."""
     row_ptr = [int(v) for v in row_ptr]
     nnz = row_ptr[-1]
     q = nnz // (2 * U)
-    out = [U]
-    for c in range(U + 1):
-        t = c * nnz // U
-        bound = t
-        if 0 < t < nnz and q > 0:
-            r = max(i for i in range(len(row_ptr) - 1) if row_ptr[i] <= t)  # the row holding block t
-            da, dz = t - row_ptr[r], row_ptr[r + 1] - t
-            if da <= dz:
-                if da <= q:
-                    bound = t - da
-            elif dz <= q:
-                bound = t + dz
-        out.append(bound)
-    return np.asarray(out, dtype=np.int32)
+    t = [c * nnz // U for c in range(U + 1)]
+    if q == 0:
+        return np.asarray([U] + t, dtype=np.int32)
+    inside = [sorted({v for v in row_ptr[bisect.bisect_left(row_ptr, t[c] - q):bisect.bisect_right(row_ptr, t[c] + q)]})
+              for c in range(U)]
+
+    def largest(c, x):
+        if not inside[c]:
+            return t[c] if t[c] <= x else -1
+        i = bisect.bisect_right(inside[c], x)
+        return inside[c][i - 1] if i else -1
+
+    def bounds_for(L):
+        b = [0]
+        for c in range(1, U):
+            v = largest(c, b[-1] + L)
+            if v < b[-1]:
+                return None
+            b.append(v)
+        return b + [nnz] if nnz - b[-1] <= L else None
+
+    lo, hi = -(-nnz // U), nnz  # bounds_for(nnz) always succeeds
+    while lo < hi:
+        mid = (lo + hi) // 2
+        if bounds_for(mid) is None:
+            lo = mid + 1
+        else:
+            hi = mid
+    return np.asarray([U] + bounds_for(lo), dtype=np.int32)

@@ -74,3 +74,19 @@ def test_stream_bounds_are_a_partition_that_keeps_short_rows_whole(R, C, nnz, U,
         lo, hi = int(row_ptr[r]), int(row_ptr[r + 1])
         if hi - lo <= 2 * q + 1:
             assert not np.any((b > lo) & (b < hi)), r
+    if q == 0:
+        assert np.array_equal(b, t)
+        return
+    # where the window [t - q, t + q] holds a row start the bound is one
+    for c in range(1, U):
+        if any(t[c] - q <= v <= t[c] + q for v in starts):
+            assert int(b[c]) in starts
+    # the largest range is the minimum over every allowed choice of bounds:
+    # a dynamic programme over the candidates of each bound, written here
+    cands = [[0]] + [sorted({int(v) for v in row_ptr if t[c] - q <= v <= t[c] + q} or {int(t[c])})
+                     for c in range(1, U)]
+    best = {0: 0}
+    for c in range(1, U):
+        best = {v: min(max(m, v - u) for u, m in best.items() if u <= v) for v in cands[c]}
+    optimum = min(max(m, nnz - u) for u, m in best.items())
+    assert np.diff(b).max() == optimum
