@@ -297,33 +297,34 @@ void launch_group_plans(const bsl_bsr *o, cudaStream_t s)
 // (larger bounds only relax what follows, so that choice succeeds whenever
 // any does).  With q = 0 the bounds are the equal shares.
 
-// index of the last row start <= x among row_ptr[lo..hi], given row_ptr[lo] <= x
-// (row_ptr non-decreasing)
-__device__ int last_start_le(const int32_t *__restrict__ row_ptr, int lo, int hi, int64_t x)
+// index of the last row start <= x among rp[lo..hi], given rp[lo] <= x (rp
+// non-decreasing; shared or global memory)
+__device__ int last_start_le(const int32_t *rp, int lo, int hi, int64_t x)
 {
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(row_ptr + mid) <= x) lo = mid;
+        if (rp[mid] <= x) lo = mid;
         else hi = mid - 1;
     }
     return lo;
 }
 
 struct BoundsCtx {
-    const int32_t *row_ptr;
+    const int32_t *rp;  // row_ptr (a shared-memory copy when it fits)
     int64_t nnz, q;
     int U;
     const int *wlo, *whi;  // [U] row-index range of the row starts inside CTA c's window (wlo > whi: none)
+    const int *t;          // [U] equal shares floor(c * nnz / U)
 };
 
 // the largest allowed bound of CTA c that is <= x, or -1
 __device__ int64_t largest_bound(const BoundsCtx &k, int c, int64_t x)
 {
-    const int64_t t = static_cast<int64_t>(c) * k.nnz / k.U;
+    const int64_t t = k.t[c];
     const int lo = k.wlo[c], hi = k.whi[c];
     if (lo > hi) return t <= x ? t : -1;  // no row start in the window
-    if (__ldg(k.row_ptr + lo) > x) return -1;
-    return __ldg(k.row_ptr + last_start_le(k.row_ptr, lo, hi, x));
+    if (k.rp[lo] > x) return -1;
+    return k.rp[last_start_le(k.rp, lo, hi, x)];
 }
 
 // the bounds for the largest range L (written to sb when given); false if
@@ -342,13 +343,25 @@ __device__ bool bounds_for(const BoundsCtx &k, int64_t L, int32_t *sb)
     return k.nnz - prev <= L;
 }
 
-// One CTA (U <= 1024): each CTA's window located once, then the smallest
-// feasible L by rounds of parallel probes (each round tests evenly spaced
-// values below the smallest L known to work), then thread 0 writes the bounds.
+// one allowed bound of CTA c: the window's last row start, else t (0 <= c <= U)
+__device__ int64_t some_bound(const BoundsCtx &k, int c)
+{
+    if (c == 0) return 0;
+    if (c == k.U) return k.nnz;
+    return k.wlo[c] > k.whi[c] ? k.t[c] : k.rp[k.whi[c]];
+}
+
+constexpr int kBoundsRowsInSmem = 8192;  // row_ptr entries copied to shared memory, at most
+
+// One CTA (U <= 1024): each CTA's window located once; the largest range of
+// one allowed choice is a feasible L to start from; then the smallest feasible L by
+// rounds of parallel probes (each round tests evenly spaced values below the
+// smallest L known to work), and thread 0 writes the bounds.
 __global__ void __launch_bounds__(1024) k_stream_bounds(const int32_t *__restrict__ row_ptr, int32_t R,
                                                         int32_t nnz, int32_t U, int32_t *__restrict__ sb)
 {
-    __shared__ int wlo[1024], whi[1024];
+    __shared__ int32_t srp[kBoundsRowsInSmem];
+    __shared__ int wlo[1024], whi[1024], tt[1024];
     __shared__ unsigned long long best;
     const int64_t q = nnz / (2LL * U);
     if (threadIdx.x == 0) sb[0] = U;
@@ -357,27 +370,39 @@ __global__ void __launch_bounds__(1024) k_stream_bounds(const int32_t *__restric
             sb[1 + c] = static_cast<int32_t>(static_cast<int64_t>(c) * nnz / U);
         return;
     }
+    const bool in_smem = R + 1 <= kBoundsRowsInSmem;
+    if (in_smem)
+        for (int i = threadIdx.x; i <= R; i += blockDim.x) srp[i] = row_ptr[i];
+    if (threadIdx.x == 0) best = 0;
+    __syncthreads();
+    const int32_t *rp = in_smem ? srp : row_ptr;
     for (int c = threadIdx.x; c < U; c += blockDim.x) {
         const int64_t t = static_cast<int64_t>(c) * nnz / U;
-        const int hi = last_start_le(row_ptr, 0, R, t + q);  // row_ptr[0] = 0 <= t + q
-        int lo = hi;  // the first start >= t - q, searched back from hi
-        if (__ldg(row_ptr + hi) < t - q) {
-            lo = hi + 1;  // none inside the window
-        } else {
-            int a = 0, b = hi;  // first index in [a, b] with row_ptr >= t - q (b qualifies)
+        const int hi = last_start_le(rp, 0, R, t + q);  // rp[0] = 0 <= t + q
+        int lo = hi + 1;                                // none inside the window
+        if (rp[hi] >= t - q) {
+            int a = 0, b = hi;  // the first index in [a, b] with rp >= t - q (b qualifies)
             while (a < b) {
                 const int mid = (a + b) >> 1;
-                if (__ldg(row_ptr + mid) >= t - q) b = mid;
+                if (rp[mid] >= t - q) b = mid;
                 else a = mid + 1;
             }
             lo = a;
         }
         wlo[c] = lo;
         whi[c] = hi;
+        tt[c] = static_cast<int>(t);
     }
     __syncthreads();
-    const BoundsCtx k{row_ptr, nnz, q, U, wlo, whi};
-    int64_t lo = (static_cast<int64_t>(nnz) + U - 1) / U, hi = nnz;  // hi always works; the answer is in [lo, hi]
+    const BoundsCtx k{rp, nnz, q, U, wlo, whi, tt};
+    // the largest range of one allowed choice (some_bound) is an L that works,
+    // and a close one
+    for (int c = threadIdx.x; c < U; c += blockDim.x)
+        atomicMax(&best, static_cast<unsigned long long>(some_bound(k, c + 1) - some_bound(k, c)));
+    __syncthreads();
+    int64_t lo = (static_cast<int64_t>(nnz) + U - 1) / U, hi = static_cast<int64_t>(best);
+    hi = hi < lo ? lo : (hi > nnz ? nnz : hi);
+    __syncthreads();
     while (lo < hi) {
         const int64_t step = (hi - lo + blockDim.x - 1) / blockDim.x;
         if (threadIdx.x == 0) best = static_cast<unsigned long long>(hi);
@@ -391,7 +416,10 @@ __global__ void __launch_bounds__(1024) k_stream_bounds(const int32_t *__restric
         hi = b;
         __syncthreads();
     }
-    if (threadIdx.x == 0) bounds_for(k, lo, sb);
+    if (threadIdx.x == 0 && !bounds_for(k, lo, sb)) {
+        // only with a row_ptr that is not non-decreasing: the allowed choice instead
+        for (int c = 0; c <= U; ++c) sb[1 + c] = static_cast<int32_t>(some_bound(k, c));
+    }
 }
 
 }  // namespace
