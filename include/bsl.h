@@ -117,11 +117,11 @@ typedef struct {
     int32_t *sbounds;     /* [BSL_SBOUNDS_LEN] block ranges of the weight-streaming forward's CTAs:
                            * [0] = U, the CTA count of the device bsl_pack ran on (its SM
                            * count), [1 + c] = first block of CTA c, c = 0..U ([1 + U] = nnz).
-                           * Bound c is the start of the block row holding block
-                           * floor(c * nnz / U) or of the next one, whichever is nearer, when
-                           * that is at most nnz / (2U) blocks away, else floor(c * nnz / U)
-                           * itself: block rows of up to nnz / U + 1 blocks are never split
-                           * between CTAs. */
+                           * Bound c lies within q = nnz / (2U) blocks of floor(c * nnz / U):
+                           * on a block-row start inside that window when there is one (among
+                           * those, the choice that minimises the largest CTA range), else at
+                           * floor(c * nnz / U) itself: block rows of up to 2q + 1 blocks are
+                           * never split between CTAs. */
 } bsl_bsr;
 
 /* Human-readable name of a status code (static string). */

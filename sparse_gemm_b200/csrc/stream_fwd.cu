@@ -9,9 +9,10 @@
 //
 // Decomposition: the BSR block list [0, nnz) is cut into contiguous ranges,
 // one per CTA of a one-CTA-per-SM grid: equal shares, each moved to a
-// nearby block-row start where there is one (the pack computes these
-// bounds), so block rows of up to a CTA's share never straddle two CTAs and
-// only longer ones do.  Each CTA's range is cut into equal shares for its 8
+// nearby block-row start where there is one, the starts chosen to make the
+// largest range as small as they can (the pack computes these bounds), so
+// block rows of up to a CTA's share never straddle two CTAs and only longer
+// ones do.  Each CTA's range is cut into equal shares for its 8
 // warps (block counts, not block rows, are balanced).
 // Each warp streams its share through its own ring of slots; a slot holds one
 // weight block and the activation slice X[0:MP, c*b:(c+1)*b] it multiplies,
