@@ -113,3 +113,34 @@ def test_dependent_chain_eager_and_graph(M):
         poison()
         g.replay()
         check(f"graph replay {rep}")
+
+
+@pytest.mark.parametrize("M", [16, 300])
+def test_calls_right_after_an_in_place_repack_see_the_new_weight(M):
+    """The pack's kernels write the weight and its plans; the contractions
+    launched right behind them (no synchronisation) must read what they
+    wrote, not the previous pattern."""
+    X0, W1, m1, b1, _, _, _ = make_chain(M, 80 + M)
+    rng = np.random.default_rng(90 + M)
+    m2 = synth.mask_uniform(N // B, K // B, NNZ, rng)  # same block count, new pattern
+    assert not np.array_equal(m1, m2)
+    W2 = synth.bf16_bits(rng.integers(-1, 2, size=(N, K)).astype(np.float32))
+    dY = synth.bf16_bits(rng.integers(-1, 2, size=(M, N)).astype(np.float32))
+    want_y = exact_bf16(oracle.forward(X0, W2, m2, B, bias=b1)[0])
+    want_dx = exact_bf16(oracle.backward_input(dY, W2, m2, B)[0])
+    want_dw = exact_bf16(oracle.backward_weight(dY, X0, m2, B)[0])
+
+    Wp = sg.pack(to_dev(W1), mask_dev(m1), B)
+    Xd, bd, dYd = to_dev(X0), to_dev(b1), to_dev(dY)
+    sg.forward(Xd, Wp, bias=bd)  # the old pattern is in use just before the re-pack
+    W2d, m2d = to_dev(W2), mask_dev(m2)
+    torch.cuda.synchronize()
+    Wp.repack(W2d, m2d)
+    Y = sg.forward(Xd, Wp, bias=bd)
+    dX = sg.backward_input(dYd, Wp)
+    dW = sg.backward_weight(dYd, Xd, Wp)
+    torch.cuda.synchronize()
+    assert sg.device_status(Wp) == 0
+    assert np.array_equal(bits(Y), want_y)
+    assert np.array_equal(bits(dX), want_dx)
+    assert np.array_equal(bits(dW).reshape(want_dw.shape), want_dw)

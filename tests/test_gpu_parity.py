@@ -209,6 +209,28 @@ def test_forward_stream_rows_across_many_ctas(case_args, with_bias):
     assert_parity(got, ref, S, "forward_stream" + (" + bias" if with_bias else ""))
 
 
+def test_stream_bounds_with_more_block_rows_than_fit_in_shared_memory():
+    """8400 block rows: the pack's bound search reads row_ptr from global
+    memory instead of its shared-memory copy (8192 entries); the bounds must
+    still equal the host model's and the forward the oracle's."""
+    M, R, C, b = 16, 8400, 4, 32
+    rng = np.random.default_rng(47)
+    mask = (rng.random((R, C)) < 0.5).astype(np.uint8)
+    mask[rng.integers(0, R, size=40), :] = 1  # some full rows
+    mask[rng.integers(0, R, size=40), :] = 0  # some empty rows
+    W = synth.bf16_bits((rng.standard_normal((R * b, C * b)) / np.sqrt(C * b)).astype(np.float32))
+    X = synth.bf16_bits(rng.standard_normal((M, C * b)).astype(np.float32))
+    Wp = sg.pack(to_dev(W), mask_dev(mask), b)
+    row_ptr = np.concatenate([[0], np.cumsum(mask.sum(axis=1))]).astype(np.int64)
+    assert np.array_equal(Wp.row_ptr.cpu().numpy(), row_ptr)
+    U = torch.cuda.get_device_properties(Wp.values.device).multi_processor_count
+    assert np.array_equal(Wp.sbounds[:U + 2].cpu().numpy(), _plan.stream_bounds(row_ptr, U))
+    got = to_f64(sg.forward_stream(to_dev(X), Wp))
+    assert sg.device_status(Wp) == 0
+    ref, S = oracle.forward(X, W, mask, b)
+    assert_parity(got, ref, S, "forward_stream, 8400 block rows")
+
+
 def test_forward_stream_replayed_from_a_cuda_graph():
     # every call leaves the cross-CTA counters at zero, so every replay of a
     # captured call finds them fresh (a row whose count were carried over
