@@ -60,6 +60,9 @@
 // first takes the remaining units, so every launch leaves the counter at zero
 // and no memset precedes the kernel; two launches of the same contraction on
 // one weight must not run at the same time (they would share the counter).
+// A launch with no more units than CTAs (one unit each) leaves the counter
+// alone: CTA i does unit i, with no atomic round trip before its first plan
+// load.
 //
 // Roles per CTA (persistent grid, one CTA per SM):
 //   warps 0..P-1   producers: TMA tile copies of the activation tile and of
@@ -539,6 +542,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
         // new unit is taken only once a chunk slot is free, so the CTA holds at
         // most one unit beyond the one its producers are issuing.
         bool ok = true, drained = false;  // drained: this CTA's take past the last unit is done
+        const bool fixed = args.units <= static_cast<int>(gridDim.x);
         int cc = 0;                       // chunks staged
         for (int j = 0; ok; ++j) {
             int good = 1;
@@ -550,7 +554,9 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
             }
             int ord = -1;
             if (lane == 0) {
-                ord = take_unit(args.sched, args.units);
+                // no more units than CTAs: CTA i does unit i and the counter is not used
+                if (fixed) ord = j == 0 ? static_cast<int>(blockIdx.x) : -1;
+                else ord = take_unit(args.sched, args.units);
                 drained = ord < 0;
             }
             ord = __shfl_sync(0xffffffffu, ord, 0);
@@ -638,7 +644,7 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
             set_status(args.status, BSL_ERR_TIMEOUT);
             // take the remaining units too (they are left undone: the status
             // reports the timeout), so that the counter still returns to zero
-            if (!drained)
+            if (!drained && !fixed)
                 while (take_unit(args.sched, args.units) >= 0) {
                 }
         }
