@@ -60,9 +60,8 @@
 // first takes the remaining units, so every launch leaves the counter at zero
 // and no memset precedes the kernel; two launches of the same contraction on
 // one weight must not run at the same time (they would share the counter).
-// A launch with no more units than CTAs (one unit each) leaves the counter
-// alone: CTA i does unit i, with no atomic round trip before its first plan
-// load.
+// CTA i's first unit is unit i, with no atomic round trip before its first
+// plan load; a launch with no more units than CTAs leaves the counter alone.
 //
 // Roles per CTA (persistent grid, one CTA per SM):
 //   warps 0..P-1   producers: TMA tile copies of the activation tile and of
@@ -168,14 +167,16 @@ __device__ __forceinline__ void decode_unit(const SpmmArgs &a, int ord, int *mt,
     *mt = mt0 + (r - *g * nmt);
 }
 
-// Take the next unit from the per-weight counter (-1: none left).  Every CTA
-// ends with exactly one take past the last unit; the take that returns
-// units + gridDim.x - 1 is the last take of the launch, so that CTA sets the
-// counter back to zero for the next launch (stream order makes the store
-// visible to it).
+// Take the next unit from the per-weight counter (-1: none left).  Units
+// 0 .. gridDim.x - 1 are the CTAs' first units, taken without the counter,
+// so the counter hands out units from gridDim.x on.  Every CTA ends with
+// exactly one take past the last unit: units atomic takes in all, and the
+// one that finds units - 1 (unit units + gridDim.x - 1) is the last of the
+// launch, so that CTA sets the counter back to zero for the next launch
+// (stream order makes the store visible to it).
 __device__ __forceinline__ int take_unit(int32_t *sched, int units)
 {
-    const int ord = atomicAdd(sched, 1);
+    const int ord = atomicAdd(sched, 1) + static_cast<int>(gridDim.x);
     if (ord < units) return ord;
     if (ord == units + static_cast<int>(gridDim.x) - 1) *reinterpret_cast<volatile int32_t *>(sched) = 0;
     return -1;
@@ -554,9 +555,10 @@ __global__ void __launch_bounds__(SpmmCfg<B>::THREADS, 1)
             }
             int ord = -1;
             if (lane == 0) {
-                // no more units than CTAs: CTA i does unit i and the counter is not used
-                if (fixed) ord = j == 0 ? static_cast<int>(blockIdx.x) : -1;
-                else ord = take_unit(args.sched, args.units);
+                // every CTA's first unit is unit blockIdx.x (grid <= units); the
+                // counter hands out the rest, and is not used when there is no rest
+                if (j == 0) ord = static_cast<int>(blockIdx.x);
+                else ord = fixed ? -1 : take_unit(args.sched, args.units);
                 drained = ord < 0;
             }
             ord = __shfl_sync(0xffffffffu, ord, 0);
