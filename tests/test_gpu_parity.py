@@ -339,6 +339,33 @@ def test_results_are_deterministic():
         assert torch.equal(u.view(torch.int16), v.view(torch.int16))
 
 
+def test_work_counters_with_more_units_than_ctas():
+    """More units than CTAs: each CTA's first unit is its own index and the
+    counter hands out the rest; after every launch (forward and dX, several
+    M) the counters are back at zero and repeated results are bit-identical."""
+    case = synth.random_case(5000, 2048, 1024, 64, 300, 48)
+    Wp = pack_dev(case, 64)
+    X, dY = to_dev(case["X"]), to_dev(case["dY"])
+    ncta = torch.cuda.get_device_properties(X.device).multi_processor_count
+    assert (2048 // 128) * ((5000 + 255) // 256) > ncta  # forward units
+    assert (1024 // 128) * ((5000 + 255) // 256) > ncta  # dX units
+    first = None
+    for M in (5000, 4500, 5000):
+        y = sg.forward_tc(X[:M].contiguous(), Wp)
+        dx = sg.backward_input(dY[:M].contiguous(), Wp)
+        torch.cuda.synchronize()
+        assert int(Wp.sched.abs().sum()) == 0, M
+        assert sg.device_status(Wp) == 0
+        if M == 5000:
+            if first is None:
+                first = (y, dx)
+                ref, S = oracle.forward(case["X"], case["W"], case["mask"], 64, rows=np.arange(0, 5000, 97))
+                assert_parity(to_f64(y[::97]), ref, S, "forward, more units than CTAs")
+            else:
+                assert torch.equal(y.view(torch.int16), first[0].view(torch.int16))
+                assert torch.equal(dx.view(torch.int16), first[1].view(torch.int16))
+
+
 def test_work_counters_return_to_zero_after_every_launch():
     """The persistent kernels take units from counters in the packed weight,
     and the small-M forward counts CTAs in on rows they share in its
